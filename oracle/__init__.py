@@ -1,0 +1,126 @@
+"""fp64 CPU oracle for the DCNv4 forward spatial aggregation.
+
+TEST INFRASTRUCTURE ONLY: the tests, the smoke check and the CPU-baseline leg
+of the benchmark may import this package; the product path (the CUDA library
+and its Python binding) never does. The arithmetic lives in ``dcnv4_oracle.c``
+(plain C, fp64), compiled here with gcc into ``liboracle.so`` and called
+through ctypes with numpy arrays. It shares no code with the CUDA path.
+
+Definition followed: "不只是卷积的平替：我把DCNv4塞进Stable Diffusion的U-Net里"
+(jsqmd.com), section 1 (no softmax over the modulation scalars; the simplified
+forward listing: regular grid + offsets, bilinear sampling, mask-weighted sum
+over the K*K points per group) and "掌握DCNv4技术" (pwwt.cn), tuning section
+(offset_scale scales the offsets). The readings taken where the pages are
+silent are stated at the top of ``dcnv4_oracle.c``.
+
+Every function here is pinned by tests that do not reuse its code (identity,
+integer-offset brute force, torch ``grid_sample``, hand-expanded cases in
+``tests/golden/``, linearity, out-of-bounds, partition of unity, group
+equivalence, translation equivariance).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "dcnv4_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile ``dcnv4_oracle.c`` into ``liboracle.so`` (gcc, no fused multiply-add)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + ".tmp.%d" % os.getpid()
+        subprocess.check_call(["gcc", "-O2", "-std=c99", "-ffp-contract=off", "-fno-fast-math",
+                               "-shared", "-fPIC", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        i, f, p = ctypes.c_int, ctypes.c_float, ctypes.c_void_p
+        lib.oracle_output_size.argtypes = [i, i, i, i, i]
+        lib.oracle_output_size.restype = i
+        lib.oracle_dcnv4_forward.argtypes = [p, p, p] + [i] * 9 + [f]
+        lib.oracle_dcnv4_forward.restype = i
+        lib.oracle_dcnv4_forward_images.argtypes = [p, p, p] + [i] * 9 + [f, i, i]
+        lib.oracle_dcnv4_forward_images.restype = i
+        lib.oracle_dcnv4_sampling_index.argtypes = [p, p, p] + [i] * 8 + [f]
+        lib.oracle_dcnv4_sampling_index.restype = i
+        _lib = lib
+    return _lib
+
+
+def output_size(size: int, K: int, stride: int = 1, pad: int = 0, dilation: int = 1) -> int:
+    """Output extent along one axis, convolution style (<= 0 when empty)."""
+    return _load().oracle_output_size(size, K, stride, pad, dilation)
+
+
+def _f64(a) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def dcnv4_forward(x, offset_mask, G: int, K: int, stride: int = 1, pad: int = 0,
+                  dilation: int = 1, offset_scale: float = 1.0,
+                  n_begin: int | None = None, n_end: int | None = None) -> np.ndarray:
+    """fp64 forward. ``x``: [N,H,W,C]; ``offset_mask``: [N,Hout,Wout,G,3*K*K].
+
+    Returns out [N,Hout,Wout,C] (fp64). With ``n_begin``/``n_end`` only those
+    images are computed (the rest of the result stays zero).
+    """
+    x = _f64(x)
+    om = _f64(offset_mask)
+    N, H, W, C = x.shape
+    Hout, Wout = output_size(H, K, stride, pad, dilation), output_size(W, K, stride, pad, dilation)
+    if om.shape != (N, Hout, Wout, G, 3 * K * K):
+        raise ValueError(f"offset_mask shape {om.shape} != {(N, Hout, Wout, G, 3 * K * K)}")
+    out = np.zeros((N, Hout, Wout, C), dtype=np.float64)
+    if N == 0:
+        return out
+    lib = _load()
+    if n_begin is None and n_end is None:
+        rc = lib.oracle_dcnv4_forward(_ptr(x), _ptr(om), _ptr(out), N, H, W, C, G, K,
+                                      stride, pad, dilation, float(offset_scale))
+    else:
+        rc = lib.oracle_dcnv4_forward_images(_ptr(x), _ptr(om), _ptr(out), N, H, W, C, G, K,
+                                             stride, pad, dilation, float(offset_scale),
+                                             0 if n_begin is None else n_begin,
+                                             N if n_end is None else n_end)
+    if rc != 0:
+        raise ValueError("oracle rejected the arguments")
+    return out
+
+
+def sampling_index(offset_mask, H: int, W: int, G: int, K: int, stride: int = 1, pad: int = 0,
+                   dilation: int = 1, offset_scale: float = 1.0):
+    """Integer corner (y0, x0) [..., K*K, 2] int32 and 4-bit validity [..., K*K] uint8.
+
+    Bit 2*a+b of the validity byte is set when corner (y0+a, x0+b) is inside the
+    image; samples with no corner inside report (INT32_MIN, INT32_MIN).
+    """
+    om = _f64(offset_mask)
+    N, Hout, Wout, G_, R = om.shape
+    if G_ != G or R != 3 * K * K:
+        raise ValueError("offset_mask shape does not match G, K")
+    if (Hout, Wout) != (output_size(H, K, stride, pad, dilation), output_size(W, K, stride, pad, dilation)):
+        raise ValueError("offset_mask spatial shape does not match the output size")
+    corner = np.zeros((N, Hout, Wout, G, K * K, 2), dtype=np.int32)
+    valid = np.zeros((N, Hout, Wout, G, K * K), dtype=np.uint8)
+    if N:
+        rc = _load().oracle_dcnv4_sampling_index(_ptr(om), _ptr(corner), _ptr(valid), N, H, W, G, K,
+                                                 stride, pad, dilation, float(offset_scale))
+        if rc != 0:
+            raise ValueError("oracle rejected the arguments")
+    return corner, valid

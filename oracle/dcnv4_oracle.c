@@ -1,0 +1,193 @@
+/*
+ * DCNv4 forward spatial aggregation -- plain fp64 CPU oracle.
+ *
+ * TEST INFRASTRUCTURE ONLY. Nothing on the product path may include, link or
+ * call this file; it exists so that the tests, the smoke check and the CPU
+ * baseline of the benchmark have an obviously correct, independent statement
+ * of what the operator computes. It shares no code, header, table or helper
+ * with the CUDA library.
+ *
+ * What it computes (sources, by page title and section):
+ *  - "不只是卷积的平替：我把DCNv4塞进Stable Diffusion的U-Net里" (jsqmd.com),
+ *    section 1: the softmax over the aggregation weights is removed, so the
+ *    modulation scalars are used raw and may be negative or exceed 1; the
+ *    simplified forward listing of the same section adds learned offsets,
+ *    reshaped as (N, G, 2, K*K, H, W), to a regular K x K grid, bilinearly
+ *    samples the input there, weights every sample by its mask value and sums
+ *    over the K*K axis, group by group.
+ *  - "掌握DCNv4技术：3倍速度提升与80%加速效果的实战指南" (pwwt.cn), tuning
+ *    section: offset_scale multiplies the offsets.
+ *  - Operator contract of this library: channels-last x[N,H,W,C], packed
+ *    offset_mask[N,Hout,Wout,G,3*K*K] with, per group, 2*K*K offsets then
+ *    K*K masks, zero padding outside the image, out[N,Hout,Wout,C].
+ *
+ * Readings taken where the pages are silent (each is also listed in the
+ * design notes):
+ *  - grid point order is row-major, k = ky*K + kx;
+ *  - the grid is convolution style: p0 = o*stride - pad + kk*dilation;
+ *  - offsets are component-major inside the 2*K*K block: r[k] moves along
+ *    the width (x), r[K*K + k] along the height (y); masks are r[2*K*K + k];
+ *  - the scaled offset is one fp32 multiply, fl32(offset_scale * r), which is
+ *    exact when offset_scale == 1; the sample position is p0 + that value;
+ *  - zero padding is per corner: corners outside the image contribute 0,
+ *    corners inside always contribute (even with weight 0); a non-finite
+ *    offset puts the whole sample outside;
+ *  - offsets are in pixels.
+ *
+ * Precision: inputs arrive as fp64 copies of the (already rounded) storage
+ * values; everything else is fp64 except the single fp32 offset multiply.
+ * Compile with -ffp-contract=off so that no multiply-add is fused.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stddef.h>
+
+/* Output extent of one spatial axis, convolution style. Returns <= 0 when no
+ * output position exists. */
+int oracle_output_size(int in, int K, int stride, int pad, int dilation)
+{
+    long span = (long)in + 2L * pad - (long)dilation * (K - 1) - 1;
+    if (stride <= 0 || span < 0) return 0;
+    return (int)(span / stride + 1);
+}
+
+/* The scaled offset: fl32(offset_scale * r). r holds a value that is exactly
+ * representable in fp32 (it came from fp32, fp16 or bf16 storage). */
+static double scaled_offset(float offset_scale, double r)
+{
+    volatile float prod = offset_scale * (float)r; /* one fp32 rounding */
+    return (double)prod;
+}
+
+/* One output element group: out[n, ho, wo, g*Cg : (g+1)*Cg].
+ * Sums over the K*K grid points of group g the bilinear sample of x at
+ * p0 + offset, weighted by the raw mask value. */
+static void aggregate_one(const double *x, const double *om, double *out,
+                          int N, int H, int W, int C, int G, int K,
+                          int stride, int pad, int dilation, float offset_scale,
+                          int Hout, int Wout, int n, int ho, int wo, int g)
+{
+    const int Cg = C / G;
+    const int KK = K * K;
+    const double *r = om + ((((size_t)n * Hout + ho) * Wout + wo) * G + g) * (size_t)(3 * KK);
+    double *o = out + (((size_t)n * Hout + ho) * Wout + wo) * (size_t)C + (size_t)g * Cg;
+    (void)N;
+
+    for (int c = 0; c < Cg; ++c) o[c] = 0.0;
+
+    for (int k = 0; k < KK; ++k) {
+        const int ky = k / K, kx = k % K;
+        const int p0y = ho * stride - pad + ky * dilation;
+        const int p0x = wo * stride - pad + kx * dilation;
+        const double dx = scaled_offset(offset_scale, r[k]);
+        const double dy = scaled_offset(offset_scale, r[KK + k]);
+        const double m = r[2 * KK + k];
+        if (!isfinite(dx) || !isfinite(dy)) continue; /* outside the image */
+
+        /* sample position (p0y + dy, p0x + dx); its top-left corner and the
+         * fractional part, without rounding p0 + d */
+        const double fy0 = floor(dy), fx0 = floor(dx);
+        const double ly = dy - fy0, lx = dx - fx0;
+        const double y0 = (double)p0y + fy0, x0 = (double)p0x + fx0;
+
+        for (int a = 0; a <= 1; ++a) {
+            for (int b = 0; b <= 1; ++b) {
+                const double yy = y0 + a, xx = x0 + b;
+                if (!(yy >= 0.0 && yy <= (double)(H - 1) && xx >= 0.0 && xx <= (double)(W - 1)))
+                    continue; /* zero padding */
+                const double wy = a ? ly : 1.0 - ly;
+                const double wx = b ? lx : 1.0 - lx;
+                const double w = m * wy * wx;
+                const double *px = x + ((((size_t)n * H + (size_t)yy) * W + (size_t)xx) * C) + (size_t)g * Cg;
+                for (int c = 0; c < Cg; ++c) o[c] += w * px[c];
+            }
+        }
+    }
+}
+
+/* Full forward. x: [N,H,W,C]; om: [N,Hout,Wout,G,3*K*K]; out: [N,Hout,Wout,C].
+ * All fp64, contiguous. Returns 0, or -1 on inconsistent arguments. */
+int oracle_dcnv4_forward(const double *x, const double *om, double *out,
+                         int N, int H, int W, int C, int G, int K,
+                         int stride, int pad, int dilation, float offset_scale)
+{
+    if (N < 0 || H <= 0 || W <= 0 || C <= 0 || G <= 0 || K <= 0 || C % G) return -1;
+    const int Hout = oracle_output_size(H, K, stride, pad, dilation);
+    const int Wout = oracle_output_size(W, K, stride, pad, dilation);
+    if (Hout <= 0 || Wout <= 0) return -1;
+    for (int n = 0; n < N; ++n)
+        for (int ho = 0; ho < Hout; ++ho)
+            for (int wo = 0; wo < Wout; ++wo)
+                for (int g = 0; g < G; ++g)
+                    aggregate_one(x, om, out, N, H, W, C, G, K, stride, pad, dilation,
+                                  offset_scale, Hout, Wout, n, ho, wo, g);
+    return 0;
+}
+
+/* Same as oracle_dcnv4_forward restricted to images [n_begin, n_end): used to
+ * time a bounded sample of a large workload. Pointers address the full
+ * tensors. */
+int oracle_dcnv4_forward_images(const double *x, const double *om, double *out,
+                                int N, int H, int W, int C, int G, int K,
+                                int stride, int pad, int dilation, float offset_scale,
+                                int n_begin, int n_end)
+{
+    if (n_begin < 0 || n_end > N || n_begin > n_end || C % G) return -1;
+    const int Hout = oracle_output_size(H, K, stride, pad, dilation);
+    const int Wout = oracle_output_size(W, K, stride, pad, dilation);
+    if (Hout <= 0 || Wout <= 0) return -1;
+    for (int n = n_begin; n < n_end; ++n)
+        for (int ho = 0; ho < Hout; ++ho)
+            for (int wo = 0; wo < Wout; ++wo)
+                for (int g = 0; g < G; ++g)
+                    aggregate_one(x, om, out, N, H, W, C, G, K, stride, pad, dilation,
+                                  offset_scale, Hout, Wout, n, ho, wo, g);
+    return 0;
+}
+
+/* Integer part of every sample: the top-left corner (y0, x0) and a 4-bit mask
+ * of the corners that lie inside the image (bit 0: (y0,x0), bit 1: (y0,x0+1),
+ * bit 2: (y0+1,x0), bit 3: (y0+1,x0+1)).
+ * corner: [N,Hout,Wout,G,K*K,2] int32 (y0 then x0); valid: [N,Hout,Wout,G,K*K].
+ * A sample with no corner inside reports corner = (INT32_MIN, INT32_MIN). */
+int oracle_dcnv4_sampling_index(const double *om, int32_t *corner, uint8_t *valid,
+                                int N, int H, int W, int G, int K,
+                                int stride, int pad, int dilation, float offset_scale)
+{
+    const int Hout = oracle_output_size(H, K, stride, pad, dilation);
+    const int Wout = oracle_output_size(W, K, stride, pad, dilation);
+    if (Hout <= 0 || Wout <= 0 || G <= 0 || K <= 0) return -1;
+    const int KK = K * K;
+    for (int n = 0; n < N; ++n)
+        for (int ho = 0; ho < Hout; ++ho)
+            for (int wo = 0; wo < Wout; ++wo)
+                for (int g = 0; g < G; ++g) {
+                    const size_t unit = (((size_t)n * Hout + ho) * Wout + wo) * G + g;
+                    const double *r = om + unit * (size_t)(3 * KK);
+                    for (int k = 0; k < KK; ++k) {
+                        const int ky = k / K, kx = k % K;
+                        const int p0y = ho * stride - pad + ky * dilation;
+                        const int p0x = wo * stride - pad + kx * dilation;
+                        const double dx = scaled_offset(offset_scale, r[k]);
+                        const double dy = scaled_offset(offset_scale, r[KK + k]);
+                        unsigned bits = 0;
+                        double y0 = 0, x0 = 0;
+                        if (isfinite(dx) && isfinite(dy)) {
+                            y0 = (double)p0y + floor(dy);
+                            x0 = (double)p0x + floor(dx);
+                            for (int a = 0; a <= 1; ++a)
+                                for (int b = 0; b <= 1; ++b) {
+                                    const double yy = y0 + a, xx = x0 + b;
+                                    if (yy >= 0.0 && yy <= (double)(H - 1) &&
+                                        xx >= 0.0 && xx <= (double)(W - 1))
+                                        bits |= 1u << (2 * a + b);
+                                }
+                        }
+                        const size_t p = unit * KK + k;
+                        valid[p] = (uint8_t)bits;
+                        corner[2 * p + 0] = bits ? (int32_t)y0 : INT32_MIN;
+                        corner[2 * p + 1] = bits ? (int32_t)x0 : INT32_MIN;
+                    }
+                }
+    return 0;
+}
