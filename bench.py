@@ -1,0 +1,358 @@
+#!/usr/bin/env python
+"""Throughput benchmark of the DCNv4 forward spatial aggregation on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    torchrun --nproc-per-node N bench.py --gpus N ...     (one rank per GPU)
+
+A step is one dcnv4_forward call over one batch of the FlashInternImage-T
+stage-1 shaped workload (N=64, 56x56, C=64, G=4, K=3, fp16 storage, fp32
+arithmetic; seeded synthetic inputs). With N GPUs every rank processes its own
+batch of 64 images (weak scaling, no collective on the data path).
+
+Timing: W untimed warm-up steps, a ~1 s untimed soak (clocks settle and are
+sampled), then exactly K steps between CUDA events on the launching stream,
+bracketed by a barrier and a device synchronise; the time is the max over
+ranks. The steps rotate over several resident copies of the inputs whose total
+exceeds the L2 cache, so no step starts with its inputs in L2.
+
+--impl reference times the fp64 CPU oracle (the reference arm of this
+repository: there is no other implementation to install) on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import glob
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "DCNv4 fwd sampling points/s (G/s); achieved HBM GB/s as % of B200 peak"
+UNIT = "Gpoints/s"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=None, help="named workload (default: the stage-1 fp16 batch)")
+    ap.add_argument("--soak-s", type=float, default=1.0)
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_sources_sha() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "deformable_convolution_sparse_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(csrc, f), "rb") as fh:
+                h.update(f.encode() + b"\0" + fh.read())
+    return h.hexdigest()
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on the current kernel sources."""
+    sha = kernel_sources_sha()
+    for path in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md"))):
+        fields = {}
+        with open(path) as f:
+            for line in f:
+                if ":" in line and line.startswith("- "):
+                    k, v = line[2:].split(":", 1)
+                    fields[k.strip()] = v.strip().strip("`")
+        if fields.get("workload") == workload and fields.get("kernel_sources_sha256") == sha \
+                and "dram_bytes_per_launch" in fields:
+            return int(float(fields["dram_bytes_per_launch"])), os.path.relpath(path, ROOT)
+    return None, None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the GPU is under load."""
+    Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_uuid: str):
+        self.uuid = gpu_uuid
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", self.uuid, f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in self.lines:
+            parts = [p.strip() for p in l.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def cpu_baseline(w, x, om):
+    """The fp64 oracle, as it stands, on the whole batch (single thread)."""
+    import oracle
+    xd, omd = x.double().numpy(), om.double().numpy()
+    oracle.dcnv4_forward(xd, omd, **w.kwargs(), n_begin=0, n_end=1)  # load + warm
+    t0 = time.perf_counter()
+    oracle.dcnv4_forward(xd, omd, **w.kwargs())
+    dt = time.perf_counter() - t0
+    return {"value": w.points / dt / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "seconds": dt, "sample": f"the whole {w.name} batch ({w.N} images, {w.points} points), "
+                                    "fp64 C oracle, one thread"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from deformable_convolution_sparse_b200.workloads import BENCH_WORKLOAD, WORKLOADS, workload_inputs
+    import oracle
+    w = WORKLOADS[args.workload or BENCH_WORKLOAD]
+    x, om = workload_inputs(w)
+    xd, omd = x.double().numpy(), om.double().numpy()
+    n_s = max(1, min(w.N, 8))  # images per step: a bounded sample (~0.1 s of CPU work each)
+    pts = w.points // w.N * n_s
+    for _ in range(args.warmup):
+        oracle.dcnv4_forward(xd, omd, **w.kwargs(), n_begin=0, n_end=n_s)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        b = (i * n_s) % (w.N - n_s + 1)
+        oracle.dcnv4_forward(xd, omd, **w.kwargs(), n_begin=b, n_end=b + n_s)
+    dt = time.perf_counter() - t0
+    value = pts * args.steps / dt / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{w.name}: N={w.N} H=W={w.H} C={w.C} G={w.G} K={w.K} pad={w.pad} "
+                               f"dilation={w.dilation}, {w.dtype} storage", "sample_images_per_step": n_s},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": f"{n_s} of {w.N} images per step, fp64 C oracle, one thread"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    import deformable_convolution_sparse_b200 as dcn
+    from deformable_convolution_sparse_b200.workloads import BENCH_WORKLOAD, WORKLOADS, workload_inputs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v: float) -> float:
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    w = WORKLOADS[args.workload or BENCH_WORKLOAD]
+    # weak scaling: rank r owns images [64 r, 64 (r+1)) of the global batch, drawn from seed + r
+    wr = w.with_(seed=w.seed + 1000 * rank)
+    x, om = workload_inputs(wr)
+    lib = dcn.load_library()
+    dtype_code = dcn.binding.TORCH_DTYPE[x.dtype]
+
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    foot = w.algorithmic_bytes()
+    copies = max(3, math.ceil(3 * l2 / foot))
+    xs = [x.to(dev) for _ in range(copies)]
+    oms = [om.to(dev) for _ in range(copies)]
+    outs = [torch.empty((w.N, w.Hout, w.Wout, w.C), dtype=x.dtype, device=dev) for _ in range(copies)]
+    stream = torch.cuda.current_stream(dev)
+    sh = stream.cuda_stream
+    launches = [0]
+
+    def step(i):
+        j = i % copies
+        rc = lib.dcnv4_forward(xs[j].data_ptr(), oms[j].data_ptr(), outs[j].data_ptr(), w.N, w.H, w.W, w.C, w.G,
+                               w.K, w.stride, w.pad, w.dilation, w.offset_scale, dtype_code, sh)
+        if rc != 0:
+            raise dcn.DCNv4Error(rc, "dcnv4_forward")
+        launches[0] += 1
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+
+    uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    sampler = ClockSampler(uuid)
+    sampler.start()
+    t_end = time.perf_counter() + args.soak_s
+    i = 0
+    while time.perf_counter() < t_end:
+        for _ in range(200):
+            step(i)
+            i += 1
+        torch.cuda.synchronize(dev)
+
+    barrier()
+    torch.cuda.synchronize(dev)
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    launches[0] = 0
+    ev0.record(stream)
+    for i in range(args.steps):
+        step(i)
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    sampler.stop()
+    timed_launches = launches[0]
+    ms = max_over_ranks(ev0.elapsed_time(ev1))
+    ms_step = ms / args.steps
+    total_points = w.points * world * args.steps
+    value = total_points / (ms / 1e3) / 1e9
+
+    # roofline of the (only) kernel: algorithmic bytes per launch / average launch duration
+    peak, peak_kind = measured_peaks()
+    achieved = foot / (ms_step / 1e3) / 1e9
+    traffic, traffic_src = profiled_traffic(w.name)
+
+    # end to end: host buffers in, result back to the host, through dcnv4_forward_host
+    xh, omh = x.pin_memory(), om.pin_memory()
+    oh = torch.empty((w.N, w.Hout, w.Wout, w.C), dtype=x.dtype).pin_memory()
+    xd, omd, od = xs[0], oms[0], outs[0]
+
+    def e2e_step():
+        rc = lib.dcnv4_forward_host(xh.data_ptr(), omh.data_ptr(), oh.data_ptr(), xd.data_ptr(), omd.data_ptr(),
+                                    od.data_ptr(), w.N, w.H, w.W, w.C, w.G, w.K, w.stride, w.pad, w.dilation,
+                                    w.offset_scale, dtype_code, sh)
+        if rc != 0:
+            raise dcn.DCNv4Error(rc, "dcnv4_forward_host")
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1))
+    e2e_value = w.points * world * args.e2e_steps / (e2e_ms / 1e3) / 1e9
+    # the result came back through the host path: it must equal the device path bit for bit
+    if not torch.equal(oh, outs[0].cpu()):
+        raise SystemExit("end-to-end result differs from the device-resident result")
+
+    base = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        base = cpu_baseline(w, x, om)
+
+    clocks = sampler.summary()
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {
+                "workload": f"{w.name}: FlashInternImage-T stage-1 shaped DCNv4 forward, N={w.N} per GPU, "
+                            f"H=W={w.H}, C={w.C}, G={w.G} (C/G={w.Cg}), K={w.K}, stride={w.stride}, pad={w.pad}, "
+                            f"dilation={w.dilation}, offset_scale={w.offset_scale}",
+                "storage_dtype": w.dtype, "accumulate": "f32", "global_batch": w.N * world,
+                "points_per_step_per_gpu": w.points, "parallelism": f"dp{world} (independent batches)",
+                "l2": f"steps rotate over {copies} resident input/output sets, {copies * foot / 1e6:.0f} MB "
+                      f"in total vs {l2 / 1e6:.0f} MB L2",
+                "inputs": "seeded synthetic: x~N(0,1), offsets~N(0,1.5^2), masks~N(0,0.5^2)",
+            },
+            "hbm_gbs": achieved,
+            "hbm_pct_of_peak": 100.0 * achieved / peak,
+            "hbm_pct_of_8tbs_nominal": 100.0 * achieved / 8000.0,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json)"
+                         if peak_kind == "measured" else "fallback 6.65 TB/s",
+                         "kernel": "dcnv4 forward (one launch per step)",
+                         "algorithmic_bytes_per_launch": foot,
+                         "traffic": traffic, "traffic_source": traffic_src},
+            "e2e": {"value": e2e_value, "unit": UNIT, "ms_per_step": e2e_ms / args.e2e_steps,
+                    "steps": args.e2e_steps,
+                    "h2d_bytes_per_step": (x.numel() + om.numel()) * x.element_size(),
+                    "d2h_bytes_per_step": oh.numel() * oh.element_size(),
+                    "path": "dcnv4_forward_host: pinned host buffers, chunked H2D/kernel/D2H on two streams"},
+            "gpu_launches": timed_launches,
+            "clocks": clocks,
+            "cpu_baseline": base,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,11 @@
+"""B200-native DCNv4 forward spatial aggregation.
+
+The computation lives in libdcnv4.so (hand-written sm_100a CUDA kernels behind
+the C ABI of include/dcnv4.h); this package is its thin Python binding.
+``workloads`` holds the seeded synthetic input generators.
+"""
+from .binding import (  # noqa: F401
+    DCNV4_BF16, DCNV4_F16, DCNV4_F32, DCNV4_OK, EXPORTS, LIBRARY_PATH, STATUS, STATUS_NAMES,
+    DCNv4Error, abi_version, device_status, selftest_wait_timeout, forward, forward_host, load_library, output_shape, sampling_index, strerror,
+    validate,
+)

@@ -1,0 +1,232 @@
+"""ctypes binding of libdcnv4.so (the C ABI in include/dcnv4.h).
+
+Argument marshalling only: tensors are checked (device, dtype, shape,
+contiguity) and their data pointers are handed to the library together with
+the current CUDA stream; every step of the computation runs in the library's
+kernels. There is no fallback: if the library is missing or a call fails, an
+exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIBRARY_PATH = os.path.join(_PKG, "libdcnv4.so")
+
+DCNV4_F32, DCNV4_F16, DCNV4_BF16 = 0, 1, 2
+DCNV4_OK = 0
+STATUS_NAMES = {
+    0: "DCNV4_OK", 1: "DCNV4_ERR_NULL", 2: "DCNV4_ERR_SHAPE", 3: "DCNV4_ERR_GROUPS",
+    4: "DCNV4_ERR_DTYPE", 5: "DCNV4_ERR_ALIGN", 6: "DCNV4_ERR_ALIAS", 7: "DCNV4_ERR_SCALE",
+    8: "DCNV4_ERR_TOO_LARGE", 9: "DCNV4_ERR_LAUNCH", 10: "DCNV4_ERR_CUDA",
+}
+STATUS = {v: k for k, v in STATUS_NAMES.items()}
+TORCH_DTYPE = {torch.float32: DCNV4_F32, torch.float16: DCNV4_F16, torch.bfloat16: DCNV4_BF16}
+
+# every symbol include/dcnv4.h declares
+EXPORTS = ("dcnv4_output_shape", "dcnv4_validate", "dcnv4_forward", "dcnv4_sampling_index",
+           "dcnv4_forward_host", "dcnv4_device_status", "dcnv4_selftest_wait_timeout", "dcnv4_strerror",
+           "dcnv4_abi_version")
+DEVSTATUS_COPY_TIMEOUT, DEVSTATUS_SELFTEST_TIMEOUT = 1, 2
+
+_lib = None
+
+
+class DCNv4Error(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        name = STATUS_NAMES.get(status, str(status))
+        super().__init__(f"{where}: {name} ({strerror(status)})")
+
+
+def load_library():
+    """Load libdcnv4.so (built in-tree by ``deformable_convolution_sparse_b200.build``)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIBRARY_PATH):
+        raise RuntimeError(f"{LIBRARY_PATH} is missing: build it with "
+                           "`python -m deformable_convolution_sparse_b200.build`")
+    lib = ctypes.CDLL(LIBRARY_PATH)
+    i, f, p = ctypes.c_int, ctypes.c_float, ctypes.c_void_p
+    ip = ctypes.POINTER(ctypes.c_int)
+    lib.dcnv4_output_shape.argtypes = [i, i, i, i, i, i, ip, ip]
+    lib.dcnv4_output_shape.restype = i
+    lib.dcnv4_validate.argtypes = [p, p, p] + [i] * 9 + [f, i]
+    lib.dcnv4_validate.restype = i
+    lib.dcnv4_forward.argtypes = [p, p, p] + [i] * 9 + [f, i, p]
+    lib.dcnv4_forward.restype = i
+    lib.dcnv4_sampling_index.argtypes = [p, p, p] + [i] * 8 + [f, i, p]
+    lib.dcnv4_sampling_index.restype = i
+    lib.dcnv4_forward_host.argtypes = [p] * 6 + [i] * 9 + [f, i, p]
+    lib.dcnv4_forward_host.restype = i
+    lib.dcnv4_device_status.argtypes = [ctypes.POINTER(ctypes.c_uint), i]
+    lib.dcnv4_device_status.restype = i
+    lib.dcnv4_selftest_wait_timeout.argtypes = [ctypes.c_ulonglong, p]
+    lib.dcnv4_selftest_wait_timeout.restype = i
+    lib.dcnv4_strerror.argtypes = [i]
+    lib.dcnv4_strerror.restype = ctypes.c_char_p
+    lib.dcnv4_abi_version.argtypes = []
+    lib.dcnv4_abi_version.restype = i
+    _lib = lib
+    return lib
+
+
+def strerror(status: int) -> str:
+    return load_library().dcnv4_strerror(int(status)).decode()
+
+
+def abi_version() -> int:
+    return load_library().dcnv4_abi_version()
+
+
+def device_status(clear: bool = False) -> int:
+    """Device status word of the current device (waits for the device)."""
+    v = ctypes.c_uint(0)
+    rc = load_library().dcnv4_device_status(ctypes.byref(v), int(bool(clear)))
+    if rc != DCNV4_OK:
+        raise DCNv4Error(rc, "dcnv4_device_status")
+    return v.value
+
+
+def selftest_wait_timeout(limit_ns: int = 1_000_000, stream=None) -> None:
+    """Launches the bounded-wait self test (sets DEVSTATUS_SELFTEST_TIMEOUT)."""
+    rc = load_library().dcnv4_selftest_wait_timeout(int(limit_ns), _stream_handle(stream))
+    if rc != DCNV4_OK:
+        raise DCNv4Error(rc, "dcnv4_selftest_wait_timeout")
+
+
+def output_shape(H: int, W: int, K: int, stride: int = 1, pad: int = 0, dilation: int = 1):
+    """(Hout, Wout) from the library; raises DCNv4Error on invalid geometry."""
+    ho, wo = ctypes.c_int(0), ctypes.c_int(0)
+    rc = load_library().dcnv4_output_shape(H, W, K, stride, pad, dilation, ctypes.byref(ho), ctypes.byref(wo))
+    if rc != DCNV4_OK:
+        raise DCNv4Error(rc, "dcnv4_output_shape")
+    return ho.value, wo.value
+
+
+def validate(x_ptr: int, om_ptr: int, out_ptr: int, N: int, H: int, W: int, C: int, G: int, K: int,
+             stride: int = 1, pad: int = 0, dilation: int = 1, offset_scale: float = 1.0,
+             dtype: int = DCNV4_F32) -> int:
+    """Raw status of dcnv4_validate for the given pointers and sizes (no launch)."""
+    return load_library().dcnv4_validate(x_ptr, om_ptr, out_ptr, N, H, W, C, G, K, stride, pad, dilation,
+                                         float(offset_scale), int(dtype))
+
+
+def _stream_handle(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream)
+
+
+def _check_tensor(t: torch.Tensor, name: str):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be a CUDA tensor (got {t.device})")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if t.dtype not in TORCH_DTYPE:
+        raise TypeError(f"{name} has unsupported dtype {t.dtype}")
+
+
+def forward(x: torch.Tensor, offset_mask: torch.Tensor, G: int, K: int, stride: int = 1, pad: int = 0,
+            dilation: int = 1, offset_scale: float = 1.0, out: torch.Tensor | None = None,
+            stream=None) -> torch.Tensor:
+    """DCNv4 forward aggregation on the GPU through ``dcnv4_forward``.
+
+    x: [N,H,W,C]; offset_mask: [N,Hout,Wout,G,3*K*K] (per group: K*K x-offsets,
+    K*K y-offsets, K*K masks); returns out [N,Hout,Wout,C] in x's dtype. The
+    launch is asynchronous on ``stream`` (default: the current stream).
+    """
+    _check_tensor(x, "x")
+    _check_tensor(offset_mask, "offset_mask")
+    if x.dim() != 4:
+        raise ValueError("x must be [N,H,W,C]")
+    if offset_mask.dtype != x.dtype or offset_mask.device != x.device:
+        raise ValueError("offset_mask must match x in dtype and device")
+    N, H, W, C = x.shape
+    Hout, Wout = output_shape(H, W, K, stride, pad, dilation)
+    want = (N, Hout, Wout, G, 3 * K * K)
+    if tuple(offset_mask.shape) != want:
+        raise ValueError(f"offset_mask shape {tuple(offset_mask.shape)} != {want}")
+    if out is None:
+        out = torch.empty((N, Hout, Wout, C), dtype=x.dtype, device=x.device)
+    else:
+        _check_tensor(out, "out")
+        if tuple(out.shape) != (N, Hout, Wout, C) or out.dtype != x.dtype or out.device != x.device:
+            raise ValueError("out has the wrong shape, dtype or device")
+    with torch.cuda.device(x.device):
+        rc = load_library().dcnv4_forward(x.data_ptr(), offset_mask.data_ptr(), out.data_ptr(), N, H, W, C, G, K,
+                                          stride, pad, dilation, float(offset_scale), TORCH_DTYPE[x.dtype],
+                                          _stream_handle(stream))
+    if rc != DCNV4_OK:
+        raise DCNv4Error(rc, "dcnv4_forward")
+    return out
+
+
+def forward_host(x: torch.Tensor, offset_mask: torch.Tensor, G: int, K: int, stride: int = 1, pad: int = 0,
+                 dilation: int = 1, offset_scale: float = 1.0, out: torch.Tensor | None = None,
+                 staging=None, device=None, stream=None) -> torch.Tensor:
+    """Forward from host tensors through ``dcnv4_forward_host``.
+
+    x, offset_mask: CPU tensors (pin them for overlapped copies); returns the
+    CPU tensor ``out`` once the work is complete. ``staging`` = (x_dev,
+    offset_mask_dev, out_dev) device tensors of the full sizes; allocated on
+    ``device`` when not given.
+    """
+    for t, name in ((x, "x"), (offset_mask, "offset_mask")):
+        if t.device.type != "cpu" or not t.is_contiguous() or t.dtype not in TORCH_DTYPE:
+            raise ValueError(f"{name} must be a contiguous CPU tensor of a supported dtype")
+    if offset_mask.dtype != x.dtype:
+        raise ValueError("offset_mask must match x in dtype")
+    N, H, W, C = x.shape
+    Hout, Wout = output_shape(H, W, K, stride, pad, dilation)
+    if tuple(offset_mask.shape) != (N, Hout, Wout, G, 3 * K * K):
+        raise ValueError("offset_mask has the wrong shape")
+    if out is None:
+        out = torch.empty((N, Hout, Wout, C), dtype=x.dtype, pin_memory=x.is_pinned())
+    if tuple(out.shape) != (N, Hout, Wout, C) or out.dtype != x.dtype or out.device.type != "cpu" \
+            or not out.is_contiguous():
+        raise ValueError("out must be a contiguous CPU tensor of the output shape and x's dtype")
+    device = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+    if staging is None:
+        staging = (torch.empty_like(x, device=device), torch.empty_like(offset_mask, device=device),
+                   torch.empty_like(out, device=device))
+    xd, omd, od = staging
+    for t, ref, name in ((xd, x, "x_dev"), (omd, offset_mask, "offset_mask_dev"), (od, out, "out_dev")):
+        _check_tensor(t, name)
+        if t.shape != ref.shape or t.dtype != ref.dtype or t.device != xd.device:
+            raise ValueError(f"{name} must match the host tensor's shape and dtype on one device")
+    with torch.cuda.device(xd.device):
+        handle = _stream_handle(stream)
+        rc = load_library().dcnv4_forward_host(x.data_ptr(), offset_mask.data_ptr(), out.data_ptr(),
+                                               xd.data_ptr(), omd.data_ptr(), od.data_ptr(), N, H, W, C, G, K,
+                                               stride, pad, dilation, float(offset_scale), TORCH_DTYPE[x.dtype],
+                                               handle)
+        if rc != DCNV4_OK:
+            raise DCNv4Error(rc, "dcnv4_forward_host")
+        (stream or torch.cuda.current_stream()).synchronize()
+    return out
+
+
+def sampling_index(offset_mask: torch.Tensor, H: int, W: int, G: int, K: int, stride: int = 1, pad: int = 0,
+                   dilation: int = 1, offset_scale: float = 1.0, stream=None):
+    """Corner (y0, x0) [N,Hout,Wout,G,K*K,2] int32 and validity bits [N,Hout,Wout,G,K*K] uint8
+    through ``dcnv4_sampling_index``."""
+    _check_tensor(offset_mask, "offset_mask")
+    N, Hout, Wout, G_, R = offset_mask.shape
+    if G_ != G or R != 3 * K * K or (Hout, Wout) != output_shape(H, W, K, stride, pad, dilation):
+        raise ValueError("offset_mask shape does not match H, W, G, K")
+    corner = torch.empty((N, Hout, Wout, G, K * K, 2), dtype=torch.int32, device=offset_mask.device)
+    valid = torch.empty((N, Hout, Wout, G, K * K), dtype=torch.uint8, device=offset_mask.device)
+    with torch.cuda.device(offset_mask.device):
+        rc = load_library().dcnv4_sampling_index(offset_mask.data_ptr(), corner.data_ptr(), valid.data_ptr(),
+                                                 N, H, W, G, K, stride, pad, dilation, float(offset_scale),
+                                                 TORCH_DTYPE[offset_mask.dtype], _stream_handle(stream))
+    if rc != DCNV4_OK:
+        raise DCNv4Error(rc, "dcnv4_sampling_index")
+    return corner, valid

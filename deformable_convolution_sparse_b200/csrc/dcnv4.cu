@@ -1,0 +1,469 @@
+// Host side of libdcnv4.so: argument checks, kernel selection and launch.
+// The C ABI is declared (with the meaning of every argument) in include/dcnv4.h.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <algorithm>
+#include <mutex>
+
+#include <cstdlib>
+#include <cstring>
+
+#include "dcnv4.h"
+#include "dcnv4_kernels.cuh"
+#include "dcnv4_window.cuh"
+
+namespace {
+
+using dcnv4::FwdParams;
+
+int elem_size(int dtype) {
+    switch (dtype) {
+        case DCNV4_F32: return 4;
+        case DCNV4_F16: return 2;
+        case DCNV4_BF16: return 2;
+        default: return 0;
+    }
+}
+
+bool aligned(const void* p, int a) { return (reinterpret_cast<uintptr_t>(p) % static_cast<uintptr_t>(a)) == 0; }
+
+bool overlap(const void* a, long long abytes, const void* b, long long bbytes) {
+    if (abytes <= 0 || bbytes <= 0) return false;
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+    return a0 < b0 + static_cast<uintptr_t>(bbytes) && b0 < a0 + static_cast<uintptr_t>(abytes);
+}
+
+constexpr long long kLimit = 1LL << 31;  // element counts stay below 2^31 (32-bit indexing)
+
+// Shape checks shared by the forward and the index dump. Fills Hout/Wout.
+int check_geometry(int N, int H, int W, int K, int stride, int pad, int dilation, int* Hout, int* Wout) {
+    if (N < 0) return DCNV4_ERR_SHAPE;
+    const int rc = dcnv4_output_shape(H, W, K, stride, pad, dilation, Hout, Wout);
+    return rc;
+}
+
+int launch_status() {
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? DCNV4_OK : DCNV4_ERR_LAUNCH;
+}
+
+// ------------------------------------------------------------ dispatch ---
+
+constexpr int kThreads = 256;
+
+// Kernel choice: DCNV4_VARIANT=gather forces the global-gather kernel (A/B
+// comparisons); unset or anything else selects the shared-memory window kernel
+// whenever the shape allows it. DCNV4_HALO overrides the window halo (pixels).
+enum class Variant { Auto, Gather };
+
+Variant variant_from_env() {
+    const char* v = std::getenv("DCNV4_VARIANT");
+    if (v && std::strcmp(v, "gather") == 0) return Variant::Gather;
+    return Variant::Auto;
+}
+
+constexpr size_t kWindowSmemBudget = 110 * 1024;  // two CTAs per SM
+
+// Fills a WinParams for the window kernel; false when the shape does not suit it.
+template <typename T>
+bool plan_window(const void* x, const void* out, const FwdParams& f, dcnv4::WinParams* wp, size_t* smem_bytes) {
+    constexpr int E = sizeof(T);
+    const int row_bytes = f.Cg * E;
+    if (!aligned(x, 16) || !aligned(out, 16) || (f.C * E) % 16 || row_bytes % 16) return false;
+    const int Q = row_bytes / 16;
+    if (!(Q == 1 || Q == 2 || Q == 4 || Q == 5 || Q == 8)) return false;
+    int GS = f.G;
+    for (int d = 1; d <= f.G; ++d)
+        if (f.G % d == 0 && (d * row_bytes) % 128 == 0) { GS = d; break; }
+    const int PB = GS * row_bytes;
+    int R = 4;
+    if (const char* h = std::getenv("DCNV4_HALO")) R = std::atoi(h) > 0 ? std::atoi(h) : R;
+    const int R3 = 3 * f.KK;
+    static const int cand[][2] = {{8, 16}, {16, 8}, {8, 8}, {4, 16}, {4, 8}, {8, 4}, {4, 4}, {2, 4}, {2, 2}, {1, 2}, {1, 1}};
+    double best = -1.0;
+    dcnv4::WinParams bestp{};
+    size_t best_smem = 0;
+    for (const auto& c : cand) {
+        const int TH = c[0], TW = c[1];
+        const int WH = (TH - 1) * f.stride + (f.K - 1) * f.dilation + 2 * R + 1;
+        const int WW = (TW - 1) * f.stride + (f.K - 1) * f.dilation + 2 * R + 1;
+        const bool row_runs = GS == f.G;
+        const int nruns = row_runs ? TH : TH * TW;
+        const int count = (row_runs ? TW * f.G : GS) * R3;
+        const int slot = ((count * E + 16) + 15) / 16 * 16;
+        const size_t rec = static_cast<size_t>(nruns) * slot;
+        const size_t win_off = (rec + 127) / 128 * 128;
+        const size_t smem = win_off + static_cast<size_t>(WH) * WW * PB;
+        if (smem > kWindowSmemBudget) continue;
+        const int tiles_y = (f.Hout + TH - 1) / TH, tiles_x = (f.Wout + TW - 1) / TW;
+        const double useful = static_cast<double>(f.Hout) * f.Wout / (static_cast<double>(tiles_y) * TH * tiles_x * TW);
+        const double reuse = static_cast<double>(TH * TW) / (static_cast<double>(WH) * WW);
+        const double fill = std::min(1.0, TH * TW * GS / 256.0);
+        const double score = useful * reuse * fill;
+        if (score > best) {
+            best = score;
+            bestp.TH = TH; bestp.TW = TW; bestp.tiles_x = tiles_x; bestp.tiles_y = tiles_y;
+            bestp.WH = WH; bestp.WW = WW; bestp.run_slot = slot; bestp.win_off = static_cast<int>(win_off);
+            best_smem = smem;
+        }
+    }
+    if (best < 0) return false;
+    bestp.f = f;
+    bestp.GS = GS;
+    bestp.nsub = f.G / GS;
+    bestp.R = R;
+    bestp.PB = PB;
+    bestp.units = bestp.TH * bestp.TW * GS;
+    bestp.div_tw_gs = dcnv4::make_fastdiv(bestp.TW * GS);
+    bestp.div_gs = dcnv4::make_fastdiv(GS);
+    bestp.div_nsub = dcnv4::make_fastdiv(bestp.nsub);
+    bestp.div_tx = dcnv4::make_fastdiv(bestp.tiles_x);
+    bestp.div_ty = dcnv4::make_fastdiv(bestp.tiles_y);
+    *wp = bestp;
+    *smem_bytes = best_smem;
+    return true;
+}
+
+template <typename T, int Q, int KS>
+int launch_window_q(const T* x, const T* om, T* out, const dcnv4::WinParams& wp, size_t smem, cudaStream_t stream) {
+    auto kern = dcnv4::fwd_window_kernel<T, Q, KS>;
+    static bool attr_set = false;  // benign race: every thread sets the same value
+    if (!attr_set) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(kWindowSmemBudget)) != cudaSuccess)
+            return DCNV4_ERR_LAUNCH;
+        attr_set = true;
+    }
+    const long long blocks = static_cast<long long>(wp.f.N) * wp.tiles_y * wp.tiles_x * wp.nsub;
+    if (blocks > 0x7fffffffLL) return DCNV4_ERR_TOO_LARGE;
+    kern<<<static_cast<unsigned>(blocks), 256, smem, stream>>>(x, om, out, wp);
+    return launch_status();
+}
+
+template <typename T, int Q>
+int launch_window_k(const T* x, const T* om, T* out, const dcnv4::WinParams& wp, size_t smem, cudaStream_t s) {
+    if (wp.f.K == 3) return launch_window_q<T, Q, 3>(x, om, out, wp, smem, s);
+    return launch_window_q<T, Q, 0>(x, om, out, wp, smem, s);
+}
+
+template <typename T>
+int launch_window(const void* x, const void* om, void* out, const dcnv4::WinParams& wp, size_t smem, cudaStream_t s) {
+    const T* xt = static_cast<const T*>(x);
+    const T* omt = static_cast<const T*>(om);
+    T* ot = static_cast<T*>(out);
+    switch (wp.f.Cg * static_cast<int>(sizeof(T)) / 16) {
+        case 1: return launch_window_k<T, 1>(xt, omt, ot, wp, smem, s);
+        case 2: return launch_window_k<T, 2>(xt, omt, ot, wp, smem, s);
+        case 4: return launch_window_k<T, 4>(xt, omt, ot, wp, smem, s);
+        case 5: return launch_window_k<T, 5>(xt, omt, ot, wp, smem, s);
+        default: return launch_window_k<T, 8>(xt, omt, ot, wp, smem, s);
+    }
+}
+
+template <typename T>
+int launch_forward(const void* x, const void* om, void* out, FwdParams p, cudaStream_t stream) {
+    constexpr int E = sizeof(T);
+    if (variant_from_env() == Variant::Auto) {
+        dcnv4::WinParams wp;
+        size_t smem = 0;
+        if (plan_window<T>(x, out, p, &wp, &smem)) return launch_window<T>(x, om, out, wp, smem, stream);
+    }
+    const int row_bytes = p.Cg * E;
+    const bool a16 = aligned(x, 16) && aligned(out, 16) && (p.C * E) % 16 == 0;
+    const bool a32 = aligned(x, 32) && aligned(out, 32) && (p.C * E) % 32 == 0;
+    const size_t rec_bytes = static_cast<size_t>(3) * p.KK * E;
+
+    int lane_bytes = 0, vec_bytes = 0;
+    if (a16 && row_bytes % 16 == 0) {
+        if (a32 && row_bytes % 32 == 0) {
+            vec_bytes = 32;
+            lane_bytes = (E == 4 && row_bytes % 64 == 0) ? 64 : 32;
+        } else {
+            vec_bytes = 16;
+            lane_bytes = 16;
+        }
+    }
+    if (lane_bytes) {
+        p.chunks = row_bytes / lane_bytes;
+        p.lanes = p.chunks < kThreads ? p.chunks : kThreads;
+    } else {
+        p.chunks = p.Cg;
+        p.lanes = p.Cg < kThreads ? p.Cg : kThreads;
+    }
+    int upb = kThreads / p.lanes;
+    const size_t smem_cap = 40 * 1024;
+    while (upb > 1 && upb * rec_bytes + 16 > smem_cap) --upb;
+    p.units_per_block = upb;
+    const size_t smem = upb * rec_bytes + 16;
+    const int threads = upb * p.lanes;
+    const long long blocks = (static_cast<long long>(p.units) + upb - 1) / upb;
+    if (blocks > 0x7fffffffLL) return DCNV4_ERR_TOO_LARGE;
+    const dim3 grid(static_cast<unsigned>(blocks));
+
+    const T* xt = static_cast<const T*>(x);
+    const T* omt = static_cast<const T*>(om);
+    T* ot = static_cast<T*>(out);
+    const bool k3 = p.K == 3;
+    if (lane_bytes == 64) {
+        if (k3) dcnv4::fwd_vector_kernel<T, 32, 64, 3><<<grid, threads, smem, stream>>>(xt, omt, ot, p);
+        else dcnv4::fwd_vector_kernel<T, 32, 64, 0><<<grid, threads, smem, stream>>>(xt, omt, ot, p);
+    } else if (lane_bytes == 32) {
+        if (k3) dcnv4::fwd_vector_kernel<T, 32, 32, 3><<<grid, threads, smem, stream>>>(xt, omt, ot, p);
+        else dcnv4::fwd_vector_kernel<T, 32, 32, 0><<<grid, threads, smem, stream>>>(xt, omt, ot, p);
+    } else if (lane_bytes == 16) {
+        if (k3) dcnv4::fwd_vector_kernel<T, 16, 16, 3><<<grid, threads, smem, stream>>>(xt, omt, ot, p);
+        else dcnv4::fwd_vector_kernel<T, 16, 16, 0><<<grid, threads, smem, stream>>>(xt, omt, ot, p);
+    } else {
+        if (k3) dcnv4::fwd_scalar_kernel<T, 3><<<grid, threads, smem, stream>>>(xt, omt, ot, p);
+        else dcnv4::fwd_scalar_kernel<T, 0><<<grid, threads, smem, stream>>>(xt, omt, ot, p);
+    }
+    return launch_status();
+}
+
+// Two non-blocking streams per device for the host-memory entry point,
+// created on first use and kept for the life of the process.
+constexpr int kMaxDevices = 64;
+struct HostPipe {
+    cudaStream_t s[2] = {nullptr, nullptr};
+    bool ready = false;
+};
+HostPipe g_pipes[kMaxDevices];
+std::mutex g_pipe_mutex;
+
+int host_pipe(HostPipe** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DCNV4_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_pipe_mutex);
+    HostPipe& p = g_pipes[dev];
+    if (!p.ready) {
+        for (int i = 0; i < 2; ++i)
+            if (cudaStreamCreateWithFlags(&p.s[i], cudaStreamNonBlocking) != cudaSuccess) return DCNV4_ERR_CUDA;
+        p.ready = true;
+    }
+    *out = &p;
+    return DCNV4_OK;
+}
+
+FwdParams make_params(int N, int H, int W, int C, int G, int K, int stride, int pad, int dilation,
+                      float offset_scale, int Hout, int Wout) {
+    FwdParams p{};
+    p.N = N; p.H = H; p.W = W; p.C = C; p.G = G; p.K = K; p.KK = K * K; p.Cg = C / G;
+    p.stride = stride; p.pad = pad; p.dilation = dilation;
+    p.Hout = Hout; p.Wout = Wout;
+    p.units = N * Hout * Wout * G;
+    p.offset_scale = offset_scale;
+    return p;
+}
+
+}  // namespace
+
+extern "C" {
+
+int dcnv4_abi_version(void) { return DCNV4_ABI_VERSION; }
+
+const char* dcnv4_strerror(int status) {
+    switch (status) {
+        case DCNV4_OK: return "ok";
+        case DCNV4_ERR_NULL: return "a required pointer is NULL";
+        case DCNV4_ERR_SHAPE: return "invalid shape or convolution geometry";
+        case DCNV4_ERR_GROUPS: return "C is not a multiple of G";
+        case DCNV4_ERR_DTYPE: return "unknown dtype";
+        case DCNV4_ERR_ALIGN: return "a pointer is not aligned to its element size";
+        case DCNV4_ERR_ALIAS: return "an output buffer overlaps an input buffer";
+        case DCNV4_ERR_SCALE: return "offset_scale is not finite";
+        case DCNV4_ERR_TOO_LARGE: return "an element count reaches 2^31";
+        case DCNV4_ERR_LAUNCH: return "kernel launch failed";
+        case DCNV4_ERR_CUDA: return "CUDA runtime call failed";
+        default: return "unknown status";
+    }
+}
+
+int dcnv4_output_shape(int H, int W, int K, int stride, int pad, int dilation, int* Hout, int* Wout) {
+    if (H <= 0 || W <= 0 || K <= 0 || K > DCNV4_MAX_K || stride <= 0 || dilation <= 0 || pad < 0)
+        return DCNV4_ERR_SHAPE;
+    if (H > DCNV4_MAX_EXTENT || W > DCNV4_MAX_EXTENT || pad > DCNV4_MAX_EXTENT ||
+        stride > DCNV4_MAX_EXTENT || dilation > DCNV4_MAX_EXTENT)
+        return DCNV4_ERR_SHAPE;
+    const long long span_h = static_cast<long long>(H) + 2LL * pad - static_cast<long long>(dilation) * (K - 1) - 1;
+    const long long span_w = static_cast<long long>(W) + 2LL * pad - static_cast<long long>(dilation) * (K - 1) - 1;
+    if (span_h < 0 || span_w < 0) return DCNV4_ERR_SHAPE;
+    const long long ho = span_h / stride + 1, wo = span_w / stride + 1;
+    // every grid coordinate p0 = o*stride - pad + k*dilation lies in [-pad, extent + pad - 1]
+    if (ho > DCNV4_MAX_EXTENT || wo > DCNV4_MAX_EXTENT) return DCNV4_ERR_SHAPE;
+    if (Hout) *Hout = static_cast<int>(ho);
+    if (Wout) *Wout = static_cast<int>(wo);
+    return DCNV4_OK;
+}
+
+int dcnv4_validate(const void* x, const void* offset_mask, const void* out,
+                   int N, int H, int W, int C, int G, int K,
+                   int stride, int pad, int dilation, float offset_scale, int dtype) {
+    int Hout = 0, Wout = 0;
+    int rc = check_geometry(N, H, W, K, stride, pad, dilation, &Hout, &Wout);
+    if (rc) return rc;
+    if (C <= 0 || G <= 0) return DCNV4_ERR_SHAPE;
+    if (C % G) return DCNV4_ERR_GROUPS;
+    const int e = elem_size(dtype);
+    if (!e) return DCNV4_ERR_DTYPE;
+    if (!std::isfinite(offset_scale)) return DCNV4_ERR_SCALE;
+    const long long nx = static_cast<long long>(N) * H * W * C;
+    const long long nout = static_cast<long long>(N) * Hout * Wout * C;
+    const long long nom = static_cast<long long>(N) * Hout * Wout * G * 3 * K * K;
+    if (nx >= kLimit || nout >= kLimit || nom >= kLimit) return DCNV4_ERR_TOO_LARGE;
+    if (N == 0) return DCNV4_OK;
+    if (!x || !offset_mask || !out) return DCNV4_ERR_NULL;
+    if (!aligned(x, e) || !aligned(offset_mask, e) || !aligned(out, e)) return DCNV4_ERR_ALIGN;
+    if (overlap(out, nout * e, x, nx * e) || overlap(out, nout * e, offset_mask, nom * e)) return DCNV4_ERR_ALIAS;
+    return DCNV4_OK;
+}
+
+int dcnv4_forward(const void* x, const void* offset_mask, void* out,
+                  int N, int H, int W, int C, int G, int K,
+                  int stride, int pad, int dilation, float offset_scale, int dtype,
+                  void* stream) {
+    const int rc = dcnv4_validate(x, offset_mask, out, N, H, W, C, G, K, stride, pad, dilation, offset_scale, dtype);
+    if (rc) return rc;
+    if (N == 0) return DCNV4_OK;
+    int Hout = 0, Wout = 0;
+    dcnv4_output_shape(H, W, K, stride, pad, dilation, &Hout, &Wout);
+    const FwdParams p = make_params(N, H, W, C, G, K, stride, pad, dilation, offset_scale, Hout, Wout);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    switch (dtype) {
+        case DCNV4_F32: return launch_forward<float>(x, offset_mask, out, p, s);
+        case DCNV4_F16: return launch_forward<__half>(x, offset_mask, out, p, s);
+        default: return launch_forward<__nv_bfloat16>(x, offset_mask, out, p, s);
+    }
+}
+
+int dcnv4_forward_host(const void* x_host, const void* offset_mask_host, void* out_host,
+                       void* x_dev, void* offset_mask_dev, void* out_dev,
+                       int N, int H, int W, int C, int G, int K,
+                       int stride, int pad, int dilation, float offset_scale, int dtype,
+                       void* stream) {
+    int rc = dcnv4_validate(x_dev, offset_mask_dev, out_dev, N, H, W, C, G, K, stride, pad, dilation,
+                            offset_scale, dtype);
+    if (rc) return rc;
+    if (N == 0) return DCNV4_OK;
+    if (!x_host || !offset_mask_host || !out_host) return DCNV4_ERR_NULL;
+    int Hout = 0, Wout = 0;
+    dcnv4_output_shape(H, W, K, stride, pad, dilation, &Hout, &Wout);
+    const size_t e = static_cast<size_t>(elem_size(dtype));
+    const size_t x_img = static_cast<size_t>(H) * W * C * e;
+    const size_t om_img = static_cast<size_t>(Hout) * Wout * G * 3 * K * K * e;
+    const size_t out_img = static_cast<size_t>(Hout) * Wout * C * e;
+    if (overlap(out_host, static_cast<long long>(out_img * N), x_host, static_cast<long long>(x_img * N)) ||
+        overlap(out_host, static_cast<long long>(out_img * N), offset_mask_host, static_cast<long long>(om_img * N)))
+        return DCNV4_ERR_ALIAS;
+
+    HostPipe* pipe = nullptr;
+    rc = host_pipe(&pipe);
+    if (rc) return rc;
+    cudaStream_t user = static_cast<cudaStream_t>(stream);
+    cudaEvent_t ev_start = nullptr, ev_done[2] = {nullptr, nullptr};
+    auto fail = [&](int code) {
+        if (ev_start) cudaEventDestroy(ev_start);
+        for (auto& ev : ev_done)
+            if (ev) cudaEventDestroy(ev);
+        return code;
+    };
+    if (cudaEventCreateWithFlags(&ev_start, cudaEventDisableTiming) != cudaSuccess) return fail(DCNV4_ERR_CUDA);
+    for (auto& ev : ev_done)
+        if (cudaEventCreateWithFlags(&ev, cudaEventDisableTiming) != cudaSuccess) return fail(DCNV4_ERR_CUDA);
+    if (cudaEventRecord(ev_start, user) != cudaSuccess) return fail(DCNV4_ERR_CUDA);
+    for (int i = 0; i < 2; ++i)
+        if (cudaStreamWaitEvent(pipe->s[i], ev_start, 0) != cudaSuccess) return fail(DCNV4_ERR_CUDA);
+
+    // chunks of whole images: enough of them for the two copy directions to overlap
+    const int chunks = N < 8 ? N : 8;
+    const char* xh = static_cast<const char*>(x_host);
+    const char* omh = static_cast<const char*>(offset_mask_host);
+    char* oh = static_cast<char*>(out_host);
+    char* xd = static_cast<char*>(x_dev);
+    char* omd = static_cast<char*>(offset_mask_dev);
+    char* od = static_cast<char*>(out_dev);
+    int n0 = 0;
+    for (int c = 0; c < chunks; ++c) {
+        const int n1 = static_cast<int>((static_cast<long long>(N) * (c + 1)) / chunks);
+        const int nc = n1 - n0;
+        if (nc == 0) continue;
+        cudaStream_t s = pipe->s[c & 1];
+        if (cudaMemcpyAsync(xd + n0 * x_img, xh + n0 * x_img, nc * x_img, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+            cudaMemcpyAsync(omd + n0 * om_img, omh + n0 * om_img, nc * om_img, cudaMemcpyHostToDevice, s) != cudaSuccess)
+            return fail(DCNV4_ERR_CUDA);
+        rc = dcnv4_forward(xd + n0 * x_img, omd + n0 * om_img, od + n0 * out_img, nc, H, W, C, G, K, stride, pad,
+                           dilation, offset_scale, dtype, s);
+        if (rc) return fail(rc);
+        if (cudaMemcpyAsync(oh + n0 * out_img, od + n0 * out_img, nc * out_img, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+            return fail(DCNV4_ERR_CUDA);
+        n0 = n1;
+    }
+    for (int i = 0; i < 2; ++i) {
+        if (cudaEventRecord(ev_done[i], pipe->s[i]) != cudaSuccess || cudaStreamWaitEvent(user, ev_done[i], 0) != cudaSuccess)
+            return fail(DCNV4_ERR_CUDA);
+    }
+    // events may be destroyed while pending: the waits already queued keep their meaning
+    fail(DCNV4_OK);
+    return DCNV4_OK;
+}
+
+int dcnv4_device_status(unsigned int* status, int clear) {
+    if (!status) return DCNV4_ERR_NULL;
+    unsigned v = 0;
+    if (cudaMemcpyFromSymbol(&v, dcnv4::g_device_status, sizeof(v)) != cudaSuccess) return DCNV4_ERR_CUDA;
+    *status = v;
+    if (clear) {
+        const unsigned z = 0;
+        if (cudaMemcpyToSymbol(dcnv4::g_device_status, &z, sizeof(z)) != cudaSuccess) return DCNV4_ERR_CUDA;
+    }
+    return DCNV4_OK;
+}
+
+int dcnv4_selftest_wait_timeout(unsigned long long limit_ns, void* stream) {
+    if (limit_ns == 0 || limit_ns > 2000000000ull) return DCNV4_ERR_SHAPE;
+    dcnv4::selftest_wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns);
+    return launch_status();
+}
+
+int dcnv4_sampling_index(const void* offset_mask, int32_t* corner, uint8_t* valid,
+                         int N, int H, int W, int G, int K,
+                         int stride, int pad, int dilation, float offset_scale, int dtype,
+                         void* stream) {
+    int Hout = 0, Wout = 0;
+    int rc = check_geometry(N, H, W, K, stride, pad, dilation, &Hout, &Wout);
+    if (rc) return rc;
+    if (G <= 0) return DCNV4_ERR_SHAPE;
+    const int e = elem_size(dtype);
+    if (!e) return DCNV4_ERR_DTYPE;
+    if (!std::isfinite(offset_scale)) return DCNV4_ERR_SCALE;
+    const long long npts = static_cast<long long>(N) * Hout * Wout * G * K * K;
+    if (3 * npts >= kLimit) return DCNV4_ERR_TOO_LARGE;
+    if (N == 0) return DCNV4_OK;
+    if (!offset_mask || !corner || !valid) return DCNV4_ERR_NULL;
+    if (!aligned(offset_mask, e) || !aligned(corner, 4)) return DCNV4_ERR_ALIGN;
+    if (overlap(corner, 8 * npts, offset_mask, 3 * npts * e) || overlap(valid, npts, offset_mask, 3 * npts * e) ||
+        overlap(valid, npts, corner, 8 * npts))
+        return DCNV4_ERR_ALIAS;
+    FwdParams p = make_params(N, H, W, G, G, K, stride, pad, dilation, offset_scale, Hout, Wout);
+    const long long want = (npts + 255) / 256;
+    const unsigned blocks = static_cast<unsigned>(want < 148 * 32 ? want : 148 * 32);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    switch (dtype) {
+        case DCNV4_F32:
+            dcnv4::sampling_index_kernel<float><<<blocks, 256, 0, s>>>(
+                static_cast<const float*>(offset_mask), corner, valid, p);
+            break;
+        case DCNV4_F16:
+            dcnv4::sampling_index_kernel<__half><<<blocks, 256, 0, s>>>(
+                static_cast<const __half*>(offset_mask), corner, valid, p);
+            break;
+        default:
+            dcnv4::sampling_index_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(
+                static_cast<const __nv_bfloat16*>(offset_mask), corner, valid, p);
+            break;
+    }
+    return launch_status();
+}
+
+}  // extern "C"

@@ -1,0 +1,189 @@
+/*
+ * dcnv4.h -- C ABI of libdcnv4.so, the B200 (sm_100a) DCNv4 forward spatial
+ * aggregation.
+ *
+ * The operation (sources by page title and section):
+ *   "不只是卷积的平替：我把DCNv4塞进Stable Diffusion的U-Net里" (jsqmd.com),
+ *   section 1: DCNv4 drops the softmax over the aggregation weights, so the
+ *   per-point modulation scalars are used as they are (any sign, any size);
+ *   its simplified forward listing adds learned offsets to a regular K x K
+ *   grid, samples the input bilinearly at the moved points and sums the
+ *   samples weighted by the masks, separately for each channel group.
+ *   "掌握DCNv4技术：3倍速度提升与80%加速效果的实战指南" (pwwt.cn), tuning
+ *   section: offset_scale multiplies the offsets; group sets the number of
+ *   channel groups.
+ *
+ * For output pixel (n, ho, wo), group g (channels [g*Cg, (g+1)*Cg), Cg = C/G)
+ * and grid point k = ky*K + kx (row-major), with r = offset_mask[n,ho,wo,g,:]:
+ *   p0y = ho*stride - pad + ky*dilation,  p0x = wo*stride - pad + kx*dilation
+ *   dx  = fl32(offset_scale * r[k]),      dy  = fl32(offset_scale * r[K*K + k])
+ *   m   = r[2*K*K + k]                    (raw modulation scalar, no softmax)
+ *   out[n,ho,wo,g*Cg + c] = sum_k m * bilinear(x[n,:,:,g*Cg + c], p0y + dy, p0x + dx)
+ * where bilinear() reads zero outside the image, corner by corner: corners
+ * (y0+a, x0+b), y0 = p0y + floor(dy), x0 = p0x + floor(dx), a,b in {0,1},
+ * weighted (a ? fy : 1-fy) * (b ? fx : 1-fx), fy = dy - floor(dy),
+ * fx = dx - floor(dx). Corners inside the image always take part (also with
+ * weight 0); a non-finite offset puts the whole sample outside. Products and
+ * sums are fp32; the result is rounded once (round-to-nearest-even) to the
+ * storage type.
+ *
+ * Layouts (all contiguous, row-major, caller-owned DEVICE memory unless
+ * stated otherwise):
+ *   x           [N, H, W, C]                  channels-last
+ *   offset_mask [N, Hout, Wout, G, 3*K*K]     per group: K*K x-offsets (along
+ *                                             the width), K*K y-offsets, K*K masks
+ *   out         [N, Hout, Wout, C]
+ * with Hout = (H + 2*pad - dilation*(K-1) - 1)/stride + 1 (the same for W).
+ * x, offset_mask and out share one storage type (dtype).
+ *
+ * Conventions:
+ *   - Every call is thread-safe; the library keeps no pointer after return
+ *     and allocates no device memory.
+ *   - Compute calls are asynchronous on `stream` (a cudaStream_t; NULL is the
+ *     legacy default stream) and never synchronise. Arguments are checked on
+ *     the host before anything is launched; on a non-zero return nothing was
+ *     launched (except DCNV4_ERR_LAUNCH, reported when the launch itself
+ *     failed).
+ *   - Buffer sizes cannot be checked through raw pointers: the caller
+ *     guarantees each buffer holds the element count its layout implies.
+ *   - NaN / Inf inside x or the masks are data, not errors.
+ */
+#ifndef DCNV4_H
+#define DCNV4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define DCNV4_ABI_VERSION 1
+
+/* symbols of the shared library (it is built with hidden default visibility) */
+#if defined(__GNUC__)
+#define DCNV4_API __attribute__((visibility("default")))
+#else
+#define DCNV4_API
+#endif
+
+/* Storage type of x, offset_mask and out. Arithmetic is fp32 in all cases. */
+typedef enum {
+    DCNV4_F32 = 0,
+    DCNV4_F16 = 1,
+    DCNV4_BF16 = 2
+} dcnv4_dtype_t;
+
+typedef enum {
+    DCNV4_OK = 0,
+    DCNV4_ERR_NULL = 1,      /* a required pointer is NULL (N > 0)                      */
+    DCNV4_ERR_SHAPE = 2,     /* N < 0; H, W, C, G, K, stride or dilation <= 0; pad < 0;  */
+                             /* Hout or Wout <= 0; K > DCNV4_MAX_K; a spatial extent or  */
+                             /* grid coordinate beyond DCNV4_MAX_EXTENT                  */
+    DCNV4_ERR_GROUPS = 3,    /* C is not a multiple of G                                */
+    DCNV4_ERR_DTYPE = 4,     /* dtype is not a dcnv4_dtype_t value                      */
+    DCNV4_ERR_ALIGN = 5,     /* a pointer is not aligned to its element size            */
+    DCNV4_ERR_ALIAS = 6,     /* an output buffer overlaps an input buffer               */
+    DCNV4_ERR_SCALE = 7,     /* offset_scale is NaN or infinite                         */
+    DCNV4_ERR_TOO_LARGE = 8, /* an element count reaches 2^31                           */
+    DCNV4_ERR_LAUNCH = 9,    /* the kernel launch failed (CUDA error after launch)      */
+    DCNV4_ERR_CUDA = 10      /* a CUDA runtime call other than a launch failed          */
+} dcnv4_status_t;
+
+#define DCNV4_MAX_K 16
+#define DCNV4_MAX_EXTENT (1 << 22)
+
+/* Output extent, convolution style (the formula above).
+ * Writes *Hout, *Wout (either may be NULL) and returns DCNV4_OK, or
+ * DCNV4_ERR_SHAPE when an argument is out of range or an extent would be <= 0
+ * (outputs are then left untouched). Host only; no CUDA call. */
+DCNV4_API int dcnv4_output_shape(int H, int W, int K, int stride, int pad, int dilation,
+                       int *Hout, int *Wout);
+
+/* Checks the arguments of dcnv4_forward without launching anything.
+ * Pointers are only compared (NULL, alignment to the element size, overlap of
+ * out with x or offset_mask over the byte ranges their shapes imply); they
+ * are never dereferenced. N == 0 is valid (pointers may then be NULL).
+ * Returns DCNV4_OK or the first failing dcnv4_status_t. Host only. */
+DCNV4_API int dcnv4_validate(const void *x, const void *offset_mask, const void *out,
+                   int N, int H, int W, int C, int G, int K,
+                   int stride, int pad, int dilation, float offset_scale, int dtype);
+
+/* The forward aggregation (the formula above) for the whole batch.
+ * x, offset_mask: read only; out: fully overwritten. All three are device
+ * pointers in the layouts above. Runs dcnv4_validate first and returns its
+ * code without launching when it fails. On success one kernel is launched
+ * on `stream` (none when N == 0) and DCNV4_OK is returned; the result is
+ * ready when the stream reaches that point. */
+DCNV4_API int dcnv4_forward(const void *x, const void *offset_mask, void *out,
+                  int N, int H, int W, int C, int G, int K,
+                  int stride, int pad, int dilation, float offset_scale, int dtype,
+                  void *stream);
+
+/* The integer half of the forward, exposed so that it can be compared bit for
+ * bit: for every sampling point (n, ho, wo, g, k) it writes the top-left
+ * corner (y0, x0) into corner[2*p], corner[2*p+1] and a 4-bit mask of the
+ * corners inside the image into valid[p] (bit 0: (y0,x0), bit 1: (y0,x0+1),
+ * bit 2: (y0+1,x0), bit 3: (y0+1,x0+1)), p = (((n*Hout+ho)*Wout+wo)*G+g)*K*K+k.
+ * A point with no corner inside reports corner = (INT32_MIN, INT32_MIN).
+ * corner: device int32 [N,Hout,Wout,G,K*K,2]; valid: device uint8
+ * [N,Hout,Wout,G,K*K]. The coordinates are computed by the same device code
+ * that the forward kernels use. Same checks as dcnv4_forward with C = G
+ * (x is not read; the x and out checks do not apply). */
+DCNV4_API int dcnv4_sampling_index(const void *offset_mask, int32_t *corner, uint8_t *valid,
+                         int N, int H, int W, int G, int K,
+                         int stride, int pad, int dilation, float offset_scale, int dtype,
+                         void *stream);
+
+/* The forward from and to HOST memory, for callers whose data lives on the
+ * host. x_host, offset_mask_host: inputs in host memory (pinned memory lets
+ * the copies run asynchronously and overlap; pageable memory works but the
+ * copies then block the calling thread); out_host: host memory receiving the
+ * result. x_dev, offset_mask_dev, out_dev: caller-owned device buffers of the
+ * full sizes of x, offset_mask and out, used as staging (their contents
+ * afterwards: the copied inputs and the result). The batch is split into
+ * chunks of whole images; each chunk's host-to-device copies, kernel and
+ * device-to-host copy are queued on one of two library-owned non-blocking
+ * streams (created once per device on first use and kept until exit), so the
+ * copies of neighbouring chunks overlap in the two copy directions. The call
+ * is ordered after the work already queued on `stream`, and `stream` waits for
+ * all of it before its next work: synchronise `stream` before reading
+ * out_host. Checks: those of dcnv4_forward on the device buffers, plus NULL
+ * host pointers (DCNV4_ERR_NULL) and out_host overlapping x_host or
+ * offset_mask_host (DCNV4_ERR_ALIAS). A failing CUDA copy, event or stream
+ * call returns DCNV4_ERR_CUDA. */
+DCNV4_API int dcnv4_forward_host(const void *x_host, const void *offset_mask_host, void *out_host,
+                                 void *x_dev, void *offset_mask_dev, void *out_dev,
+                                 int N, int H, int W, int C, int G, int K,
+                                 int stride, int pad, int dilation, float offset_scale, int dtype,
+                                 void *stream);
+
+/* Device-side status word of the current device (bit flags below). The
+ * shared-memory window kernel waits for its bulk copies with a time limit
+ * (1 s); if a wait ever gives up, the CTA sets DCNV4_DEVSTATUS_COPY_TIMEOUT,
+ * waits once more (bounded) for copies in flight and leaves its tile
+ * unwritten, so a stuck copy shows up here instead of as a hung GPU.
+ * Reads the word into *status (synchronous: waits for the device) and, when
+ * `clear` is non-zero, resets it to 0. Returns DCNV4_OK, DCNV4_ERR_NULL or
+ * DCNV4_ERR_CUDA. */
+#define DCNV4_DEVSTATUS_COPY_TIMEOUT 1u
+#define DCNV4_DEVSTATUS_SELFTEST_TIMEOUT 2u
+DCNV4_API int dcnv4_device_status(unsigned int *status, int clear);
+
+/* Exercises the bounded wait without any fault: one CTA arms an mbarrier for
+ * 16 bytes that are never sent, waits `limit_ns` nanoseconds (1 ns .. 2 s),
+ * sets DCNV4_DEVSTATUS_SELFTEST_TIMEOUT and returns. Asynchronous on `stream`.
+ * Returns DCNV4_OK, DCNV4_ERR_SHAPE (limit out of range) or DCNV4_ERR_LAUNCH. */
+DCNV4_API int dcnv4_selftest_wait_timeout(unsigned long long limit_ns, void *stream);
+
+/* Static description of an error code; never NULL. */
+DCNV4_API const char *dcnv4_strerror(int status);
+
+/* DCNV4_ABI_VERSION of the built library. */
+DCNV4_API int dcnv4_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DCNV4_H */

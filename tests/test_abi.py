@@ -1,0 +1,130 @@
+"""Host-side tests of the C ABI (no GPU needed): the library loads, exports
+every symbol include/dcnv4.h declares, and its argument checks return the
+documented status for every error class without launching anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import oracle
+from deformable_convolution_sparse_b200 import binding as B
+from deformable_convolution_sparse_b200.workloads import WORKLOADS
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "dcnv4.h")
+
+
+def _declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"DCNV4_API\s+[\w\s\*]*?\b(dcnv4_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_exports():
+    assert _declared_symbols() == sorted(B.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol():
+    lib = B.load_library()
+    for name in _declared_symbols():
+        assert hasattr(lib, name), name
+    assert B.abi_version() == 1
+
+
+def test_strerror_covers_every_status():
+    for code, name in B.STATUS_NAMES.items():
+        msg = B.strerror(code)
+        assert msg and msg != "unknown status", name
+    assert B.strerror(12345) == "unknown status"
+
+
+@pytest.mark.parametrize("H,W,K,s,p,d", [(56, 56, 3, 1, 1, 1), (256, 256, 3, 1, 1, 2), (14, 9, 3, 2, 1, 1),
+                                         (9, 11, 5, 3, 2, 2), (4, 4, 2, 2, 0, 2), (1, 1, 1, 1, 0, 1),
+                                         (7, 5, 1, 4, 0, 1), (3, 3, 16, 1, 8, 1)])
+def test_output_shape_matches_oracle(H, W, K, s, p, d):
+    assert B.output_shape(H, W, K, s, p, d) == (oracle.output_size(H, K, s, p, d), oracle.output_size(W, K, s, p, d))
+
+
+def test_named_workloads_state_the_right_output_size():
+    for w in WORKLOADS.values():
+        assert (w.Hout, w.Wout) == B.output_shape(w.H, w.W, w.K, w.stride, w.pad, w.dilation), w.name
+        assert w.Hout == oracle.output_size(w.H, w.K, w.stride, w.pad, w.dilation), w.name
+
+
+@pytest.mark.parametrize("args", [(0, 5, 3, 1, 1, 1), (5, 0, 3, 1, 1, 1), (5, 5, 0, 1, 1, 1), (5, 5, 3, 0, 1, 1),
+                                  (5, 5, 3, 1, -1, 1), (5, 5, 3, 1, 1, 0), (2, 2, 5, 1, 0, 1), (5, 5, 17, 1, 8, 1),
+                                  (1 << 23, 5, 3, 1, 1, 1)])
+def test_output_shape_rejects_bad_geometry(args):
+    lib = B.load_library()
+    ho, wo = ctypes.c_int(-7), ctypes.c_int(-7)
+    assert lib.dcnv4_output_shape(*args, ctypes.byref(ho), ctypes.byref(wo)) == B.STATUS["DCNV4_ERR_SHAPE"]
+    assert (ho.value, wo.value) == (-7, -7)
+
+
+# fake, never dereferenced device addresses
+X, OM, OUT = 0x10000000, 0x20000000, 0x30000000
+GOOD = dict(N=2, H=8, W=8, C=16, G=2, K=3, stride=1, pad=1, dilation=1, offset_scale=1.0, dtype=B.DCNV4_F16)
+
+
+def _v(x=X, om=OM, out=OUT, **kw):
+    a = dict(GOOD)
+    a.update(kw)
+    return B.validate(x, om, out, a["N"], a["H"], a["W"], a["C"], a["G"], a["K"], a["stride"], a["pad"],
+                      a["dilation"], a["offset_scale"], a["dtype"])
+
+
+def test_validate_accepts_good_arguments():
+    assert _v() == B.DCNV4_OK
+    assert _v(dtype=B.DCNV4_F32) == B.DCNV4_OK
+    assert _v(dtype=B.DCNV4_BF16, offset_scale=-0.5) == B.DCNV4_OK
+    assert _v(x=0, om=0, out=0, N=0) == B.DCNV4_OK  # empty batch: nothing is touched
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(x=0), "DCNV4_ERR_NULL"), (dict(om=0), "DCNV4_ERR_NULL"), (dict(out=0), "DCNV4_ERR_NULL"),
+    (dict(N=-1), "DCNV4_ERR_SHAPE"), (dict(H=0), "DCNV4_ERR_SHAPE"), (dict(C=0), "DCNV4_ERR_SHAPE"),
+    (dict(G=0), "DCNV4_ERR_SHAPE"), (dict(K=0), "DCNV4_ERR_SHAPE"), (dict(stride=0), "DCNV4_ERR_SHAPE"),
+    (dict(pad=-1), "DCNV4_ERR_SHAPE"), (dict(dilation=-2), "DCNV4_ERR_SHAPE"),
+    (dict(H=2, W=2, pad=0), "DCNV4_ERR_SHAPE"),
+    (dict(C=18, G=4), "DCNV4_ERR_GROUPS"),
+    (dict(dtype=3), "DCNV4_ERR_DTYPE"), (dict(dtype=-1), "DCNV4_ERR_DTYPE"),
+    (dict(x=X + 1), "DCNV4_ERR_ALIGN"), (dict(om=OM + 1), "DCNV4_ERR_ALIGN"), (dict(out=OUT + 3), "DCNV4_ERR_ALIGN"),
+    (dict(x=X + 2, dtype=B.DCNV4_F32), "DCNV4_ERR_ALIGN"),
+    (dict(out=X), "DCNV4_ERR_ALIAS"), (dict(out=OM + 64), "DCNV4_ERR_ALIAS"), (dict(x=OUT - 32), "DCNV4_ERR_ALIAS"),
+    (dict(offset_scale=float("nan")), "DCNV4_ERR_SCALE"), (dict(offset_scale=float("inf")), "DCNV4_ERR_SCALE"),
+    (dict(N=1 << 20, H=64, W=64, C=64, G=4), "DCNV4_ERR_TOO_LARGE"),
+])
+def test_validate_reports_each_error_class(kw, status):
+    assert _v(**kw) == B.STATUS[status]
+
+
+def test_inputs_may_overlap_each_other():
+    # x and offset_mask are both read only: sharing memory is allowed
+    assert _v(om=X) == B.DCNV4_OK
+
+
+def test_forward_returns_validation_errors_before_any_cuda_call():
+    lib = B.load_library()
+    a = dict(GOOD)
+    rc = lib.dcnv4_forward(X, OM, OUT, a["N"], a["H"], a["W"], 18, 4, a["K"], 1, 1, 1, 1.0, a["dtype"], None)
+    assert rc == B.STATUS["DCNV4_ERR_GROUPS"]
+    rc = lib.dcnv4_forward(X, OM, X, a["N"], a["H"], a["W"], 16, 2, 3, 1, 1, 1, 1.0, a["dtype"], None)
+    assert rc == B.STATUS["DCNV4_ERR_ALIAS"]
+    # an empty batch launches nothing and succeeds, also without a GPU
+    assert lib.dcnv4_forward(0, 0, 0, 0, 8, 8, 16, 2, 3, 1, 1, 1, 1.0, a["dtype"], None) == B.DCNV4_OK
+
+
+def test_sampling_index_checks():
+    lib = B.load_library()
+    assert lib.dcnv4_sampling_index(OM, X, OUT, 1, 8, 8, 2, 3, 1, 1, 1, 1.0, 5, None) == B.STATUS["DCNV4_ERR_DTYPE"]
+    assert lib.dcnv4_sampling_index(0, X, OUT, 1, 8, 8, 2, 3, 1, 1, 1, 1.0, 1, None) == B.STATUS["DCNV4_ERR_NULL"]
+    assert lib.dcnv4_sampling_index(OM, X + 2, OUT, 1, 8, 8, 2, 3, 1, 1, 1, 1.0, 1, None) == B.STATUS["DCNV4_ERR_ALIGN"]
+    assert lib.dcnv4_sampling_index(OM, OM, OUT, 1, 8, 8, 2, 3, 1, 1, 1, 1.0, 1, None) == B.STATUS["DCNV4_ERR_ALIAS"]
+    assert lib.dcnv4_sampling_index(0, 0, 0, 0, 8, 8, 2, 3, 1, 1, 1, 1.0, 1, None) == B.DCNV4_OK
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    x = torch.zeros(1, 8, 8, 16)
+    om = torch.zeros(1, 8, 8, 2, 27)
+    with pytest.raises(ValueError, match="CUDA"):
+        B.forward(x, om, G=2, K=3, pad=1)
