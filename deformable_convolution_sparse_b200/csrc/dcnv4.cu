@@ -1,12 +1,16 @@
 // Host side of libdcnv4.so: argument checks, kernel selection and launch.
 // The C ABI is declared (with the meaning of every argument) in include/dcnv4.h.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <cmath>
 #include <cstdint>
 #include <algorithm>
+#include <cmath>
 #include <mutex>
 
+#include <cstdio>
 #include <cstdlib>
 #include <cstring>
 
@@ -54,8 +58,9 @@ int launch_status() {
 constexpr int kThreads = 256;
 
 // Kernel choice: DCNV4_VARIANT=gather forces the global-gather kernel (A/B
-// comparisons); unset or anything else selects the shared-memory window kernel
-// whenever the shape allows it. DCNV4_HALO overrides the window halo (pixels).
+// comparisons); unset or anything else selects the persistent shared-memory
+// tile kernel whenever the shape allows it. DCNV4_HALO overrides the window
+// halo (pixels) and DCNV4_TILE=<TH>x<TW> the output tile, for tuning runs.
 enum class Variant { Auto, Gather };
 
 Variant variant_from_env() {
@@ -64,101 +69,198 @@ Variant variant_from_env() {
     return Variant::Auto;
 }
 
-constexpr size_t kWindowSmemBudget = 110 * 1024;  // two CTAs per SM
+constexpr size_t kTileSmemLimit = 226 * 1024;  // dynamic shared memory per CTA (sm_100: 227 KB with the static part)
+constexpr int kTileUnitsMax = 512;  // consumer threads (16 warps) per CTA, plus one producer warp
 
-// Fills a WinParams for the window kernel; false when the shape does not suit it.
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    });
+    return fn;
+}
+
+template <typename T> CUtensorMapDataType tma_dtype();
+template <> CUtensorMapDataType tma_dtype<float>() { return CU_TENSOR_MAP_DATA_TYPE_FLOAT32; }
+template <> CUtensorMapDataType tma_dtype<__half>() { return CU_TENSOR_MAP_DATA_TYPE_FLOAT16; }
+template <> CUtensorMapDataType tma_dtype<__nv_bfloat16>() { return CU_TENSOR_MAP_DATA_TYPE_BFLOAT16; }
+
+struct TilePlan {
+    dcnv4::TileParams p;
+    CUtensorMap map;
+    size_t smem;
+    int threads;
+};
+
+int sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return 0;
+    return n;
+}
+
+// Chooses group subset, tile and halo for the tile kernel and encodes the
+// tensor map of x; false when the shape or the alignment does not suit it.
 template <typename T>
-bool plan_window(const void* x, const void* out, const FwdParams& f, dcnv4::WinParams* wp, size_t* smem_bytes) {
+bool plan_tile(const void* x, const void* om, const void* out, const FwdParams& f, TilePlan* plan) {
     constexpr int E = sizeof(T);
     const int row_bytes = f.Cg * E;
     if (!aligned(x, 16) || !aligned(out, 16) || (f.C * E) % 16 || row_bytes % 16) return false;
     const int Q = row_bytes / 16;
     if (!(Q == 1 || Q == 2 || Q == 4 || Q == 5 || Q == 8)) return false;
-    int GS = f.G;
-    for (int d = 1; d <= f.G; ++d)
-        if (f.G % d == 0 && (d * row_bytes) % 128 == 0) { GS = d; break; }
-    const int PB = GS * row_bytes;
-    int R = 4;
+    if (f.KK > 64) return false;  // the per-unit mask of points outside the window has 64 bits
+    int R = 5;
     if (const char* h = std::getenv("DCNV4_HALO")) R = std::atoi(h) > 0 ? std::atoi(h) : R;
+    int forceTH = 0, forceTW = 0, forceGS = 0;
+    if (const char* t = std::getenv("DCNV4_TILE")) std::sscanf(t, "%dx%d", &forceTH, &forceTW);
+    if (const char* g = std::getenv("DCNV4_GS")) forceGS = std::atoi(g);
     const int R3 = 3 * f.KK;
-    static const int cand[][2] = {{8, 16}, {16, 8}, {8, 8}, {4, 16}, {4, 8}, {8, 4}, {4, 4}, {2, 4}, {2, 2}, {1, 2}, {1, 1}};
+    const int nsm = sm_count();
+    if (nsm <= 0) return false;
+
+    static const int THs[] = {1, 2, 4, 7, 8, 14, 16, 28, 32};
+    static const int TWs[] = {1, 2, 4, 7, 8, 14, 16, 28, 32};
     double best = -1.0;
-    dcnv4::WinParams bestp{};
+    dcnv4::TileParams bp{};
+    int best_threads = 0, best_c2 = 0;
     size_t best_smem = 0;
-    for (const auto& c : cand) {
-        const int TH = c[0], TW = c[1];
-        const int WH = (TH - 1) * f.stride + (f.K - 1) * f.dilation + 2 * R + 1;
-        const int WW = (TW - 1) * f.stride + (f.K - 1) * f.dilation + 2 * R + 1;
+    for (int GS = 1; GS <= f.G; ++GS) {
+        if (f.G % GS || (forceGS && GS != forceGS)) continue;
+        const int PB = GS * row_bytes;
+        const int sub_ch = GS * f.Cg;
+        int c2 = 0;
+        for (int d = std::min(sub_ch, 256); d >= 1; --d)
+            if (sub_ch % d == 0 && (d * E) % 16 == 0) { c2 = d; break; }
+        if (c2 == 0 || sub_ch / c2 > 256) continue;
+        // a pixel stride that is a multiple of 128 bytes keeps the gathers free of
+        // bank conflicts (see the kernel); other strides pay for some
+        const double banks = (PB % 128 == 0) ? 1.0 : 0.6;
         const bool row_runs = GS == f.G;
-        const int nruns = row_runs ? TH : TH * TW;
-        const int count = (row_runs ? TW * f.G : GS) * R3;
-        const int slot = ((count * E + 16) + 15) / 16 * 16;
-        const size_t rec = static_cast<size_t>(nruns) * slot;
-        const size_t win_off = (rec + 127) / 128 * 128;
-        const size_t smem = win_off + static_cast<size_t>(WH) * WW * PB;
-        if (smem > kWindowSmemBudget) continue;
-        const int tiles_y = (f.Hout + TH - 1) / TH, tiles_x = (f.Wout + TW - 1) / TW;
-        const double useful = static_cast<double>(f.Hout) * f.Wout / (static_cast<double>(tiles_y) * TH * tiles_x * TW);
-        const double reuse = static_cast<double>(TH * TW) / (static_cast<double>(WH) * WW);
-        const double fill = std::min(1.0, TH * TW * GS / 256.0);
-        const double score = useful * reuse * fill;
-        if (score > best) {
-            best = score;
-            bestp.TH = TH; bestp.TW = TW; bestp.tiles_x = tiles_x; bestp.tiles_y = tiles_y;
-            bestp.WH = WH; bestp.WW = WW; bestp.run_slot = slot; bestp.win_off = static_cast<int>(win_off);
-            best_smem = smem;
+        for (int TH : THs) {
+            for (int TW : TWs) {
+                if (forceTH && (TH != forceTH || TW != forceTW)) continue;
+                const int units = TH * TW * GS;
+                if (units > kTileUnitsMax || units < 32) continue;
+                if (TH > f.Hout + 7 || TW > f.Wout + 7) continue;
+                const int WH = (TH - 1) * f.stride + (f.K - 1) * f.dilation + 2 * R + 1;
+                const int WW = (TW - 1) * f.stride + (f.K - 1) * f.dilation + 2 * R + 1;
+                if (WH > 256 || WW > 256) continue;
+                const int nruns = row_runs ? TH : TH * TW;
+                const int count = (row_runs ? TW * f.G : GS) * R3;
+                const int slot = (count * E + 32 + 15) / 16 * 16;
+                const size_t rec = (static_cast<size_t>(nruns) * slot + 127) / 128 * 128;
+                const size_t win = (static_cast<size_t>(WH) * WW * PB + 127) / 128 * 128;
+                const size_t smem = 2 * (rec + win);
+                if (smem > kTileSmemLimit) continue;
+                const int threads = (units + 31) / 32 * 32 + 32;  // consumers + the producer warp
+                const int tiles_y = (f.Hout + TH - 1) / TH, tiles_x = (f.Wout + TW - 1) / TW;
+                const long long tiles = static_cast<long long>(f.N) * tiles_y * tiles_x * (f.G / GS);
+                const int per_sm = std::max(1, static_cast<int>(std::min<size_t>(
+                                                   (kTileSmemLimit + 2048) / (smem + 1024), 2048 / threads)));
+                const double slots = static_cast<double>(nsm) * per_sm;
+                const double waves = static_cast<double>(tiles) / slots;
+                const double balance = waves / std::ceil(waves);
+                const double useful =
+                    static_cast<double>(f.Hout) * f.Wout / (static_cast<double>(tiles_y) * TH * tiles_x * TW);
+                const double reuse = static_cast<double>(TH * TW) / (static_cast<double>(WH) * WW);
+                const double fill = static_cast<double>(units) / (threads - 32);
+                const double occ = std::min(1.0, per_sm * (threads - 32) / 512.0);
+                const double score = useful * balance * fill * occ * banks * std::sqrt(reuse);
+                if (score > best) {
+                    best = score;
+                    bp.TH = TH; bp.TW = TW; bp.tiles_x = tiles_x; bp.tiles_y = tiles_y;
+                    bp.WH = WH; bp.WW = WW; bp.run_slot = slot; bp.rec_bytes = static_cast<int>(rec);
+                    bp.buf_bytes = static_cast<int>(rec + win);
+                    bp.tiles = static_cast<int>(tiles); bp.units = units;
+                    bp.GS = GS; bp.PB = PB; bp.cblk = sub_ch / c2;
+                    best_threads = threads;
+                    best_smem = smem;
+                    best_c2 = c2;
+                }
+            }
         }
     }
     if (best < 0) return false;
-    bestp.f = f;
-    bestp.GS = GS;
-    bestp.nsub = f.G / GS;
-    bestp.R = R;
-    bestp.PB = PB;
-    bestp.units = bestp.TH * bestp.TW * GS;
-    bestp.div_tw_gs = dcnv4::make_fastdiv(bestp.TW * GS);
-    bestp.div_gs = dcnv4::make_fastdiv(GS);
-    bestp.div_nsub = dcnv4::make_fastdiv(bestp.nsub);
-    bestp.div_tx = dcnv4::make_fastdiv(bestp.tiles_x);
-    bestp.div_ty = dcnv4::make_fastdiv(bestp.tiles_y);
-    *wp = bestp;
-    *smem_bytes = best_smem;
+    const int GS = bp.GS, PB = bp.PB, c2 = best_c2;
+    bp.f = f;
+    bp.nsub = f.G / GS;
+    bp.R = R;
+    const size_t om_bytes = static_cast<size_t>(f.N) * f.Hout * f.Wout * f.G * R3 * E;
+    bp.om_lo = reinterpret_cast<unsigned long long>(om);
+    bp.om_hi = bp.om_lo + om_bytes;
+    bp.div_tw_gs = dcnv4::make_fastdiv(bp.TW * GS);
+    bp.div_gs = dcnv4::make_fastdiv(GS);
+    bp.div_nsub = dcnv4::make_fastdiv(bp.nsub);
+    bp.div_tx = dcnv4::make_fastdiv(bp.tiles_x);
+    bp.div_ty = dcnv4::make_fastdiv(bp.tiles_y);
+
+    auto encode = tensor_map_encoder();
+    if (!encode) return false;
+    const cuuint64_t dims[5] = {static_cast<cuuint64_t>(c2), static_cast<cuuint64_t>(f.C / c2),
+                                static_cast<cuuint64_t>(f.W), static_cast<cuuint64_t>(f.H),
+                                static_cast<cuuint64_t>(f.N)};
+    const cuuint64_t strides[4] = {static_cast<cuuint64_t>(c2) * E, static_cast<cuuint64_t>(f.C) * E,
+                                   static_cast<cuuint64_t>(f.W) * f.C * E,
+                                   static_cast<cuuint64_t>(f.H) * f.W * f.C * E};
+    const cuuint32_t box[5] = {static_cast<cuuint32_t>(c2), static_cast<cuuint32_t>(bp.cblk),
+                               static_cast<cuuint32_t>(bp.WW), static_cast<cuuint32_t>(bp.WH), 1u};
+    const cuuint32_t estr[5] = {1u, 1u, 1u, 1u, 1u};
+    if (encode(&plan->map, tma_dtype<T>(), 5, const_cast<void*>(x), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return false;
+    plan->p = bp;
+    plan->smem = best_smem;
+    plan->threads = best_threads;
+    if (const char* d = std::getenv("DCNV4_DEBUG"); d && *d == '1')
+        std::fprintf(stderr,
+                     "dcnv4 tile plan: tile %dx%d GS %d (nsub %d) R %d window %dx%d PB %d cblk %d tiles %d units %d "
+                     "threads %d smem %zu\n",
+                     bp.TH, bp.TW, GS, bp.nsub, R, bp.WH, bp.WW, PB, bp.cblk, bp.tiles, bp.units, best_threads,
+                     best_smem);
     return true;
 }
 
 template <typename T, int Q, int KS>
-int launch_window_q(const T* x, const T* om, T* out, const dcnv4::WinParams& wp, size_t smem, cudaStream_t stream) {
-    auto kern = dcnv4::fwd_window_kernel<T, Q, KS>;
-    static bool attr_set = false;  // benign race: every thread sets the same value
-    if (!attr_set) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(kWindowSmemBudget)) != cudaSuccess)
-            return DCNV4_ERR_LAUNCH;
-        attr_set = true;
-    }
-    const long long blocks = static_cast<long long>(wp.f.N) * wp.tiles_y * wp.tiles_x * wp.nsub;
-    if (blocks > 0x7fffffffLL) return DCNV4_ERR_TOO_LARGE;
-    kern<<<static_cast<unsigned>(blocks), 256, smem, stream>>>(x, om, out, wp);
+int launch_tile_q(const T* x, const T* om, T* out, const TilePlan& plan, cudaStream_t stream) {
+    auto kern = dcnv4::fwd_tile_kernel<T, Q, KS>;
+    static std::once_flag once;
+    static cudaError_t attr = cudaSuccess;
+    std::call_once(once, [&] {
+        attr = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kTileSmemLimit));
+    });
+    if (attr != cudaSuccess) return DCNV4_ERR_LAUNCH;
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, plan.threads, plan.smem) != cudaSuccess || per_sm < 1)
+        return DCNV4_ERR_LAUNCH;
+    const long long slots = static_cast<long long>(sm_count()) * per_sm;
+    const unsigned grid = static_cast<unsigned>(std::min<long long>(plan.p.tiles, slots));
+    kern<<<grid, plan.threads, plan.smem, stream>>>(plan.map, x, om, out, plan.p);
     return launch_status();
 }
 
 template <typename T, int Q>
-int launch_window_k(const T* x, const T* om, T* out, const dcnv4::WinParams& wp, size_t smem, cudaStream_t s) {
-    if (wp.f.K == 3) return launch_window_q<T, Q, 3>(x, om, out, wp, smem, s);
-    return launch_window_q<T, Q, 0>(x, om, out, wp, smem, s);
+int launch_tile_k(const T* x, const T* om, T* out, const TilePlan& plan, cudaStream_t s) {
+    if (plan.p.f.K == 3) return launch_tile_q<T, Q, 3>(x, om, out, plan, s);
+    return launch_tile_q<T, Q, 0>(x, om, out, plan, s);
 }
 
 template <typename T>
-int launch_window(const void* x, const void* om, void* out, const dcnv4::WinParams& wp, size_t smem, cudaStream_t s) {
+int launch_tile(const void* x, const void* om, void* out, const TilePlan& plan, cudaStream_t s) {
     const T* xt = static_cast<const T*>(x);
     const T* omt = static_cast<const T*>(om);
     T* ot = static_cast<T*>(out);
-    switch (wp.f.Cg * static_cast<int>(sizeof(T)) / 16) {
-        case 1: return launch_window_k<T, 1>(xt, omt, ot, wp, smem, s);
-        case 2: return launch_window_k<T, 2>(xt, omt, ot, wp, smem, s);
-        case 4: return launch_window_k<T, 4>(xt, omt, ot, wp, smem, s);
-        case 5: return launch_window_k<T, 5>(xt, omt, ot, wp, smem, s);
-        default: return launch_window_k<T, 8>(xt, omt, ot, wp, smem, s);
+    switch (plan.p.f.Cg * static_cast<int>(sizeof(T)) / 16) {
+        case 1: return launch_tile_k<T, 1>(xt, omt, ot, plan, s);
+        case 2: return launch_tile_k<T, 2>(xt, omt, ot, plan, s);
+        case 4: return launch_tile_k<T, 4>(xt, omt, ot, plan, s);
+        case 5: return launch_tile_k<T, 5>(xt, omt, ot, plan, s);
+        default: return launch_tile_k<T, 8>(xt, omt, ot, plan, s);
     }
 }
 
@@ -166,9 +268,8 @@ template <typename T>
 int launch_forward(const void* x, const void* om, void* out, FwdParams p, cudaStream_t stream) {
     constexpr int E = sizeof(T);
     if (variant_from_env() == Variant::Auto) {
-        dcnv4::WinParams wp;
-        size_t smem = 0;
-        if (plan_window<T>(x, out, p, &wp, &smem)) return launch_window<T>(x, om, out, wp, smem, stream);
+        TilePlan plan;
+        if (plan_tile<T>(x, om, out, p, &plan)) return launch_tile<T>(x, om, out, plan, stream);
     }
     const int row_bytes = p.Cg * E;
     const bool a16 = aligned(x, 16) && aligned(out, 16) && (p.C * E) % 16 == 0;

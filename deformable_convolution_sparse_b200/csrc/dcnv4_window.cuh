@@ -1,15 +1,20 @@
-// Shared-memory window kernel of the DCNv4 forward aggregation (sm_100a).
+// Persistent shared-memory window kernel of the DCNv4 forward aggregation (sm_100a).
 //
 // The scattered 2x2 corner gathers are the whole cost of the op ("DCNv4：重塑视觉模型核心",
 // bqwf.cn, section 2.2: memory access dominates). Served from L1 they return a
 // couple of 32-byte sectors per clock; served from shared memory with a
-// bank-aware layout they return the full 128 bytes per clock. So each CTA takes
-// a tile of output pixels (TH x TW) and a subset of GS channel groups, brings the
-// input window its samples can reach (the tile's grid positions widened by a
-// halo of R pixels; zero outside the image) and the tile's offset/mask records
-// into shared memory with bulk copies (cp.async.bulk on the TMA engine, one
-// instruction per contiguous row, completion counted on an mbarrier), and then
-// gathers from shared memory.
+// bank-aware layout they return the full 128 bytes per clock. So the kernel
+// works tile by tile: a tile is TH x TW output pixels of one image and a subset
+// of GS channel groups. For each tile the CTA brings into shared memory
+//  - the input window its samples can reach: the tile's grid positions widened
+//    by a halo of R pixels, all GS*Cg channels of each pixel, as ONE TMA tensor
+//    load (cp.async.bulk.tensor, 5-D map over x); pixels outside the image
+//    arrive as zeros from the TMA unit itself;
+//  - the tile's offset/mask records, as one bulk copy (cp.async.bulk) per
+//    contiguous run (a tile row when the CTA owns all groups, else a pixel);
+// both counted on one mbarrier per buffer. CTAs are persistent and double
+// buffered: while the threads gather tile i from one buffer, warp 0 has
+// already issued the copies of tile i+1 into the other.
 //
 // Thread <-> work: one thread per (pixel, group) unit, covering all Cg channels
 // of the unit as Q 16-byte chunks. The window stores a pixel's GS*Cg channels
@@ -19,9 +24,13 @@
 // per LDS.128 when every lane starts at a rotated chunk (rot below), so each
 // 128-byte shared-memory wavefront carries 128 useful bytes.
 //
-// Samples whose 2x2 corners fall outside the window, or whose mask value is not
-// finite, take the global-memory path of the gather kernel (same arithmetic).
+// Samples whose 2x2 corners fall outside the window (offsets beyond the halo),
+// or whose mask value is not finite, are marked during the pass over the
+// window and gathered afterwards from global memory with per-corner validity,
+// so a warp waits for that memory latency once rather than once per point.
 #pragma once
+
+#include <cuda.h>
 
 #include "dcnv4_kernels.cuh"
 
@@ -30,7 +39,7 @@ namespace dcnv4 {
 // Device-side status word (bit flags below), read and cleared from the host
 // through dcnv4_device_status().
 __device__ unsigned int g_device_status;
-constexpr unsigned kStatusCopyTimeout = 1u;     // a bulk-copy wait gave up in the forward kernel
+constexpr unsigned kStatusCopyTimeout = 1u;     // a copy wait gave up in the forward kernel
 constexpr unsigned kStatusSelftestTimeout = 2u; // the self-test wait gave up (expected)
 
 // n / d for 0 <= n < 2^31 by multiply-high and shift (Granlund & Montgomery,
@@ -53,20 +62,22 @@ __device__ __forceinline__ unsigned fdiv(unsigned n, const FastDiv& f) {
     return (__umulhi(n, f.mul) + n) >> f.shift;
 }
 
-struct WinParams {
+struct TileParams {
     FwdParams f;
-    int TH, TW;            // output tile
+    int TH, TW;             // output tile
     int tiles_x, tiles_y;
-    int GS, nsub;          // groups per CTA, G / GS
-    int R;                 // halo in pixels around the tile's grid positions
-    int WH, WW;            // window extent (pixels)
-    int PB;                // bytes per window pixel: GS * Cg * sizeof(T)
-    int run_slot;          // shared bytes reserved per record run
-    int win_off;           // shared-memory byte offset of the window
-    int units;             // TH * TW * GS
-    FastDiv div_tw_gs;     // TW * GS
-    FastDiv div_gs;        // GS
-    FastDiv div_nsub, div_tx, div_ty;
+    int GS, nsub;           // groups per tile, G / GS
+    int R;                  // halo in pixels around the tile's grid positions
+    int WH, WW;             // window extent (pixels)
+    int PB;                 // bytes per window pixel: GS * Cg * sizeof(T)
+    int cblk;               // channel blocks of the tensor map per group subset
+    int tiles;              // N * tiles_y * tiles_x * nsub
+    int units;              // TH * TW * GS
+    int run_slot;           // shared bytes per record run
+    int rec_bytes;          // record area of one buffer (multiple of 128)
+    int buf_bytes;          // one buffer: records + window (multiple of 128)
+    unsigned long long om_lo, om_hi;  // byte range of the offset_mask tensor
+    FastDiv div_tw_gs, div_gs, div_nsub, div_tx, div_ty;
 };
 
 // ------------------------------------------------------ mbarrier + bulk copy ---
@@ -76,7 +87,11 @@ __device__ __forceinline__ unsigned smem_addr(const void* p) {
 }
 __device__ __forceinline__ void mbar_init(uint64_t* bar, unsigned count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void fence_barrier_init() {
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void fence_proxy_async() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, unsigned bytes) {
@@ -112,18 +127,24 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, unsigned parity
     }
 }
 // global -> shared bulk copy of `bytes` (multiple of 16; both addresses 16-byte
-// aligned), completion counted on `bar`. No cluster multicast.
-__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, unsigned bytes, uint64_t* bar) {
+// aligned) with its byte count posted on `bar` first. No cluster multicast.
+__device__ __forceinline__ void bulk_g2s_counted(void* dst, const void* src, unsigned bytes, uint64_t* bar) {
+    mbar_expect_tx(bar, bytes);
     asm volatile(
         "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
             smem_addr(dst)),
         "l"(src), "r"(bytes), "r"(smem_addr(bar))
         : "memory");
 }
-// expect + issue one bulk copy (called by the issuing thread)
-__device__ __forceinline__ void bulk_g2s_counted(void* dst, const void* src, unsigned bytes, uint64_t* bar) {
-    mbar_expect_tx(bar, bytes);
-    bulk_g2s(dst, src, bytes, bar);
+// One TMA tile load from a 5-D tensor map (no multicast); out-of-range
+// elements are written as zeros. The caller posts the byte count.
+__device__ __forceinline__ void tma_load_5d(void* dst, const CUtensorMap* map, int c0, int c1, int c2, int c3, int c4,
+                                            uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5, "
+        "%6}], [%7];" ::"r"(smem_addr(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4), "r"(smem_addr(bar))
+        : "memory");
 }
 
 constexpr uint64_t kCopyWaitLimitNs = 1000000000ull;  // 1 s
@@ -160,219 +181,258 @@ __device__ __forceinline__ uint4 pack_chunk(const float2* a) {
     return v;
 }
 
-// Brings `nbytes` of global memory at `src` (aligned to the element size) to
-// shared memory at slot + (src & 15): the 16-byte-aligned middle by one bulk
-// copy (issued by this thread), the ragged head and tail (< 16 bytes each) by
-// plain element copies. The bulk copy's byte count is posted on `bar` here.
-// The caller synchronises the block before reading the slot.
+// ------------------------------------------------------------ tiles ---
+
+struct TileCoord {
+    int n, gsub, ho0, wo0, nh, nw, wy0, wx0;
+};
+
+__device__ __forceinline__ TileCoord tile_coord(const TileParams& p, unsigned t) {
+    TileCoord c;
+    const unsigned t1 = fdiv(t, p.div_nsub);
+    c.gsub = static_cast<int>(t - t1 * p.nsub);
+    const unsigned t2 = fdiv(t1, p.div_tx);
+    const int tx = static_cast<int>(t1 - t2 * p.tiles_x);
+    const unsigned n = fdiv(t2, p.div_ty);
+    const int ty = static_cast<int>(t2 - n * p.tiles_y);
+    c.n = static_cast<int>(n);
+    c.ho0 = ty * p.TH;
+    c.wo0 = tx * p.TW;
+    c.nh = min(p.TH, p.f.Hout - c.ho0);
+    c.nw = min(p.TW, p.f.Wout - c.wo0);
+    c.wy0 = c.ho0 * p.f.stride - p.f.pad - p.R;
+    c.wx0 = c.wo0 * p.f.stride - p.f.pad - p.R;
+    return c;
+}
+
+// Address and element count of record run r of a tile.
 template <typename T>
-__device__ __forceinline__ void stage_bytes(const T* src, int count, unsigned char* slot, uint64_t* bar) {
+__device__ __forceinline__ const unsigned char* run_src(const TileParams& p, const TileCoord& c, const T* om, int r,
+                                                        int* count) {
+    const FwdParams& f = p.f;
+    const bool row_runs = p.GS == f.G;
+    const int py = row_runs ? r : r / c.nw;
+    const int px = row_runs ? 0 : r - py * c.nw;
+    const size_t first_unit = (static_cast<size_t>((c.n * f.Hout + c.ho0 + py) * f.Wout + c.wo0 + px)) * f.G +
+                              static_cast<size_t>(c.gsub) * p.GS;
+    *count = (row_runs ? c.nw * f.G : p.GS) * 3 * f.KK;
+    return reinterpret_cast<const unsigned char*>(om + first_unit * 3 * f.KK);
+}
+
+// Warp 0 queues every copy of tile t into buffer `buf` on `bar`: the window
+// (one TMA load) and the record runs (one bulk copy each, widened to 16-byte
+// boundaries when that stays inside the offset_mask tensor, else the aligned
+// middle by bulk copy and the ragged ends by plain stores).
+template <typename T>
+__device__ __forceinline__ void issue_tile(const TileParams& p, const CUtensorMap* xmap, const T* om, unsigned t,
+                                           unsigned char* buf, uint64_t* bar, int lane) {
     constexpr int E = sizeof(T);
-    const uintptr_t a = reinterpret_cast<uintptr_t>(src);
-    const int shift = static_cast<int>(a & 15);
-    const int nbytes = count * E;
-    int head = (16 - shift) & 15;
-    if (head > nbytes) head = nbytes;
-    const int mid = (nbytes - head) & ~15;
-    const unsigned char* s = reinterpret_cast<const unsigned char*>(src);
-    unsigned char* d = slot + shift;
-    if (mid > 0) bulk_g2s_counted(d + head, s + head, static_cast<unsigned>(mid), bar);
-    for (int i = 0; i < head / E; ++i) reinterpret_cast<T*>(d)[i] = src[i];
-    for (int i = (head + mid) / E; i < count; ++i) reinterpret_cast<T*>(d)[i] = src[i];
+    const TileCoord c = tile_coord(p, t);
+    const bool row_runs = p.GS == p.f.G;
+    const int nruns = row_runs ? c.nh : c.nh * c.nw;
+    for (int r = lane; r < nruns; r += 32) {
+        int count;
+        const unsigned char* s = run_src<T>(p, c, om, r, &count);
+        const unsigned long long a = reinterpret_cast<unsigned long long>(s);
+        const unsigned long long b = a + static_cast<unsigned long long>(count) * E;
+        const unsigned long long a16 = a & ~15ull, b16 = (b + 15) & ~15ull;
+        unsigned char* slot = buf + r * p.run_slot;  // byte a lands at slot + (a & 15)
+        if (a16 >= p.om_lo && b16 <= p.om_hi) {
+            bulk_g2s_counted(slot, reinterpret_cast<const void*>(a16), static_cast<unsigned>(b16 - a16), bar);
+        } else {
+            const unsigned long long ma = (a + 15) & ~15ull, mb = b & ~15ull;
+            if (mb > ma)
+                bulk_g2s_counted(slot + (ma - a16), reinterpret_cast<const void*>(ma), static_cast<unsigned>(mb - ma),
+                                 bar);
+            const T* src = reinterpret_cast<const T*>(s);
+            T* dst = reinterpret_cast<T*>(slot + (a & 15));
+            const int head = mb > ma ? static_cast<int>((ma - a) / E) : count;
+            for (int i = 0; i < head; ++i) dst[i] = src[i];
+            if (mb > ma)
+                for (int i = static_cast<int>((mb - a) / E); i < count; ++i) dst[i] = src[i];
+        }
+    }
+    if (lane == 0) {
+        mbar_expect_tx(bar, static_cast<unsigned>(p.WH * p.WW * p.PB));
+        tma_load_5d(buf + p.rec_bytes, xmap, 0, c.gsub * p.cblk, c.wx0, c.wy0, c.n, bar);
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar);  // the single arrival; the phase completes with the last byte
 }
 
 // ------------------------------------------------------------ the kernel ---
 
+// Warp roles: warps 0 .. nc-1 consume (gather), warp nc produces (issues the
+// copies). Two buffers form a ring; buffer b has a "full" barrier (one
+// producer arrival plus the copied bytes) and an "empty" barrier (one arrival
+// per consumer warp once it is done with the tile). No CTA-wide barrier is
+// taken after the set-up, so a warp held up by a global-memory gather does not
+// stall the others. Every wait is bounded; a wait that gives up sets the
+// device status word and the warp leaves (the producer after letting its
+// copies in flight land).
 template <typename T, int Q, int KS>
-__global__ void __launch_bounds__(256, 2)
-fwd_window_kernel(const T* __restrict__ x, const T* __restrict__ om, T* __restrict__ out, WinParams p) {
+__global__ void __launch_bounds__(544, 1)
+fwd_tile_kernel(const __grid_constant__ CUtensorMap xmap, const T* __restrict__ x, const T* __restrict__ om,
+                T* __restrict__ out, TileParams p) {
     extern __shared__ __align__(128) unsigned char smem[];
-    __shared__ __align__(8) uint64_t bar;
+    __shared__ __align__(8) uint64_t full_bar[2];
+    __shared__ __align__(8) uint64_t empty_bar[2];
     constexpr int E = sizeof(T);
     constexpr int CH = 16 / E;  // channels per 16-byte chunk
     const FwdParams& f = p.f;
     const int K = KS > 0 ? KS : f.K;
     const int KK = K * K;
     const int R3 = 3 * KK;
-    const int tid = threadIdx.x;
-    const int nthr = blockDim.x;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int nc = static_cast<int>(blockDim.x >> 5) - 1;  // consumer warps
+    const bool row_runs = p.GS == f.G;
 
-    // tile of this CTA
-    const unsigned b = blockIdx.x;
-    const unsigned b1 = fdiv(b, p.div_nsub);
-    const int gsub = static_cast<int>(b - b1 * p.nsub);
-    const unsigned b2 = fdiv(b1, p.div_tx);
-    const int tx = static_cast<int>(b1 - b2 * p.tiles_x);
-    const unsigned n_ = fdiv(b2, p.div_ty);
-    const int ty = static_cast<int>(b2 - n_ * p.tiles_y);
-    const int n = static_cast<int>(n_);
-    const int ho0 = ty * p.TH, wo0 = tx * p.TW;
-    const int nh = min(p.TH, f.Hout - ho0), nw = min(p.TW, f.Wout - wo0);
-    const int wy0 = ho0 * f.stride - f.pad - p.R;   // window origin in image coordinates
-    const int wx0 = wo0 * f.stride - f.pad - p.R;
-    unsigned char* win = smem + p.win_off;
-    const bool row_runs = p.GS == f.G;              // the CTA owns all groups of its pixels
-    const int nruns = row_runs ? nh : nh * nw;
-
-    if (tid == 0) mbar_init(&bar, 1);
+    if (tid == 0) {
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&full_bar[b], 1);
+            mbar_init(&empty_bar[b], static_cast<unsigned>(nc));
+        }
+        fence_barrier_init();
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&xmap)) : "memory");
+    }
     __syncthreads();
+    const int first = static_cast<int>(blockIdx.x);
+    if (first >= p.tiles) return;
+    const int ntiles = (p.tiles - first + static_cast<int>(gridDim.x) - 1) / static_cast<int>(gridDim.x);
 
-    // 1. window rows: the in-image part of each row arrives by bulk copy (one
-    //    per row, or one per pixel when the CTA owns a subset of the groups);
-    //    the rest of the window is zeroed
-    const size_t pix_bytes = static_cast<size_t>(f.C) * E;
-    const unsigned char* xn = reinterpret_cast<const unsigned char*>(x) +
-                              static_cast<size_t>(n) * f.H * f.W * pix_bytes + static_cast<size_t>(gsub) * p.PB;
-    const int xs = max(0, wx0), xe = min(f.W, wx0 + p.WW);  // in-image columns [xs, xe)
-    const int ncols = xe - xs;
-    if (row_runs) {
-        for (int wy = tid; wy < p.WH; wy += nthr) {
-            const int y = wy0 + wy;
-            if (y >= 0 && y < f.H && ncols > 0)
-                bulk_g2s_counted(win + (wy * p.WW + (xs - wx0)) * p.PB, xn + (static_cast<size_t>(y) * f.W + xs) * pix_bytes,
-                                 static_cast<unsigned>(ncols * p.PB), &bar);
-        }
-    } else {
-        const int npix = p.WH * max(ncols, 0);
-        for (int i = tid; i < npix; i += nthr) {
-            const int wy = i / ncols, c = i - (i / ncols) * ncols;
-            const int y = wy0 + wy;
-            if (y >= 0 && y < f.H)
-                bulk_g2s_counted(win + (wy * p.WW + (xs - wx0) + c) * p.PB,
-                                 xn + (static_cast<size_t>(y) * f.W + xs + c) * pix_bytes, static_cast<unsigned>(p.PB),
-                                 &bar);
-        }
-    }
-    if (wy0 < 0 || wy0 + p.WH > f.H || ncols < p.WW) {
-        // zero the out-of-image part of the window (edge tiles only): whole
-        // rows above/below the image, the column margins elsewhere
-        const int cpp = p.PB >> 4;
-        const int rowq = p.WW * cpp;
-        const int left = ncols > 0 ? (xs - wx0) * cpp : rowq;
-        const int right0 = ncols > 0 ? (xe - wx0) * cpp : rowq;
-        const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-        for (int wy = 0; wy < p.WH; ++wy) {
-            uint4* row = reinterpret_cast<uint4*>(win) + wy * rowq;
-            const int y = wy0 + wy;
-            if (y < 0 || y >= f.H) {
-                for (int i = tid; i < rowq; i += nthr) row[i] = z;
-            } else {
-                for (int i = tid; i < left; i += nthr) row[i] = z;
-                for (int i = right0 + tid; i < rowq; i += nthr) row[i] = z;
+    if (warp == nc) {
+        // ---------------------------------------------------------------- producer
+        for (int i = 0; i < ntiles; ++i) {
+            const int b = i & 1;
+            if (i >= 2) {
+                const bool ok = mbar_wait_bounded(&empty_bar[b], ((i >> 1) - 1) & 1, kCopyWaitLimitNs);
+                if (!__all_sync(0xffffffffu, ok)) {
+                    if (lane == 0) atomicOr(&g_device_status, kStatusCopyTimeout);
+                    // let the copies already queued land before leaving
+                    for (int j = max(0, i - 2); j < i; ++j)
+                        mbar_wait_bounded(&full_bar[j & 1], (j >> 1) & 1, kCopyWaitLimitNs);
+                    return;
+                }
             }
+            fence_proxy_async();  // the consumers' reads of buffer b before the async writes
+            issue_tile<T>(p, &xmap, om, static_cast<unsigned>(first + i * static_cast<int>(gridDim.x)),
+                          smem + b * p.buf_bytes, &full_bar[b], lane);
         }
-    }
-    // 2. the tile's offset/mask records: one run per tile row when the CTA owns
-    //    all groups (contiguous in memory), else one run per pixel
-    for (int r = tid; r < nruns; r += nthr) {
-        const int py = row_runs ? r : r / nw;
-        const int px = row_runs ? 0 : r - py * nw;
-        const size_t first_unit =
-            (static_cast<size_t>((n * f.Hout + ho0 + py) * f.Wout + wo0 + px)) * f.G + gsub * p.GS;
-        const int count = (row_runs ? nw * f.G : p.GS) * R3;
-        stage_bytes<T>(om + first_unit * R3, count, smem + r * p.run_slot, &bar);
-    }
-    __syncthreads();                  // every expect_tx is posted
-    if (tid == 0) mbar_arrive(&bar);  // the single arrival: the phase completes with the last byte
-    if (!mbar_wait_bounded(&bar, 0, kCopyWaitLimitNs)) {
-        atomicOr(&g_device_status, kStatusCopyTimeout);
-        mbar_wait_bounded(&bar, 0, kCopyWaitLimitNs);  // let copies in flight land before leaving
         return;
     }
-    __syncthreads();                  // the plain stores (zeros, record edges) too
 
-    // 3. gather
-    const int q8 = tid & 7;
+    // -------------------------------------------------------------------- consumers
+    const int q8 = lane & 7;
     int rot = 0;
     if constexpr (Q == 2) rot = q8 >> 2;
     if constexpr (Q == 4) rot = q8 >> 1;
     if constexpr (Q == 8) rot = q8;
+    int choff[Q];
+#pragma unroll
+    for (int j = 0; j < Q; ++j) {
+        int c = rot + j;
+        if (c >= Q) c -= Q;
+        choff[j] = c;
+    }
     const int rowB = p.WW * p.PB;
     const float wymax = static_cast<float>(p.WH - 2), wxmax = static_cast<float>(p.WW - 2);
     const int rowC = f.W * f.C;
-    const T* ximg = x + static_cast<size_t>(n) * f.H * rowC;
+    const float fdil = static_cast<float>(f.dilation);
 
-    for (int u = tid; u < p.units; u += nthr) {
-        const unsigned py_ = fdiv(static_cast<unsigned>(u), p.div_tw_gs);
-        const int rem = u - static_cast<int>(py_) * p.TW * p.GS;
-        const unsigned px_ = fdiv(static_cast<unsigned>(rem), p.div_gs);
-        const int gl = rem - static_cast<int>(px_) * p.GS;
-        const int py = static_cast<int>(py_), px = static_cast<int>(px_);
-        if (py >= nh || px >= nw) continue;
-        const int ho = ho0 + py, wo = wo0 + px, g = gsub * p.GS + gl;
-
-        // this unit's record in shared memory
-        const size_t first_unit =
-            row_runs ? (static_cast<size_t>((n * f.Hout + ho) * f.Wout + wo0)) * f.G
-                     : (static_cast<size_t>((n * f.Hout + ho) * f.Wout + wo)) * f.G + gsub * p.GS;
-        const int run = row_runs ? py : py * nw + px;
-        const int within = row_runs ? (px * f.G + g) : gl;
-        const uintptr_t ga = reinterpret_cast<uintptr_t>(om + first_unit * R3);
-        const T* rec = reinterpret_cast<const T*>(smem + run * p.run_slot + (ga & 15)) + within * R3;
-
-        // chunk j of this thread is channel chunk (rot + j) mod Q of the unit
-        int choff[Q];
-#pragma unroll
-        for (int j = 0; j < Q; ++j) {
-            int c = rot + j;
-            if (c >= Q) c -= Q;
-            choff[j] = c;
+    for (int i = 0; i < ntiles; ++i) {
+        const unsigned t = static_cast<unsigned>(first + i * static_cast<int>(gridDim.x));
+        const int b = i & 1;
+        const unsigned char* buf = smem + b * p.buf_bytes;
+        const bool ok = mbar_wait_bounded(&full_bar[b], (i >> 1) & 1, kCopyWaitLimitNs);
+        if (!__all_sync(0xffffffffu, ok)) {
+            if (lane == 0) atomicOr(&g_device_status, kStatusCopyTimeout);
+            return;
         }
-        const unsigned char* ubase = win + gl * (Q * 16);
-        float2 acc[Q][CH / 2];
-#pragma unroll
-        for (int j = 0; j < Q; ++j)
-#pragma unroll
-            for (int i = 0; i < CH / 2; ++i) acc[j][i] = make_float2(0.f, 0.f);
 
-        const int by = ho * f.stride - f.pad;  // grid row of ky = 0 (image coordinates)
-        const int bx = wo * f.stride - f.pad;
-        const float fwy = static_cast<float>(by - wy0), fwx = static_cast<float>(bx - wx0);
-        const float fdil = static_cast<float>(f.dilation);
+        const TileCoord c = tile_coord(p, t);
+        const unsigned char* win = buf + p.rec_bytes;
+        const T* ximg = x + static_cast<size_t>(c.n) * f.H * rowC;
+
+        for (int u = warp * 32 + lane; u < p.units; u += nc * 32) {
+            const unsigned py_ = fdiv(static_cast<unsigned>(u), p.div_tw_gs);
+            const int rem = u - static_cast<int>(py_) * p.TW * p.GS;
+            const unsigned px_ = fdiv(static_cast<unsigned>(rem), p.div_gs);
+            const int gl = rem - static_cast<int>(px_) * p.GS;
+            const int py = static_cast<int>(py_), px = static_cast<int>(px_);
+            if (py >= c.nh || px >= c.nw) continue;
+            const int ho = c.ho0 + py, wo = c.wo0 + px, g = c.gsub * p.GS + gl;
+
+            // this unit's record in shared memory
+            const int run = row_runs ? py : py * c.nw + px;
+            int count;
+            const unsigned long long ra = reinterpret_cast<unsigned long long>(run_src<T>(p, c, om, run, &count));
+            const int within = row_runs ? (px * f.G + g) : gl;
+            const T* rec = reinterpret_cast<const T*>(buf + run * p.run_slot + (ra & 15)) + within * R3;
+
+            const unsigned char* ubase = win + gl * (Q * 16);
+            float2 acc[Q][CH / 2];
+#pragma unroll
+            for (int j = 0; j < Q; ++j)
+#pragma unroll
+                for (int q = 0; q < CH / 2; ++q) acc[j][q] = make_float2(0.f, 0.f);
+
+            const int by = ho * f.stride - f.pad;  // grid row of ky = 0 (image coordinates)
+            const int bx = wo * f.stride - f.pad;
+            const float fwy = static_cast<float>(by - c.wy0), fwx = static_cast<float>(bx - c.wx0);
+            unsigned long long slow = 0ull;  // points left for the global-memory pass (K*K <= 64)
 
 #pragma unroll (KS > 0 ? KS * KS : 1)
-        for (int k = 0; k < KK; ++k) {
-            const int ky = k / K, kx = k - (k / K) * K;
-            const float rx = ElemTraits<T>::to_float(rec[k]);
-            const float ry = ElemTraits<T>::to_float(rec[KK + k]);
-            const float m = ElemTraits<T>::to_float(rec[2 * KK + k]);
-            const float dy = __fmul_rn(f.offset_scale, ry);
-            const float dx = __fmul_rn(f.offset_scale, rx);
-            const float fy0 = floorf(dy), fx0 = floorf(dx);
-            const float ly = dy - fy0, lx = dx - fx0;
-            // window-relative top-left corner (exact: every term is a small integer)
-            const float wyf = fy0 + (fwy + static_cast<float>(ky) * fdil);
-            const float wxf = fx0 + (fwx + static_cast<float>(kx) * fdil);
-            const float wy0w = 1.f - ly, wx0w = 1.f - lx;
-            const float a0 = m * wy0w, a1 = m * ly;
-            if (wyf >= 0.f && wyf <= wymax && wxf >= 0.f && wxf <= wxmax && fabsf(m) < INFINITY) {
-                // all four corners inside the window; outside-image corners read
-                // the window's zeros and the finite weight adds exactly 0
-                const float w00 = a0 * wx0w, w01 = a0 * lx, w10 = a1 * wx0w, w11 = a1 * lx;
-                const int off = (static_cast<int>(wyf) * p.WW + static_cast<int>(wxf)) * p.PB;
-                const unsigned char* pb = ubase + off;
+            for (int k = 0; k < KK; ++k) {
+                const int ky = k / K, kx = k - (k / K) * K;
+                const float rx = ElemTraits<T>::to_float(rec[k]);
+                const float ry = ElemTraits<T>::to_float(rec[KK + k]);
+                const float m = ElemTraits<T>::to_float(rec[2 * KK + k]);
+                const float dy = __fmul_rn(f.offset_scale, ry);
+                const float dx = __fmul_rn(f.offset_scale, rx);
+                const float fy0 = floorf(dy), fx0 = floorf(dx);
+                // window-relative top-left corner (exact: every term is a small integer)
+                const float wyf = fy0 + (fwy + static_cast<float>(ky) * fdil);
+                const float wxf = fx0 + (fwx + static_cast<float>(kx) * fdil);
+                if (wyf >= 0.f && wyf <= wymax && wxf >= 0.f && wxf <= wxmax && fabsf(m) < INFINITY) {
+                    // all four corners inside the window; outside-image corners read
+                    // the window's zeros and the finite weight adds exactly 0
+                    const float ly = dy - fy0, lx = dx - fx0;
+                    const float a0 = m * (1.f - ly), a1 = m * ly;
+                    const float w00 = a0 * (1.f - lx), w01 = a0 * lx, w10 = a1 * (1.f - lx), w11 = a1 * lx;
+                    const int off = (static_cast<int>(wyf) * p.WW + static_cast<int>(wxf)) * p.PB;
+                    const unsigned char* pb = ubase + off;
 #pragma unroll
-                for (int j = 0; j < Q; ++j) {
-                    const unsigned char* pc = pb + (choff[j] << 4);
-                    const uint4 v00 = *reinterpret_cast<const uint4*>(pc);
-                    const uint4 v01 = *reinterpret_cast<const uint4*>(pc + p.PB);
-                    const uint4 v10 = *reinterpret_cast<const uint4*>(pc + rowB);
-                    const uint4 v11 = *reinterpret_cast<const uint4*>(pc + rowB + p.PB);
-                    fma_chunk<T>(acc[j], w00, v00);
-                    fma_chunk<T>(acc[j], w01, v01);
-                    fma_chunk<T>(acc[j], w10, v10);
-                    fma_chunk<T>(acc[j], w11, v11);
+                    for (int j = 0; j < Q; ++j) {
+                        const unsigned char* pc = pb + (choff[j] << 4);
+                        const uint4 v00 = *reinterpret_cast<const uint4*>(pc);
+                        const uint4 v01 = *reinterpret_cast<const uint4*>(pc + p.PB);
+                        const uint4 v10 = *reinterpret_cast<const uint4*>(pc + rowB);
+                        const uint4 v11 = *reinterpret_cast<const uint4*>(pc + rowB + p.PB);
+                        fma_chunk<T>(acc[j], w00, v00);
+                        fma_chunk<T>(acc[j], w01, v01);
+                        fma_chunk<T>(acc[j], w10, v10);
+                        fma_chunk<T>(acc[j], w11, v11);
+                    }
+                } else {
+                    slow |= 1ull << k;
                 }
-            } else {
-                // global gather with per-corner validity
-                const int p0y = by + ky * f.dilation, p0x = bx + kx * f.dilation;
-                const Sample s = locate(p0y, p0x, ry, rx, f.offset_scale, f.H, f.W);
+            }
+            // the points outside the window: global gather with per-corner validity
+            while (slow) {
+                const int k = __ffsll(static_cast<long long>(slow)) - 1;
+                slow &= slow - 1ull;
+                const int ky = k / K, kx = k - (k / K) * K;
+                const float rx = ElemTraits<T>::to_float(rec[k]);
+                const float ry = ElemTraits<T>::to_float(rec[KK + k]);
+                const float m = ElemTraits<T>::to_float(rec[2 * KK + k]);
+                const Sample s = locate(by + ky * f.dilation, bx + kx * f.dilation, ry, rx, f.offset_scale, f.H, f.W);
                 if (s.bits == 0u) continue;
+                const float a0 = m * (1.f - s.ly), a1 = m * s.ly;
                 float w[4];
-                w[0] = (s.bits & 1u) ? a0 * wx0w : 0.f;
-                w[1] = (s.bits & 2u) ? a0 * lx : 0.f;
-                w[2] = (s.bits & 4u) ? a1 * wx0w : 0.f;
-                w[3] = (s.bits & 8u) ? a1 * lx : 0.f;
+                w[0] = (s.bits & 1u) ? a0 * (1.f - s.lx) : 0.f;
+                w[1] = (s.bits & 2u) ? a0 * s.lx : 0.f;
+                w[2] = (s.bits & 4u) ? a1 * (1.f - s.lx) : 0.f;
+                w[3] = (s.bits & 8u) ? a1 * s.lx : 0.f;
                 const T* c00 = ximg + (s.y0 * f.W + s.x0) * f.C + g * f.Cg;
 #pragma unroll
                 for (int cn = 0; cn < 4; ++cn) {
@@ -380,20 +440,22 @@ fwd_window_kernel(const T* __restrict__ x, const T* __restrict__ om, T* __restri
                     const T* pc = c00 + (cn >> 1) * rowC + (cn & 1) * f.C;
 #pragma unroll
                     for (int j = 0; j < Q; ++j) {
-                        uint32_t t[4];
-                        load_vec<16>(pc + choff[j] * CH, t);
-                        fma_chunk<T>(acc[j], w[cn], make_uint4(t[0], t[1], t[2], t[3]));
+                        uint32_t tt[4];
+                        load_vec<16>(pc + choff[j] * CH, tt);
+                        fma_chunk<T>(acc[j], w[cn], make_uint4(tt[0], tt[1], tt[2], tt[3]));
                     }
                 }
             }
-        }
 
-        T* o = out + (static_cast<size_t>((n * f.Hout + ho) * f.Wout + wo)) * f.C + g * f.Cg;
+            T* o = out + (static_cast<size_t>((c.n * f.Hout + ho) * f.Wout + wo)) * f.C + g * f.Cg;
 #pragma unroll
-        for (int j = 0; j < Q; ++j) {
-            const uint4 v = pack_chunk<T>(acc[j]);
-            *reinterpret_cast<uint4*>(o + choff[j] * CH) = v;
+            for (int j = 0; j < Q; ++j) {
+                const uint4 v = pack_chunk<T>(acc[j]);
+                *reinterpret_cast<uint4*>(o + choff[j] * CH) = v;
+            }
         }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty_bar[b]);  // this warp is done with buffer b
     }
 }
 
@@ -404,6 +466,7 @@ __global__ void selftest_wait_timeout_kernel(unsigned long long limit_ns) {
     __shared__ __align__(8) uint64_t bar;
     if (threadIdx.x == 0) {
         mbar_init(&bar, 1);
+        fence_barrier_init();
         mbar_expect_tx(&bar, 16);
         mbar_arrive(&bar);
         if (!mbar_wait_bounded(&bar, 0, limit_ns)) atomicOr(&g_device_status, kStatusSelftestTimeout);
