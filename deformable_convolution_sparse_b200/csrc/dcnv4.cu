@@ -226,9 +226,16 @@ bool plan_tile(const void* x, const void* om, const void* out, const FwdParams& 
     return true;
 }
 
-template <typename T, int Q, int KS>
+// fp16 storage: weights rounded to fp16 for the mixed-precision FMA (default)
+// or kept in fp32 (DCNV4_F16_EXACT=1, for comparisons).
+bool f16_exact_from_env() {
+    const char* v = std::getenv("DCNV4_F16_EXACT");
+    return v && *v == '1';
+}
+
+template <typename T, int Q, int KS, bool HW>
 int launch_tile_q(const T* x, const T* om, T* out, const TilePlan& plan, cudaStream_t stream) {
-    auto kern = dcnv4::fwd_tile_kernel<T, Q, KS>;
+    auto kern = dcnv4::fwd_tile_kernel<T, Q, KS, HW>;
     static std::once_flag once;
     static cudaError_t attr = cudaSuccess;
     std::call_once(once, [&] {
@@ -244,10 +251,18 @@ int launch_tile_q(const T* x, const T* om, T* out, const TilePlan& plan, cudaStr
     return launch_status();
 }
 
+template <typename T, int Q, bool HW>
+int launch_tile_k(const T* x, const T* om, T* out, const TilePlan& plan, cudaStream_t s) {
+    if (plan.p.f.K == 3) return launch_tile_q<T, Q, 3, HW>(x, om, out, plan, s);
+    return launch_tile_q<T, Q, 0, HW>(x, om, out, plan, s);
+}
+
 template <typename T, int Q>
 int launch_tile_k(const T* x, const T* om, T* out, const TilePlan& plan, cudaStream_t s) {
-    if (plan.p.f.K == 3) return launch_tile_q<T, Q, 3>(x, om, out, plan, s);
-    return launch_tile_q<T, Q, 0>(x, om, out, plan, s);
+    if constexpr (std::is_same<T, __half>::value) {
+        if (!f16_exact_from_env()) return launch_tile_k<T, Q, true>(x, om, out, plan, s);
+    }
+    return launch_tile_k<T, Q, false>(x, om, out, plan, s);
 }
 
 template <typename T>

@@ -151,9 +151,27 @@ constexpr uint64_t kCopyWaitLimitNs = 1000000000ull;  // 1 s
 
 // ------------------------------------------------------------ chunk math ---
 
-// fp32 FMA of one 16-byte chunk (16/sizeof(T) channels) into acc (pairs)
-template <typename T>
+// Accumulates w * x over one 16-byte chunk (16/sizeof(T) channels) into acc
+// (pairs of fp32 accumulators).
+//  - HW (fp16 storage only): the weight is rounded once to fp16 and each
+//    fp16 x fp16 product, exact in fp32, is added to the fp32 accumulator by
+//    one mixed-precision FMA (fma.rn.f32.f16): no conversion of x and no
+//    register pairing, which halves the FMA-pipe work per channel.
+//  - otherwise: x is widened to fp32 and multiplied by the fp32 weight with
+//    packed fp32x2 FMAs.
+template <typename T, bool HW = false>
 __device__ __forceinline__ void fma_chunk(float2* acc, float w, const uint4& v) {
+    if constexpr (HW && std::is_same<T, __half>::value) {
+        const unsigned short wh = __half_as_ushort(__float2half_rn(w));
+        const uint32_t vw[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            asm("{\n\t.reg .f16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+                "fma.rn.f32.f16 %0, lo, %3, %0;\n\tfma.rn.f32.f16 %1, hi, %3, %1;\n\t}"
+                : "+f"(acc[q].x), "+f"(acc[q].y)
+                : "r"(vw[q]), "h"(wh));
+        return;
+    }
     const float2 ww = make_float2(w, w);
     if constexpr (sizeof(T) == 4) {
         acc[0] = __ffma2_rn(ww, make_float2(__uint_as_float(v.x), __uint_as_float(v.y)), acc[0]);
@@ -270,7 +288,7 @@ __device__ __forceinline__ void issue_tile(const TileParams& p, const CUtensorMa
 // stall the others. Every wait is bounded; a wait that gives up sets the
 // device status word and the warp leaves (the producer after letting its
 // copies in flight land).
-template <typename T, int Q, int KS>
+template <typename T, int Q, int KS, bool HW>
 __global__ void __launch_bounds__(544, 1)
 fwd_tile_kernel(const __grid_constant__ CUtensorMap xmap, const T* __restrict__ x, const T* __restrict__ om,
                 T* __restrict__ out, TileParams p) {
@@ -408,10 +426,10 @@ fwd_tile_kernel(const __grid_constant__ CUtensorMap xmap, const T* __restrict__ 
                         const uint4 v01 = *reinterpret_cast<const uint4*>(pc + p.PB);
                         const uint4 v10 = *reinterpret_cast<const uint4*>(pc + rowB);
                         const uint4 v11 = *reinterpret_cast<const uint4*>(pc + rowB + p.PB);
-                        fma_chunk<T>(acc[j], w00, v00);
-                        fma_chunk<T>(acc[j], w01, v01);
-                        fma_chunk<T>(acc[j], w10, v10);
-                        fma_chunk<T>(acc[j], w11, v11);
+                        fma_chunk<T, HW>(acc[j], w00, v00);
+                        fma_chunk<T, HW>(acc[j], w01, v01);
+                        fma_chunk<T, HW>(acc[j], w10, v10);
+                        fma_chunk<T, HW>(acc[j], w11, v11);
                     }
                 } else {
                     slow |= 1ull << k;
@@ -442,7 +460,7 @@ fwd_tile_kernel(const __grid_constant__ CUtensorMap xmap, const T* __restrict__ 
                     for (int j = 0; j < Q; ++j) {
                         uint32_t tt[4];
                         load_vec<16>(pc + choff[j] * CH, tt);
-                        fma_chunk<T>(acc[j], w[cn], make_uint4(tt[0], tt[1], tt[2], tt[3]));
+                        fma_chunk<T, HW>(acc[j], w[cn], make_uint4(tt[0], tt[1], tt[2], tt[3]));
                     }
                 }
             }

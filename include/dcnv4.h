@@ -23,9 +23,12 @@
  * (y0+a, x0+b), y0 = p0y + floor(dy), x0 = p0x + floor(dx), a,b in {0,1},
  * weighted (a ? fy : 1-fy) * (b ? fx : 1-fx), fy = dy - floor(dy),
  * fx = dx - floor(dx). Corners inside the image always take part (also with
- * weight 0); a non-finite offset puts the whole sample outside. Products and
- * sums are fp32; the result is rounded once (round-to-nearest-even) to the
- * storage type.
+ * weight 0); a non-finite offset puts the whole sample outside. The corner
+ * weight m * (1-fy or fy) * (1-fx or fx) is computed in fp32. For fp32 and
+ * bf16 storage it multiplies x in fp32; for fp16 storage it is rounded once to
+ * fp16 and the fp16 x fp16 product, exact in fp32, is accumulated by a
+ * mixed-precision FMA. Sums are fp32; the result is rounded once
+ * (round-to-nearest-even) to the storage type.
  *
  * Layouts (all contiguous, row-major, caller-owned DEVICE memory unless
  * stated otherwise):

@@ -1,0 +1,60 @@
+"""GPU tests of dcnv4_forward_host: inputs and result in host memory, the
+device buffers only as staging, the copies and kernels pipelined over image
+chunks. The result must equal the device-resident forward bit for bit."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import deformable_convolution_sparse_b200 as dcn
+from deformable_convolution_sparse_b200.workloads import WORKLOADS, make_inputs, workload_inputs
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("pinned", [True, False])
+@pytest.mark.parametrize("N", [1, 3, 8, 11])
+def test_host_path_equals_device_path(N, pinned, cuda_device):
+    x, om = make_inputs(N, 17, 19, 64, 4, 3, 17, 19, "f16", ("normal", 0, 1.5), ("normal", 0, 0.5), seed=N)
+    if pinned:
+        x, om = x.pin_memory(), om.pin_memory()
+    out = dcn.forward_host(x, om, G=4, K=3, pad=1, device=cuda_device)
+    ref = dcn.forward(x.to(cuda_device), om.to(cuda_device), G=4, K=3, pad=1).cpu()
+    assert torch.equal(out, ref)
+
+
+def test_host_path_full_workload_against_oracle(cuda_device):
+    w = WORKLOADS["stage1_f16"]
+    x, om = workload_inputs(w)
+    out = dcn.forward_host(x.pin_memory(), om.pin_memory(), device=cuda_device, **w.kwargs())
+    ref = oracle.dcnv4_forward(x.double().numpy(), om.double().numpy(), **w.kwargs())
+    err = np.abs(out.double().numpy() - ref).max()
+    assert err <= 4e-3 * np.abs(ref).max()
+
+
+def test_host_path_reuses_caller_staging_and_orders_after_stream_work(cuda_device):
+    x, om = make_inputs(4, 9, 9, 32, 2, 3, 9, 9, "f32", seed=3)
+    staging = (torch.full_like(x, 7.0, device=cuda_device), torch.full_like(om, 7.0, device=cuda_device),
+               torch.full((4, 9, 9, 32), 7.0, device=cuda_device))
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        torch.cuda._sleep(1_000_000)  # queued work the call must come after
+        out = dcn.forward_host(x.pin_memory(), om.pin_memory(), G=2, K=3, pad=1, staging=staging, stream=s)
+    ref = oracle.dcnv4_forward(x.double().numpy(), om.double().numpy(), G=2, K=3, pad=1)
+    assert np.abs(out.double().numpy() - ref).max() <= 1e-5 * np.abs(ref).max()
+    assert torch.equal(staging[0].cpu(), x) and torch.equal(staging[2].cpu(), out)
+
+
+def test_host_path_rejects_bad_arguments(cuda_device):
+    lib = dcn.load_library()
+    x = torch.zeros(2, 8, 8, 16).pin_memory()
+    om = torch.zeros(2, 8, 8, 2, 27).pin_memory()
+    out = torch.zeros(2, 8, 8, 16).pin_memory()
+    xd, omd, od = x.to(cuda_device), om.to(cuda_device), out.to(cuda_device)
+    args = (2, 8, 8, 16, 2, 3, 1, 1, 1, 1.0, 0, None)
+    assert lib.dcnv4_forward_host(0, om.data_ptr(), out.data_ptr(), xd.data_ptr(), omd.data_ptr(), od.data_ptr(),
+                                  *args) == dcn.STATUS["DCNV4_ERR_NULL"]
+    assert lib.dcnv4_forward_host(x.data_ptr(), om.data_ptr(), x.data_ptr(), xd.data_ptr(), omd.data_ptr(),
+                                  od.data_ptr(), *args) == dcn.STATUS["DCNV4_ERR_ALIAS"]
+    assert lib.dcnv4_forward_host(x.data_ptr(), om.data_ptr(), out.data_ptr(), xd.data_ptr(), omd.data_ptr(),
+                                  xd.data_ptr(), *args) == dcn.STATUS["DCNV4_ERR_ALIAS"]

@@ -23,15 +23,18 @@ TOL = {"f32": 1e-5, "f16": 4e-3, "bf16": 4e-3}
 TD = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}
 
 
-@pytest.fixture(params=["window", "gather"])
+@pytest.fixture(params=["window", "window_f16exact", "gather"])
 def variant(request, monkeypatch):
-    """Both kernels: the shared-memory window kernel (default choice) and the
-    global-gather kernel (forced with DCNV4_VARIANT=gather, also the window
-    kernel's path for samples outside its window)."""
+    """Every kernel path: the shared-memory tile kernel (default choice; for
+    fp16 storage with fp16-rounded weights), the same kernel with fp32 weights
+    for fp16 (DCNV4_F16_EXACT=1), and the global-gather kernel (forced with
+    DCNV4_VARIANT=gather)."""
+    monkeypatch.delenv("DCNV4_VARIANT", raising=False)
+    monkeypatch.delenv("DCNV4_F16_EXACT", raising=False)
     if request.param == "gather":
         monkeypatch.setenv("DCNV4_VARIANT", "gather")
-    else:
-        monkeypatch.delenv("DCNV4_VARIANT", raising=False)
+    elif request.param == "window_f16exact":
+        monkeypatch.setenv("DCNV4_F16_EXACT", "1")
     return request.param
 
 
@@ -284,3 +287,22 @@ def test_bounded_wait_selftest_sets_status_and_context_survives(cuda_device):
 def test_no_copy_timeouts_during_the_parity_runs(cuda_device):
     st = dcn.device_status(clear=True)
     assert not st & dcn.binding.DEVSTATUS_COPY_TIMEOUT
+
+
+@pytest.mark.parametrize("name", ["stage1_f16", "stage3_f16", "sd_latent_f16"])
+def test_fp16_weight_rounding_stays_far_inside_the_tolerance(name, monkeypatch, cuda_device):
+    """fp16 storage: the default path rounds each bilinear weight to fp16
+    before the exact fp16 x fp16 product; its error against the oracle must
+    stay a small fraction of the 4e-3 * max|out| bar, and close to the error of
+    the fp32-weight path."""
+    w = WORKLOADS[name]
+    x, om = workload_inputs(w)
+    ref = oracle.dcnv4_forward(x.double().numpy(), om.double().numpy(), **w.kwargs())
+    scale = np.abs(ref).max()
+    errs = {}
+    for exact in ("0", "1"):
+        monkeypatch.setenv("DCNV4_F16_EXACT", exact)
+        out = dcn.forward(x.to(cuda_device), om.to(cuda_device), **w.kwargs())
+        errs[exact] = np.abs(out.double().cpu().numpy() - ref).max() / scale
+    assert errs["0"] <= 1e-3, errs        # a quarter of the 4e-3 bar
+    assert errs["0"] <= 2.0 * errs["1"] + 2e-4, errs
