@@ -21,14 +21,14 @@ DCNV4_OK = 0
 STATUS_NAMES = {
     0: "DCNV4_OK", 1: "DCNV4_ERR_NULL", 2: "DCNV4_ERR_SHAPE", 3: "DCNV4_ERR_GROUPS",
     4: "DCNV4_ERR_DTYPE", 5: "DCNV4_ERR_ALIGN", 6: "DCNV4_ERR_ALIAS", 7: "DCNV4_ERR_SCALE",
-    8: "DCNV4_ERR_TOO_LARGE", 9: "DCNV4_ERR_LAUNCH", 10: "DCNV4_ERR_CUDA",
+    8: "DCNV4_ERR_TOO_LARGE", 9: "DCNV4_ERR_LAUNCH", 10: "DCNV4_ERR_CUDA", 11: "DCNV4_ERR_STAGING",
 }
 STATUS = {v: k for k, v in STATUS_NAMES.items()}
 TORCH_DTYPE = {torch.float32: DCNV4_F32, torch.float16: DCNV4_F16, torch.bfloat16: DCNV4_BF16}
 
 # every symbol include/dcnv4.h declares
 EXPORTS = ("dcnv4_output_shape", "dcnv4_validate", "dcnv4_forward", "dcnv4_sampling_index",
-           "dcnv4_forward_host", "dcnv4_device_status", "dcnv4_selftest_wait_timeout", "dcnv4_strerror",
+           "dcnv4_forward_host", "dcnv4_forward_host_noalloc", "dcnv4_device_status", "dcnv4_selftest_wait_timeout", "dcnv4_strerror",
            "dcnv4_abi_version")
 DEVSTATUS_COPY_TIMEOUT, DEVSTATUS_SELFTEST_TIMEOUT = 1, 2
 
@@ -63,6 +63,8 @@ def load_library():
     lib.dcnv4_sampling_index.restype = i
     lib.dcnv4_forward_host.argtypes = [p] * 6 + [i] * 9 + [f, i, p]
     lib.dcnv4_forward_host.restype = i
+    lib.dcnv4_forward_host_noalloc.argtypes = [p] * 3 + [i] * 9 + [f, i, p]
+    lib.dcnv4_forward_host_noalloc.restype = i
     lib.dcnv4_device_status.argtypes = [ctypes.POINTER(ctypes.c_uint), i]
     lib.dcnv4_device_status.restype = i
     lib.dcnv4_selftest_wait_timeout.argtypes = [ctypes.c_ulonglong, p]
@@ -210,6 +212,44 @@ def forward_host(x: torch.Tensor, offset_mask: torch.Tensor, G: int, K: int, str
         if rc != DCNV4_OK:
             raise DCNv4Error(rc, "dcnv4_forward_host")
         (stream or torch.cuda.current_stream()).synchronize()
+    return out
+
+
+NOALLOC_STAGING_BYTES = 32 << 20
+
+
+def forward_host_noalloc(x: torch.Tensor, offset_mask: torch.Tensor, G: int, K: int, stride: int = 1,
+                         pad: int = 0, dilation: int = 1, offset_scale: float = 1.0,
+                         out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Forward from host tensors through ``dcnv4_forward_host_noalloc``.
+
+    For callers that must not allocate device memory at call time: the
+    library stages through its own fixed 32 MiB device array per GPU (shared
+    by every call on that GPU; calls that overlap on the GPU race on it). The
+    output tensor is allocated on the host here when not given; pass ``out``
+    to allocate nothing at all. Returns ``out`` once the work is complete.
+    """
+    for t, name in ((x, "x"), (offset_mask, "offset_mask")):
+        if t.device.type != "cpu" or not t.is_contiguous() or t.dtype not in TORCH_DTYPE:
+            raise ValueError(f"{name} must be a contiguous CPU tensor of a supported dtype")
+    if offset_mask.dtype != x.dtype:
+        raise ValueError("offset_mask must match x in dtype")
+    N, H, W, C = x.shape
+    Hout, Wout = output_shape(H, W, K, stride, pad, dilation)
+    if tuple(offset_mask.shape) != (N, Hout, Wout, G, 3 * K * K):
+        raise ValueError("offset_mask has the wrong shape")
+    if out is None:
+        out = torch.empty((N, Hout, Wout, C), dtype=x.dtype, pin_memory=x.is_pinned())
+    if tuple(out.shape) != (N, Hout, Wout, C) or out.dtype != x.dtype or out.device.type != "cpu" \
+            or not out.is_contiguous():
+        raise ValueError("out must be a contiguous CPU tensor of the output shape and x's dtype")
+    handle = _stream_handle(stream)
+    rc = load_library().dcnv4_forward_host_noalloc(x.data_ptr(), offset_mask.data_ptr(), out.data_ptr(), N, H, W,
+                                                   C, G, K, stride, pad, dilation, float(offset_scale),
+                                                   TORCH_DTYPE[x.dtype], handle)
+    if rc != DCNV4_OK:
+        raise DCNv4Error(rc, "dcnv4_forward_host_noalloc")
+    (stream or torch.cuda.current_stream()).synchronize()
     return out
 
 

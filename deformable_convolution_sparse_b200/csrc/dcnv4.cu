@@ -392,6 +392,7 @@ const char* dcnv4_strerror(int status) {
         case DCNV4_ERR_TOO_LARGE: return "an element count reaches 2^31";
         case DCNV4_ERR_LAUNCH: return "kernel launch failed";
         case DCNV4_ERR_CUDA: return "CUDA runtime call failed";
+        case DCNV4_ERR_STAGING: return "one image does not fit half of the static staging area";
         default: return "unknown status";
     }
 }
@@ -583,3 +584,103 @@ int dcnv4_sampling_index(const void* offset_mask, int32_t* corner, uint8_t* vali
 }
 
 }  // extern "C"
+
+// --------------------------------------------------------------------------
+// Allocation-free host entry point: staging in a fixed device array.
+
+namespace {
+
+__device__ __align__(256) unsigned char g_noalloc_staging[DCNV4_NOALLOC_STAGING_BYTES];
+
+unsigned char* g_noalloc_addr[kMaxDevices];
+std::mutex g_noalloc_mutex;
+
+// Device address of the staging array on the current device, looked up once
+// per device (cudaGetSymbolAddress with that device current).
+int noalloc_staging(unsigned char** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DCNV4_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (!g_noalloc_addr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_staging) != cudaSuccess || !p) return DCNV4_ERR_CUDA;
+        g_noalloc_addr[dev] = static_cast<unsigned char*>(p);
+    }
+    *out = g_noalloc_addr[dev];
+    return DCNV4_OK;
+}
+
+size_t round256(size_t b) { return (b + 255) / 256 * 256; }
+
+}  // namespace
+
+extern "C" int dcnv4_forward_host_noalloc(const void* x_host, const void* offset_mask_host, void* out_host,
+                                          int N, int H, int W, int C, int G, int K,
+                                          int stride, int pad, int dilation, float offset_scale, int dtype,
+                                          void* stream) {
+    // the host buffers get the checks the device buffers get elsewhere
+    int rc = dcnv4_validate(x_host, offset_mask_host, out_host, N, H, W, C, G, K, stride, pad, dilation,
+                            offset_scale, dtype);
+    if (rc) return rc;
+    if (N == 0) return DCNV4_OK;
+    int Hout = 0, Wout = 0;
+    dcnv4_output_shape(H, W, K, stride, pad, dilation, &Hout, &Wout);
+    const size_t e = static_cast<size_t>(elem_size(dtype));
+    const size_t x_img = static_cast<size_t>(H) * W * C * e;
+    const size_t om_img = static_cast<size_t>(Hout) * Wout * G * 3 * K * K * e;
+    const size_t out_img = static_cast<size_t>(Hout) * Wout * C * e;
+    const size_t half = DCNV4_NOALLOC_STAGING_BYTES / 2;
+    // images per chunk: x, offset_mask and out of the chunk, each 256-byte aligned, in one half
+    int per_chunk = 0;
+    while (per_chunk < N && round256((per_chunk + 1) * x_img) + round256((per_chunk + 1) * om_img) +
+                                    round256((per_chunk + 1) * out_img) <= half)
+        ++per_chunk;
+    if (per_chunk == 0) return DCNV4_ERR_STAGING;
+
+    unsigned char* staging = nullptr;
+    rc = noalloc_staging(&staging);
+    if (rc) return rc;
+    HostPipe* pipe = nullptr;
+    rc = host_pipe(&pipe);
+    if (rc) return rc;
+    cudaStream_t user = static_cast<cudaStream_t>(stream);
+    cudaEvent_t ev_start = nullptr, ev_done[2] = {nullptr, nullptr};
+    auto release = [&](int code) {
+        if (ev_start) cudaEventDestroy(ev_start);
+        for (auto& ev : ev_done)
+            if (ev) cudaEventDestroy(ev);
+        return code;
+    };
+    if (cudaEventCreateWithFlags(&ev_start, cudaEventDisableTiming) != cudaSuccess) return release(DCNV4_ERR_CUDA);
+    for (auto& ev : ev_done)
+        if (cudaEventCreateWithFlags(&ev, cudaEventDisableTiming) != cudaSuccess) return release(DCNV4_ERR_CUDA);
+    if (cudaEventRecord(ev_start, user) != cudaSuccess) return release(DCNV4_ERR_CUDA);
+    for (int i = 0; i < 2; ++i)
+        if (cudaStreamWaitEvent(pipe->s[i], ev_start, 0) != cudaSuccess) return release(DCNV4_ERR_CUDA);
+
+    const char* xh = static_cast<const char*>(x_host);
+    const char* omh = static_cast<const char*>(offset_mask_host);
+    char* oh = static_cast<char*>(out_host);
+    int c = 0;
+    for (int n0 = 0; n0 < N; n0 += per_chunk, ++c) {
+        const int nc = std::min(per_chunk, N - n0);
+        // chunk c uses half c & 1 on stream c & 1: a half is reused only by a
+        // later chunk of the same stream, after this chunk's copies are done
+        unsigned char* xd = staging + (c & 1) * half;
+        unsigned char* omd = xd + round256(nc * x_img);
+        unsigned char* od = omd + round256(nc * om_img);
+        cudaStream_t s = pipe->s[c & 1];
+        if (cudaMemcpyAsync(xd, xh + n0 * x_img, nc * x_img, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+            cudaMemcpyAsync(omd, omh + n0 * om_img, nc * om_img, cudaMemcpyHostToDevice, s) != cudaSuccess)
+            return release(DCNV4_ERR_CUDA);
+        rc = dcnv4_forward(xd, omd, od, nc, H, W, C, G, K, stride, pad, dilation, offset_scale, dtype, s);
+        if (rc) return release(rc);
+        if (cudaMemcpyAsync(oh + n0 * out_img, od, nc * out_img, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+            return release(DCNV4_ERR_CUDA);
+    }
+    for (int i = 0; i < 2; ++i) {
+        if (cudaEventRecord(ev_done[i], pipe->s[i]) != cudaSuccess || cudaStreamWaitEvent(user, ev_done[i], 0) != cudaSuccess)
+            return release(DCNV4_ERR_CUDA);
+    }
+    return release(DCNV4_OK);
+}

@@ -90,7 +90,9 @@ typedef enum {
     DCNV4_ERR_SCALE = 7,     /* offset_scale is NaN or infinite                         */
     DCNV4_ERR_TOO_LARGE = 8, /* an element count reaches 2^31                           */
     DCNV4_ERR_LAUNCH = 9,    /* the kernel launch failed (CUDA error after launch)      */
-    DCNV4_ERR_CUDA = 10      /* a CUDA runtime call other than a launch failed          */
+    DCNV4_ERR_CUDA = 10,     /* a CUDA runtime call other than a launch failed          */
+    DCNV4_ERR_STAGING = 11   /* dcnv4_forward_host_noalloc: one image does not fit its  */
+                             /* half of the library's static staging area               */
 } dcnv4_status_t;
 
 #define DCNV4_MAX_K 16
@@ -160,6 +162,38 @@ DCNV4_API int dcnv4_forward_host(const void *x_host, const void *offset_mask_hos
                                  int N, int H, int W, int C, int G, int K,
                                  int stride, int pad, int dilation, float offset_scale, int dtype,
                                  void *stream);
+
+/* Allocation-free variant of dcnv4_forward_host (the pages have no
+ * counterpart: this is a service of this library). Some callers cannot
+ * allocate device memory when they call us: a serving process that handed all
+ * free GPU memory to its own pool at start-up (a fresh cudaMalloc would fail or
+ * fragment that budget), or a latency-critical path where cudaMalloc/cudaFree
+ * may synchronise the device and stall other streams. They can use this entry
+ * point, which takes only the host buffers: it stages through a fixed device
+ * array inside the library, DCNV4_NOALLOC_STAGING_BYTES (32 MiB) per GPU,
+ * allocated when the library's device code is loaded on that GPU and kept
+ * until the process exits. It never calls cudaMalloc, cudaFree or an
+ * allocating library routine.
+ *   - The array is split into two halves; the batch is processed in chunks of
+ *     whole images, each chunk's x, offset_mask and out (each rounded up to
+ *     256 bytes) in one half. A batch whose single image does not fit in one
+ *     half (16 MiB) is rejected with DCNV4_ERR_STAGING before anything is
+ *     queued.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current) and keeps it; make that
+ *     first call before any stream capture on the device.
+ *   - Every call on a device shares the one array and it keeps the last call's
+ *     contents; nothing in it needs to start at zero (inputs are copied in
+ *     whole, the output is written in whole). Calls whose work overlaps on the
+ *     GPU race on the array: queue them on one stream, or order them.
+ *   - Ordering, streams and the other checks are those of dcnv4_forward_host
+ *     (the host pointers are checked for NULL, alignment and overlap); the
+ *     result is in out_host once `stream` reaches the end of the call's work. */
+#define DCNV4_NOALLOC_STAGING_BYTES (32u << 20)
+DCNV4_API int dcnv4_forward_host_noalloc(const void *x_host, const void *offset_mask_host, void *out_host,
+                                         int N, int H, int W, int C, int G, int K,
+                                         int stride, int pad, int dilation, float offset_scale, int dtype,
+                                         void *stream);
 
 /* Device-side status word of the current device (bit flags below). The
  * shared-memory window kernel waits for its bulk copies with a time limit
