@@ -237,10 +237,25 @@ __device__ __forceinline__ const unsigned char* run_src(const TileParams& p, con
     return reinterpret_cast<const unsigned char*>(om + first_unit * 3 * f.KK);
 }
 
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(smem_dst)), "l"(gsrc) : "memory");
+}
+// one arrival on `bar` once every cp.async this thread issued before has landed
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+// Arrivals the "full" barrier of a buffer waits for: the producer's lane 0,
+// plus every producer lane's cp.async arrival when the records are per pixel.
+__host__ __device__ __forceinline__ unsigned full_arrivals(bool row_runs) { return row_runs ? 1u : 33u; }
+
 // Warp 0 queues every copy of tile t into buffer `buf` on `bar`: the window
-// (one TMA load) and the record runs (one bulk copy each, widened to 16-byte
-// boundaries when that stays inside the offset_mask tensor, else the aligned
-// middle by bulk copy and the ragged ends by plain stores).
+// (one TMA load) and the record runs, widened to 16-byte boundaries when that
+// stays inside the offset_mask tensor (else the aligned middle is copied and
+// the ragged ends by plain stores). A tile row's records are one run and go by
+// one bulk copy (cp.async.bulk). When the CTA owns only some of the groups the
+// runs are per pixel and short; those go by 16-byte cp.async from all 32 lanes
+// (a bulk copy costs the TMA unit tens of cycles each, too many for 100+ runs).
 template <typename T>
 __device__ __forceinline__ void issue_tile(const TileParams& p, const CUtensorMap* xmap, const T* om, unsigned t,
                                            unsigned char* buf, uint64_t* bar, int lane) {
@@ -248,7 +263,33 @@ __device__ __forceinline__ void issue_tile(const TileParams& p, const CUtensorMa
     const TileCoord c = tile_coord(p, t);
     const bool row_runs = p.GS == p.f.G;
     const int nruns = row_runs ? c.nh : c.nh * c.nw;
-    for (int r = lane; r < nruns; r += 32) {
+    if (!row_runs) {
+        for (int r = lane; r < nruns; r += 32) {
+            int count;
+            const unsigned char* s = run_src<T>(p, c, om, r, &count);
+            const unsigned long long a = reinterpret_cast<unsigned long long>(s);
+            const unsigned long long b = a + static_cast<unsigned long long>(count) * E;
+            unsigned long long a16 = a & ~15ull, b16 = (b + 15) & ~15ull;
+            unsigned char* slot = buf + r * p.run_slot;  // byte a lands at slot + (a & 15)
+            const bool inside = a16 >= p.om_lo && b16 <= p.om_hi;
+            if (!inside) {
+                // the ragged ends by plain copies, the aligned middle below
+                const unsigned long long ma = (a + 15) & ~15ull, mb = b & ~15ull;
+                const T* src = reinterpret_cast<const T*>(s);
+                T* dst = reinterpret_cast<T*>(slot + (a & 15));
+                const int head = mb > ma ? static_cast<int>((ma - a) / E) : count;
+                for (int i = 0; i < head; ++i) dst[i] = src[i];
+                if (mb > ma)
+                    for (int i = static_cast<int>((mb - a) / E); i < count; ++i) dst[i] = src[i];
+                a16 = ma;
+                b16 = mb > ma ? mb : ma;
+            }
+            for (unsigned long long q = a16; q < b16; q += 16)
+                cp_async16(slot + (q - (a & ~15ull)), reinterpret_cast<const void*>(q));
+        }
+        cp_async_arrive_noinc(bar);
+    }
+    for (int r = lane; row_runs && r < nruns; r += 32) {
         int count;
         const unsigned char* s = run_src<T>(p, c, om, r, &count);
         const unsigned long long a = reinterpret_cast<unsigned long long>(s);
@@ -307,7 +348,7 @@ fwd_tile_kernel(const __grid_constant__ CUtensorMap xmap, const T* __restrict__ 
 
     if (tid == 0) {
         for (int b = 0; b < 2; ++b) {
-            mbar_init(&full_bar[b], 1);
+            mbar_init(&full_bar[b], full_arrivals(row_runs));
             mbar_init(&empty_bar[b], static_cast<unsigned>(nc));
         }
         fence_barrier_init();
