@@ -116,7 +116,8 @@ bool plan_tile(const void* x, const void* om, const void* out, const FwdParams& 
     if (f.KK > 64) return false;  // the per-unit mask of points outside the window has 64 bits
     int R = 5;
     if (const char* h = std::getenv("DCNV4_HALO")) R = std::atoi(h) > 0 ? std::atoi(h) : R;
-    int forceTH = 0, forceTW = 0, forceGS = 0;
+    int forceTH = 0, forceTW = 0, forceGS = 0, forceNrec = 0;
+    if (const char* n = std::getenv("DCNV4_NREC")) forceNrec = (std::atoi(n) == 2 || std::atoi(n) == 3) ? std::atoi(n) : 0;
     if (const char* t = std::getenv("DCNV4_TILE")) std::sscanf(t, "%dx%d", &forceTH, &forceTW);
     if (const char* g = std::getenv("DCNV4_GS")) forceGS = std::atoi(g);
     const int R3 = 3 * f.KK;
@@ -155,27 +156,37 @@ bool plan_tile(const void* x, const void* om, const void* out, const FwdParams& 
                 const int slot = (count * E + 32 + 15) / 16 * 16;
                 const size_t rec = (static_cast<size_t>(nruns) * slot + 127) / 128 * 128;
                 const size_t win = (static_cast<size_t>(WH) * WW * PB + 127) / 128 * 128;
-                const size_t smem = 2 * (rec + win);
+                // records get a third buffer (a longer lead for their DRAM reads) when it fits
+                int nrec = (2 * win + 3 * rec <= kTileSmemLimit) ? 3 : 2;
+                if (forceNrec) nrec = forceNrec;
+                const size_t smem = 2 * win + nrec * rec;
                 if (smem > kTileSmemLimit) continue;
                 const int threads = (units + 31) / 32 * 32 + 32;  // consumers + the producer warp
                 const int tiles_y = (f.Hout + TH - 1) / TH, tiles_x = (f.Wout + TW - 1) / TW;
                 const long long tiles = static_cast<long long>(f.N) * tiles_y * tiles_x * (f.G / GS);
+                // the choice must not depend on N: an image's result (which samples take
+                // the window path) then never depends on the batch it comes in. The wave
+                // balance is judged for a nominal batch of 64 images.
+                const long long tiles_nominal = 64LL * tiles_y * tiles_x * (f.G / GS);
                 const int per_sm = std::max(1, static_cast<int>(std::min<size_t>(
                                                    (kTileSmemLimit + 2048) / (smem + 1024), 2048 / threads)));
                 const double slots = static_cast<double>(nsm) * per_sm;
-                const double waves = static_cast<double>(tiles) / slots;
+                const double waves = static_cast<double>(tiles_nominal) / slots;
                 const double balance = waves / std::ceil(waves);
                 const double useful =
                     static_cast<double>(f.Hout) * f.Wout / (static_cast<double>(tiles_y) * TH * tiles_x * TW);
                 const double reuse = static_cast<double>(TH * TW) / (static_cast<double>(WH) * WW);
                 const double fill = static_cast<double>(units) / (threads - 32);
-                const double occ = std::min(1.0, per_sm * (threads - 32) / 512.0);
-                const double score = useful * balance * fill * occ * banks * std::sqrt(reuse);
+                const double occ = std::min(1.0, per_sm * (threads - 32) / 384.0);
+                const double depth = nrec == 3 ? 1.0 : 0.9;
+                // a ragged tile loses threads and still loads a full window: useful counts twice
+                const double score = useful * useful * balance * fill * occ * banks * depth * std::sqrt(reuse);
                 if (score > best) {
                     best = score;
                     bp.TH = TH; bp.TW = TW; bp.tiles_x = tiles_x; bp.tiles_y = tiles_y;
                     bp.WH = WH; bp.WW = WW; bp.run_slot = slot; bp.rec_bytes = static_cast<int>(rec);
-                    bp.buf_bytes = static_cast<int>(rec + win);
+                    bp.win_bytes = static_cast<int>(win);
+                    bp.nrec = nrec;
                     bp.tiles = static_cast<int>(tiles); bp.units = units;
                     bp.GS = GS; bp.PB = PB; bp.cblk = sub_ch / c2;
                     best_threads = threads;
@@ -220,9 +231,9 @@ bool plan_tile(const void* x, const void* om, const void* out, const FwdParams& 
     if (const char* d = std::getenv("DCNV4_DEBUG"); d && *d == '1')
         std::fprintf(stderr,
                      "dcnv4 tile plan: tile %dx%d GS %d (nsub %d) R %d window %dx%d PB %d cblk %d tiles %d units %d "
-                     "threads %d smem %zu\n",
+                     "threads %d nrec %d smem %zu\n",
                      bp.TH, bp.TW, GS, bp.nsub, R, bp.WH, bp.WW, PB, bp.cblk, bp.tiles, bp.units, best_threads,
-                     best_smem);
+                     bp.nrec, best_smem);
     return true;
 }
 
@@ -233,9 +244,9 @@ bool f16_exact_from_env() {
     return v && *v == '1';
 }
 
-template <typename T, int Q, int KS, bool HW>
+template <typename T, int Q, int KS, bool HW, int PBC>
 int launch_tile_q(const T* x, const T* om, T* out, const TilePlan& plan, cudaStream_t stream) {
-    auto kern = dcnv4::fwd_tile_kernel<T, Q, KS, HW>;
+    auto kern = dcnv4::fwd_tile_kernel<T, Q, KS, HW, PBC>;
     static std::once_flag once;
     static cudaError_t attr = cudaSuccess;
     std::call_once(once, [&] {
@@ -253,8 +264,15 @@ int launch_tile_q(const T* x, const T* om, T* out, const TilePlan& plan, cudaStr
 
 template <typename T, int Q, bool HW>
 int launch_tile_k(const T* x, const T* om, T* out, const TilePlan& plan, cudaStream_t s) {
-    if (plan.p.f.K == 3) return launch_tile_q<T, Q, 3, HW>(x, om, out, plan, s);
-    return launch_tile_q<T, Q, 0, HW>(x, om, out, plan, s);
+    // a 128-byte window pixel (the common case) as a compile-time stride
+    if constexpr (Q != 5) {
+        if (plan.p.PB == 128) {
+            if (plan.p.f.K == 3) return launch_tile_q<T, Q, 3, HW, 128>(x, om, out, plan, s);
+            return launch_tile_q<T, Q, 0, HW, 128>(x, om, out, plan, s);
+        }
+    }
+    if (plan.p.f.K == 3) return launch_tile_q<T, Q, 3, HW, 0>(x, om, out, plan, s);
+    return launch_tile_q<T, Q, 0, HW, 0>(x, om, out, plan, s);
 }
 
 template <typename T, int Q>

@@ -74,8 +74,9 @@ struct TileParams {
     int tiles;              // N * tiles_y * tiles_x * nsub
     int units;              // TH * TW * GS
     int run_slot;           // shared bytes per record run
-    int rec_bytes;          // record area of one buffer (multiple of 128)
-    int buf_bytes;          // one buffer: records + window (multiple of 128)
+    int rec_bytes;          // one record buffer (multiple of 128)
+    int win_bytes;          // one window buffer (multiple of 128)
+    int nrec;               // record buffers (2 or 3); windows always use 2
     unsigned long long om_lo, om_hi;  // byte range of the offset_mask tensor
     FastDiv div_tw_gs, div_gs, div_nsub, div_tx, div_ty;
 };
@@ -245,97 +246,110 @@ __device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
     asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 
-// Arrivals the "full" barrier of a buffer waits for: the producer's lane 0,
-// plus every producer lane's cp.async arrival when the records are per pixel.
-__host__ __device__ __forceinline__ unsigned full_arrivals(bool row_runs) { return row_runs ? 1u : 33u; }
+// Arrivals the records' "full" barrier waits for: the producer's lane 0, plus
+// every producer lane's cp.async arrival when the records are per pixel.
+__host__ __device__ __forceinline__ unsigned rec_full_arrivals(bool row_runs) { return row_runs ? 1u : 33u; }
 
-// Warp 0 queues every copy of tile t into buffer `buf` on `bar`: the window
-// (one TMA load) and the record runs, widened to 16-byte boundaries when that
-// stays inside the offset_mask tensor (else the aligned middle is copied and
-// the ragged ends by plain stores). A tile row's records are one run and go by
-// one bulk copy (cp.async.bulk). When the CTA owns only some of the groups the
-// runs are per pixel and short; those go by 16-byte cp.async from all 32 lanes
-// (a bulk copy costs the TMA unit tens of cycles each, too many for 100+ runs).
+// Producer warp: queues the copies of tile t's offset/mask records into `buf`
+// on `bar`. Runs are widened to 16-byte boundaries when that stays inside the
+// offset_mask tensor (else the aligned middle is copied and the ragged ends by
+// plain stores). A tile row's records are one run and go by one bulk copy
+// (cp.async.bulk). When the CTA owns only some of the groups the runs are per
+// pixel and short; those go by 16-byte cp.async from all 32 lanes (a bulk copy
+// costs the TMA unit tens of cycles each, too many for 100+ runs).
 template <typename T>
-__device__ __forceinline__ void issue_tile(const TileParams& p, const CUtensorMap* xmap, const T* om, unsigned t,
-                                           unsigned char* buf, uint64_t* bar, int lane) {
+__device__ __forceinline__ void issue_records(const TileParams& p, const T* om, const TileCoord& c,
+                                              unsigned char* buf, uint64_t* bar, int lane) {
     constexpr int E = sizeof(T);
-    const TileCoord c = tile_coord(p, t);
     const bool row_runs = p.GS == p.f.G;
     const int nruns = row_runs ? c.nh : c.nh * c.nw;
-    if (!row_runs) {
-        for (int r = lane; r < nruns; r += 32) {
-            int count;
-            const unsigned char* s = run_src<T>(p, c, om, r, &count);
-            const unsigned long long a = reinterpret_cast<unsigned long long>(s);
-            const unsigned long long b = a + static_cast<unsigned long long>(count) * E;
-            unsigned long long a16 = a & ~15ull, b16 = (b + 15) & ~15ull;
-            unsigned char* slot = buf + r * p.run_slot;  // byte a lands at slot + (a & 15)
-            const bool inside = a16 >= p.om_lo && b16 <= p.om_hi;
-            if (!inside) {
-                // the ragged ends by plain copies, the aligned middle below
-                const unsigned long long ma = (a + 15) & ~15ull, mb = b & ~15ull;
-                const T* src = reinterpret_cast<const T*>(s);
-                T* dst = reinterpret_cast<T*>(slot + (a & 15));
-                const int head = mb > ma ? static_cast<int>((ma - a) / E) : count;
-                for (int i = 0; i < head; ++i) dst[i] = src[i];
-                if (mb > ma)
-                    for (int i = static_cast<int>((mb - a) / E); i < count; ++i) dst[i] = src[i];
-                a16 = ma;
-                b16 = mb > ma ? mb : ma;
-            }
-            for (unsigned long long q = a16; q < b16; q += 16)
-                cp_async16(slot + (q - (a & ~15ull)), reinterpret_cast<const void*>(q));
-        }
-        cp_async_arrive_noinc(bar);
-    }
-    for (int r = lane; row_runs && r < nruns; r += 32) {
+    for (int r = lane; r < nruns; r += 32) {
         int count;
         const unsigned char* s = run_src<T>(p, c, om, r, &count);
         const unsigned long long a = reinterpret_cast<unsigned long long>(s);
         const unsigned long long b = a + static_cast<unsigned long long>(count) * E;
-        const unsigned long long a16 = a & ~15ull, b16 = (b + 15) & ~15ull;
+        unsigned long long a16 = a & ~15ull, b16 = (b + 15) & ~15ull;
         unsigned char* slot = buf + r * p.run_slot;  // byte a lands at slot + (a & 15)
-        if (a16 >= p.om_lo && b16 <= p.om_hi) {
-            bulk_g2s_counted(slot, reinterpret_cast<const void*>(a16), static_cast<unsigned>(b16 - a16), bar);
-        } else {
+        if (!(a16 >= p.om_lo && b16 <= p.om_hi)) {
+            // the ragged ends by plain copies, the aligned middle below
             const unsigned long long ma = (a + 15) & ~15ull, mb = b & ~15ull;
-            if (mb > ma)
-                bulk_g2s_counted(slot + (ma - a16), reinterpret_cast<const void*>(ma), static_cast<unsigned>(mb - ma),
-                                 bar);
             const T* src = reinterpret_cast<const T*>(s);
             T* dst = reinterpret_cast<T*>(slot + (a & 15));
             const int head = mb > ma ? static_cast<int>((ma - a) / E) : count;
             for (int i = 0; i < head; ++i) dst[i] = src[i];
             if (mb > ma)
                 for (int i = static_cast<int>((mb - a) / E); i < count; ++i) dst[i] = src[i];
+            a16 = ma;
+            b16 = mb > ma ? mb : ma;
+        }
+        if (b16 <= a16) continue;
+        unsigned char* d = slot + (a16 - (a & ~15ull));
+        if (row_runs) {
+            bulk_g2s_counted(d, reinterpret_cast<const void*>(a16), static_cast<unsigned>(b16 - a16), bar);
+        } else {
+            for (unsigned long long q = a16; q < b16; q += 16) cp_async16(d + (q - a16), reinterpret_cast<const void*>(q));
         }
     }
+    if (!row_runs) cp_async_arrive_noinc(bar);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar);
+}
+
+// Producer warp, lane 0: the window of tile t as one TMA load on `bar`.
+__device__ __forceinline__ void issue_window(const TileParams& p, const CUtensorMap* xmap, const TileCoord& c,
+                                             unsigned char* buf, uint64_t* bar, int lane) {
     if (lane == 0) {
         mbar_expect_tx(bar, static_cast<unsigned>(p.WH * p.WW * p.PB));
-        tma_load_5d(buf + p.rec_bytes, xmap, 0, c.gsub * p.cblk, c.wx0, c.wy0, c.n, bar);
+        tma_load_5d(buf, xmap, 0, c.gsub * p.cblk, c.wx0, c.wy0, c.n, bar);
+        mbar_arrive(bar);
     }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(bar);  // the single arrival; the phase completes with the last byte
+}
+
+// Two fp32 weights to a pair of fp16 (round to nearest even), one instruction.
+__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
+    __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// acc += w * x over one fp16 chunk with mixed-precision FMAs; `w2` holds the
+// fp16 weight in its low (hi == false) or high half.
+template <bool HI>
+__device__ __forceinline__ void fma_chunk_h(float2* acc, uint32_t w2, const uint4& v) {
+    const uint32_t vw[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        if constexpr (HI)
+            asm("{\n\t.reg .f16 lo, hi, wl, wh;\n\tmov.b32 {lo, hi}, %2;\n\tmov.b32 {wl, wh}, %3;\n\t"
+                "fma.rn.f32.f16 %0, lo, wh, %0;\n\tfma.rn.f32.f16 %1, hi, wh, %1;\n\t}"
+                : "+f"(acc[q].x), "+f"(acc[q].y)
+                : "r"(vw[q]), "r"(w2));
+        else
+            asm("{\n\t.reg .f16 lo, hi, wl, wh;\n\tmov.b32 {lo, hi}, %2;\n\tmov.b32 {wl, wh}, %3;\n\t"
+                "fma.rn.f32.f16 %0, lo, wl, %0;\n\tfma.rn.f32.f16 %1, hi, wl, %1;\n\t}"
+                : "+f"(acc[q].x), "+f"(acc[q].y)
+                : "r"(vw[q]), "r"(w2));
+    }
 }
 
 // ------------------------------------------------------------ the kernel ---
 
 // Warp roles: warps 0 .. nc-1 consume (gather), warp nc produces (issues the
-// copies). Two buffers form a ring; buffer b has a "full" barrier (one
-// producer arrival plus the copied bytes) and an "empty" barrier (one arrival
-// per consumer warp once it is done with the tile). No CTA-wide barrier is
-// taken after the set-up, so a warp held up by a global-memory gather does not
-// stall the others. Every wait is bounded; a wait that gives up sets the
-// device status word and the warp leaves (the producer after letting its
-// copies in flight land).
-template <typename T, int Q, int KS, bool HW>
+// copies). Windows use a ring of 2 buffers, records a ring of p.nrec (2 or 3):
+// records come from DRAM on first touch and get the longer lead. Every buffer
+// has a "full" barrier (producer arrivals plus the copied bytes) and an
+// "empty" barrier (one arrival per consumer warp once it is done with the
+// tile). No CTA-wide barrier is taken after the set-up, so a warp held up by a
+// global-memory gather does not stall the others. Every wait is bounded; a
+// wait that gives up sets the device status word and the warp leaves (the
+// producer after letting its copies in flight land).
+//
+// PBC: the window's pixel stride as a compile-time constant (0: p.PB).
+template <typename T, int Q, int KS, bool HW, int PBC>
 __global__ void __launch_bounds__(544, 1)
 fwd_tile_kernel(const __grid_constant__ CUtensorMap xmap, const T* __restrict__ x, const T* __restrict__ om,
                 T* __restrict__ out, TileParams p) {
     extern __shared__ __align__(128) unsigned char smem[];
-    __shared__ __align__(8) uint64_t full_bar[2];
-    __shared__ __align__(8) uint64_t empty_bar[2];
+    __shared__ __align__(8) uint64_t win_full[2], win_empty[2], rec_full[3], rec_empty[3];
     constexpr int E = sizeof(T);
     constexpr int CH = 16 / E;  // channels per 16-byte chunk
     const FwdParams& f = p.f;
@@ -345,11 +359,19 @@ fwd_tile_kernel(const __grid_constant__ CUtensorMap xmap, const T* __restrict__ 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int nc = static_cast<int>(blockDim.x >> 5) - 1;  // consumer warps
     const bool row_runs = p.GS == f.G;
+    const int nrec = p.nrec;
+    const int PB = PBC ? PBC : p.PB;
+    unsigned char* const winbuf = smem;                          // 2 windows
+    unsigned char* const recbuf = smem + 2 * p.win_bytes;        // nrec record sets
 
     if (tid == 0) {
         for (int b = 0; b < 2; ++b) {
-            mbar_init(&full_bar[b], full_arrivals(row_runs));
-            mbar_init(&empty_bar[b], static_cast<unsigned>(nc));
+            mbar_init(&win_full[b], 1);
+            mbar_init(&win_empty[b], static_cast<unsigned>(nc));
+        }
+        for (int b = 0; b < 3; ++b) {
+            mbar_init(&rec_full[b], rec_full_arrivals(row_runs));
+            mbar_init(&rec_empty[b], static_cast<unsigned>(nc));
         }
         fence_barrier_init();
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&xmap)) : "memory");
@@ -357,30 +379,49 @@ fwd_tile_kernel(const __grid_constant__ CUtensorMap xmap, const T* __restrict__ 
     __syncthreads();
     const int first = static_cast<int>(blockIdx.x);
     if (first >= p.tiles) return;
-    const int ntiles = (p.tiles - first + static_cast<int>(gridDim.x) - 1) / static_cast<int>(gridDim.x);
+    const int stride_t = static_cast<int>(gridDim.x);
+    const int ntiles = (p.tiles - first + stride_t - 1) / stride_t;
 
     if (warp == nc) {
         // ---------------------------------------------------------------- producer
-        for (int i = 0; i < ntiles; ++i) {
-            const int b = i & 1;
-            if (i >= 2) {
-                const bool ok = mbar_wait_bounded(&empty_bar[b], ((i >> 1) - 1) & 1, kCopyWaitLimitNs);
-                if (!__all_sync(0xffffffffu, ok)) {
-                    if (lane == 0) atomicOr(&g_device_status, kStatusCopyTimeout);
-                    // let the copies already queued land before leaving
-                    for (int j = max(0, i - 2); j < i; ++j)
-                        mbar_wait_bounded(&full_bar[j & 1], (j >> 1) & 1, kCopyWaitLimitNs);
-                    return;
-                }
+        // step i: the records of tile i and the window of tile i - (nrec - 2), each
+        // once the consumers are done with the buffer it reuses
+        const int lead = nrec - 2;
+        for (int i = 0; i < ntiles + lead; ++i) {
+            bool ok = true;
+            if (i < ntiles && i >= nrec)
+                ok = mbar_wait_bounded(&rec_empty[i % nrec], ((i / nrec) - 1) & 1, kCopyWaitLimitNs);
+            const int j = i - lead;
+            if (ok && j >= 2 && j < ntiles)
+                ok = mbar_wait_bounded(&win_empty[j & 1], ((j >> 1) - 1) & 1, kCopyWaitLimitNs);
+            if (!__all_sync(0xffffffffu, ok)) {
+                if (lane == 0) atomicOr(&g_device_status, kStatusCopyTimeout);
+                // let the copies already queued land before leaving
+                for (int q = max(0, i - nrec); q < min(i, ntiles); ++q)
+                    mbar_wait_bounded(&rec_full[q % nrec], (q / nrec) & 1, kCopyWaitLimitNs);
+                for (int q = max(0, j - 2); q < min(j, ntiles); ++q)
+                    mbar_wait_bounded(&win_full[q & 1], (q >> 1) & 1, kCopyWaitLimitNs);
+                return;
             }
-            fence_proxy_async();  // the consumers' reads of buffer b before the async writes
-            issue_tile<T>(p, &xmap, om, static_cast<unsigned>(first + i * static_cast<int>(gridDim.x)),
-                          smem + b * p.buf_bytes, &full_bar[b], lane);
+            fence_proxy_async();  // the consumers' reads of those buffers before the async writes
+            if (i < ntiles)
+                issue_records<T>(p, om, tile_coord(p, static_cast<unsigned>(first + i * stride_t)),
+                                 recbuf + (i % nrec) * p.rec_bytes, &rec_full[i % nrec], lane);
+            if (j >= 0 && j < ntiles)
+                issue_window(p, &xmap, tile_coord(p, static_cast<unsigned>(first + j * stride_t)),
+                             winbuf + (j & 1) * p.win_bytes, &win_full[j & 1], lane);
         }
         return;
     }
 
     // -------------------------------------------------------------------- consumers
+    // this thread's unit (the same in every tile) and its chunk rotation
+    const int u = warp * 32 + lane;
+    const bool has_unit = u < p.units;
+    const int py = static_cast<int>(fdiv(static_cast<unsigned>(u), p.div_tw_gs));
+    const int rem = u - py * p.TW * p.GS;
+    const int px = static_cast<int>(fdiv(static_cast<unsigned>(rem), p.div_gs));
+    const int gl = rem - px * p.GS;
     const int q8 = lane & 7;
     int rot = 0;
     if constexpr (Q == 2) rot = q8 >> 2;
@@ -389,44 +430,37 @@ fwd_tile_kernel(const __grid_constant__ CUtensorMap xmap, const T* __restrict__ 
     int choff[Q];
 #pragma unroll
     for (int j = 0; j < Q; ++j) {
-        int c = rot + j;
-        if (c >= Q) c -= Q;
-        choff[j] = c;
+        int cc = rot + j;
+        if (cc >= Q) cc -= Q;
+        choff[j] = cc;
     }
-    const int rowB = p.WW * p.PB;
+    const int rowB = p.WW * PB;
     const float wymax = static_cast<float>(p.WH - 2), wxmax = static_cast<float>(p.WW - 2);
     const int rowC = f.W * f.C;
     const float fdil = static_cast<float>(f.dilation);
+    const int within = row_runs ? (px * f.G + gl) : gl;  // unit index inside its record run
 
     for (int i = 0; i < ntiles; ++i) {
-        const unsigned t = static_cast<unsigned>(first + i * static_cast<int>(gridDim.x));
-        const int b = i & 1;
-        const unsigned char* buf = smem + b * p.buf_bytes;
-        const bool ok = mbar_wait_bounded(&full_bar[b], (i >> 1) & 1, kCopyWaitLimitNs);
+        const unsigned t = static_cast<unsigned>(first + i * stride_t);
+        const int rb = i % nrec, wb = i & 1;
+        bool ok = mbar_wait_bounded(&rec_full[rb], (i / nrec) & 1, kCopyWaitLimitNs);
+        ok = ok && mbar_wait_bounded(&win_full[wb], (i >> 1) & 1, kCopyWaitLimitNs);
         if (!__all_sync(0xffffffffu, ok)) {
             if (lane == 0) atomicOr(&g_device_status, kStatusCopyTimeout);
             return;
         }
-
         const TileCoord c = tile_coord(p, t);
-        const unsigned char* win = buf + p.rec_bytes;
-        const T* ximg = x + static_cast<size_t>(c.n) * f.H * rowC;
-
-        for (int u = warp * 32 + lane; u < p.units; u += nc * 32) {
-            const unsigned py_ = fdiv(static_cast<unsigned>(u), p.div_tw_gs);
-            const int rem = u - static_cast<int>(py_) * p.TW * p.GS;
-            const unsigned px_ = fdiv(static_cast<unsigned>(rem), p.div_gs);
-            const int gl = rem - static_cast<int>(px_) * p.GS;
-            const int py = static_cast<int>(py_), px = static_cast<int>(px_);
-            if (py >= c.nh || px >= c.nw) continue;
+        if (has_unit && py < c.nh && px < c.nw) {
+            const unsigned char* win = winbuf + wb * p.win_bytes;
+            const T* ximg = x + static_cast<size_t>(c.n) * f.H * rowC;
             const int ho = c.ho0 + py, wo = c.wo0 + px, g = c.gsub * p.GS + gl;
 
             // this unit's record in shared memory
             const int run = row_runs ? py : py * c.nw + px;
             int count;
             const unsigned long long ra = reinterpret_cast<unsigned long long>(run_src<T>(p, c, om, run, &count));
-            const int within = row_runs ? (px * f.G + g) : gl;
-            const T* rec = reinterpret_cast<const T*>(buf + run * p.run_slot + (ra & 15)) + within * R3;
+            const T* rec = reinterpret_cast<const T*>(recbuf + rb * p.rec_bytes + run * p.run_slot + (ra & 15)) +
+                           within * R3;
 
             const unsigned char* ubase = win + gl * (Q * 16);
             float2 acc[Q][CH / 2];
@@ -456,52 +490,122 @@ fwd_tile_kernel(const __grid_constant__ CUtensorMap xmap, const T* __restrict__ 
                     // all four corners inside the window; outside-image corners read
                     // the window's zeros and the finite weight adds exactly 0
                     const float ly = dy - fy0, lx = dx - fx0;
-                    const float a0 = m * (1.f - ly), a1 = m * ly;
-                    const float w00 = a0 * (1.f - lx), w01 = a0 * lx, w10 = a1 * (1.f - lx), w11 = a1 * lx;
-                    const int off = (static_cast<int>(wyf) * p.WW + static_cast<int>(wxf)) * p.PB;
+                    const float a1 = m * ly, a0 = m - a1;          // m (1 - ly), m ly
+                    const float w01 = a0 * lx, w00 = a0 - w01;    // a0 (1 - lx), a0 lx
+                    const float w11 = a1 * lx, w10 = a1 - w11;
+                    const int off = (static_cast<int>(wyf) * p.WW + static_cast<int>(wxf)) * PB;
                     const unsigned char* pb = ubase + off;
+                    if constexpr (HW && std::is_same<T, __half>::value) {
+                        const uint32_t wt = pack_half2(w00, w01), wbt = pack_half2(w10, w11);
 #pragma unroll
-                    for (int j = 0; j < Q; ++j) {
-                        const unsigned char* pc = pb + (choff[j] << 4);
-                        const uint4 v00 = *reinterpret_cast<const uint4*>(pc);
-                        const uint4 v01 = *reinterpret_cast<const uint4*>(pc + p.PB);
-                        const uint4 v10 = *reinterpret_cast<const uint4*>(pc + rowB);
-                        const uint4 v11 = *reinterpret_cast<const uint4*>(pc + rowB + p.PB);
-                        fma_chunk<T, HW>(acc[j], w00, v00);
-                        fma_chunk<T, HW>(acc[j], w01, v01);
-                        fma_chunk<T, HW>(acc[j], w10, v10);
-                        fma_chunk<T, HW>(acc[j], w11, v11);
+                        for (int j = 0; j < Q; ++j) {
+                            const unsigned char* pc = pb + (choff[j] << 4);
+                            const uint4 v00 = *reinterpret_cast<const uint4*>(pc);
+                            const uint4 v01 = *reinterpret_cast<const uint4*>(pc + PB);
+                            const uint4 v10 = *reinterpret_cast<const uint4*>(pc + rowB);
+                            const uint4 v11 = *reinterpret_cast<const uint4*>(pc + rowB + PB);
+                            fma_chunk_h<false>(acc[j], wt, v00);
+                            fma_chunk_h<true>(acc[j], wt, v01);
+                            fma_chunk_h<false>(acc[j], wbt, v10);
+                            fma_chunk_h<true>(acc[j], wbt, v11);
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < Q; ++j) {
+                            const unsigned char* pc = pb + (choff[j] << 4);
+                            const uint4 v00 = *reinterpret_cast<const uint4*>(pc);
+                            const uint4 v01 = *reinterpret_cast<const uint4*>(pc + PB);
+                            const uint4 v10 = *reinterpret_cast<const uint4*>(pc + rowB);
+                            const uint4 v11 = *reinterpret_cast<const uint4*>(pc + rowB + PB);
+                            fma_chunk<T, HW>(acc[j], w00, v00);
+                            fma_chunk<T, HW>(acc[j], w01, v01);
+                            fma_chunk<T, HW>(acc[j], w10, v10);
+                            fma_chunk<T, HW>(acc[j], w11, v11);
+                        }
                     }
                 } else {
                     slow |= 1ull << k;
                 }
             }
             // the points outside the window: global gather with per-corner validity
-            while (slow) {
-                const int k = __ffsll(static_cast<long long>(slow)) - 1;
-                slow &= slow - 1ull;
-                const int ky = k / K, kx = k - (k / K) * K;
-                const float rx = ElemTraits<T>::to_float(rec[k]);
-                const float ry = ElemTraits<T>::to_float(rec[KK + k]);
-                const float m = ElemTraits<T>::to_float(rec[2 * KK + k]);
-                const Sample s = locate(by + ky * f.dilation, bx + kx * f.dilation, ry, rx, f.offset_scale, f.H, f.W);
-                if (s.bits == 0u) continue;
-                const float a0 = m * (1.f - s.ly), a1 = m * s.ly;
-                float w[4];
-                w[0] = (s.bits & 1u) ? a0 * (1.f - s.lx) : 0.f;
-                w[1] = (s.bits & 2u) ? a0 * s.lx : 0.f;
-                w[2] = (s.bits & 4u) ? a1 * (1.f - s.lx) : 0.f;
-                w[3] = (s.bits & 8u) ? a1 * s.lx : 0.f;
-                const T* c00 = ximg + (s.y0 * f.W + s.x0) * f.C + g * f.Cg;
+            if constexpr (Q <= 2) {
+                // two points per pass, so that their loads are in flight together
+                while (slow) {
+                    int kk[2];
 #pragma unroll
-                for (int cn = 0; cn < 4; ++cn) {
-                    if (!(s.bits & (1u << cn))) continue;
-                    const T* pc = c00 + (cn >> 1) * rowC + (cn & 1) * f.C;
+                    for (int h = 0; h < 2; ++h) {
+                        kk[h] = slow ? __ffsll(static_cast<long long>(slow)) - 1 : -1;
+                        slow &= slow ? slow - 1ull : 0ull;
+                    }
+                    uint4 v[2][4][Q];
+                    float w[2][4];
 #pragma unroll
-                    for (int j = 0; j < Q; ++j) {
-                        uint32_t tt[4];
-                        load_vec<16>(pc + choff[j] * CH, tt);
-                        fma_chunk<T, HW>(acc[j], w[cn], make_uint4(tt[0], tt[1], tt[2], tt[3]));
+                    for (int h = 0; h < 2; ++h) {
+                        const int k = kk[h] < 0 ? kk[0] : kk[h];
+                        const int ky = k / K, kx = k - (k / K) * K;
+                        const float rx = ElemTraits<T>::to_float(rec[k]);
+                        const float ry = ElemTraits<T>::to_float(rec[KK + k]);
+                        const float m = ElemTraits<T>::to_float(rec[2 * KK + k]);
+                        Sample s = locate(by + ky * f.dilation, bx + kx * f.dilation, ry, rx, f.offset_scale, f.H, f.W);
+                        if (kk[h] < 0) s.bits = 0u;
+                        // the same weight arithmetic as the window path
+                        const float a1 = m * s.ly, a0 = m - a1;
+                        const float w01 = a0 * s.lx, w11 = a1 * s.lx;
+                        w[h][0] = (s.bits & 1u) ? a0 - w01 : 0.f;
+                        w[h][1] = (s.bits & 2u) ? w01 : 0.f;
+                        w[h][2] = (s.bits & 4u) ? a1 - w11 : 0.f;
+                        w[h][3] = (s.bits & 8u) ? w11 : 0.f;
+                        const T* c00 = ximg + (s.y0 * f.W + s.x0) * f.C + g * f.Cg;
+#pragma unroll
+                        for (int cn = 0; cn < 4; ++cn) {
+                            const bool in = (s.bits >> cn) & 1u;
+                            const T* pcg = c00 + (cn >> 1) * rowC + (cn & 1) * f.C;
+#pragma unroll
+                            for (int j = 0; j < Q; ++j) {
+                                uint32_t tt[4] = {0u, 0u, 0u, 0u};
+                                if (in) load_vec<16>(pcg + choff[j] * CH, tt);
+                                v[h][cn][j] = make_uint4(tt[0], tt[1], tt[2], tt[3]);
+                            }
+                        }
+                    }
+                    // corners outside the image (and a missing second point) carry
+                    // weight 0 and x = 0, so they add exactly 0 whatever the mask holds
+#pragma unroll
+                    for (int h = 0; h < 2; ++h)
+#pragma unroll
+                        for (int cn = 0; cn < 4; ++cn)
+#pragma unroll
+                            for (int j = 0; j < Q; ++j) fma_chunk<T, HW>(acc[j], w[h][cn], v[h][cn][j]);
+                }
+            } else {
+                while (slow) {
+                    const int k = __ffsll(static_cast<long long>(slow)) - 1;
+                    slow &= slow - 1ull;
+                    const int ky = k / K, kx = k - (k / K) * K;
+                    const float rx = ElemTraits<T>::to_float(rec[k]);
+                    const float ry = ElemTraits<T>::to_float(rec[KK + k]);
+                    const float m = ElemTraits<T>::to_float(rec[2 * KK + k]);
+                    const Sample s = locate(by + ky * f.dilation, bx + kx * f.dilation, ry, rx, f.offset_scale, f.H, f.W);
+                    if (s.bits == 0u) continue;
+                    // the same weight arithmetic as the window path
+                    const float a1 = m * s.ly, a0 = m - a1;
+                    const float w01 = a0 * s.lx, w11 = a1 * s.lx;
+                    float w[4];
+                    w[0] = (s.bits & 1u) ? a0 - w01 : 0.f;
+                    w[1] = (s.bits & 2u) ? w01 : 0.f;
+                    w[2] = (s.bits & 4u) ? a1 - w11 : 0.f;
+                    w[3] = (s.bits & 8u) ? w11 : 0.f;
+                    const T* c00 = ximg + (s.y0 * f.W + s.x0) * f.C + g * f.Cg;
+#pragma unroll
+                    for (int cn = 0; cn < 4; ++cn) {
+                        if (!(s.bits & (1u << cn))) continue;
+                        const T* pcg = c00 + (cn >> 1) * rowC + (cn & 1) * f.C;
+#pragma unroll
+                        for (int j = 0; j < Q; ++j) {
+                            uint32_t tt[4];
+                            load_vec<16>(pcg + choff[j] * CH, tt);
+                            fma_chunk<T, HW>(acc[j], w[cn], make_uint4(tt[0], tt[1], tt[2], tt[3]));
+                        }
                     }
                 }
             }
@@ -514,7 +618,10 @@ fwd_tile_kernel(const __grid_constant__ CUtensorMap xmap, const T* __restrict__ 
             }
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(&empty_bar[b]);  // this warp is done with buffer b
+        if (lane == 0) {  // this warp is done with both buffers of tile i
+            mbar_arrive(&rec_empty[rb]);
+            mbar_arrive(&win_empty[wb]);
+        }
     }
 }
 

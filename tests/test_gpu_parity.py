@@ -306,3 +306,15 @@ def test_fp16_weight_rounding_stays_far_inside_the_tolerance(name, monkeypatch, 
         errs[exact] = np.abs(out.double().cpu().numpy() - ref).max() / scale
     assert errs["0"] <= 1e-3, errs        # a quarter of the 4e-3 bar
     assert errs["0"] <= 2.0 * errs["1"] + 2e-4, errs
+
+
+@pytest.mark.parametrize("dtype", ["f32", "f16", "bf16"])
+def test_an_image_result_does_not_depend_on_its_batch(dtype, cuda_device):
+    """Batch invariance: the kernel choice and tiling depend on the image
+    geometry only, so every image gives the same bits alone or in a batch."""
+    x, om = make_inputs(12, 40, 44, 64, 4, 3, 40, 44, dtype, ("normal", 0, 2.5), ("normal", 0, 0.5), seed=31)
+    full = dcn.forward(x.to(cuda_device), om.to(cuda_device), G=4, K=3, pad=1).cpu()
+    for lo, hi in [(0, 1), (3, 8), (11, 12)]:
+        part = dcn.forward(x[lo:hi].contiguous().to(cuda_device), om[lo:hi].contiguous().to(cuda_device),
+                           G=4, K=3, pad=1).cpu()
+        assert torch.equal(part, full[lo:hi]), (lo, hi)
