@@ -1,4 +1,4 @@
-"""fp64 CPU oracle for the DCNv4 forward spatial aggregation.
+"""fp64 CPU oracle for the DCNv4 spatial aggregation, forward and backward.
 
 TEST INFRASTRUCTURE ONLY: the tests, the smoke check and the CPU-baseline leg
 of the benchmark may import this package; the product path (the CUDA library
@@ -55,6 +55,8 @@ def _load():
         lib.oracle_dcnv4_forward_images.restype = i
         lib.oracle_dcnv4_sampling_index.argtypes = [p, p, p] + [i] * 8 + [f]
         lib.oracle_dcnv4_sampling_index.restype = i
+        lib.oracle_dcnv4_backward.argtypes = [p] * 5 + [i] * 9 + [f]
+        lib.oracle_dcnv4_backward.restype = i
         _lib = lib
     return _lib
 
@@ -124,3 +126,27 @@ def sampling_index(offset_mask, H: int, W: int, G: int, K: int, stride: int = 1,
         if rc != 0:
             raise ValueError("oracle rejected the arguments")
     return corner, valid
+
+
+def dcnv4_backward(x, offset_mask, grad_out, G: int, K: int, stride: int = 1, pad: int = 0, dilation: int = 1,
+                   offset_scale: float = 1.0):
+    """fp64 backward: returns (grad_x [N,H,W,C], grad_offset_mask [N,Hout,Wout,G,3*K*K]).
+
+    The exact derivative of ``dcnv4_forward`` for a loss whose gradient with
+    respect to the output is ``grad_out`` (see dcnv4_oracle.c for the
+    formulas and the convention at integer positions)."""
+    x = _f64(x)
+    om = _f64(offset_mask)
+    go = _f64(grad_out)
+    N, H, W, C = x.shape
+    Hout, Wout = output_size(H, K, stride, pad, dilation), output_size(W, K, stride, pad, dilation)
+    if om.shape != (N, Hout, Wout, G, 3 * K * K) or go.shape != (N, Hout, Wout, C):
+        raise ValueError("offset_mask / grad_out shapes do not match x")
+    gx = np.zeros_like(x)
+    gom = np.zeros_like(om)
+    if N:
+        rc = _load().oracle_dcnv4_backward(_ptr(x), _ptr(om), _ptr(go), _ptr(gx), _ptr(gom), N, H, W, C, G, K,
+                                           stride, pad, dilation, float(offset_scale))
+        if rc != 0:
+            raise ValueError("oracle rejected the arguments")
+    return gx, gom

@@ -191,3 +191,76 @@ int oracle_dcnv4_sampling_index(const double *om, int32_t *corner, uint8_t *vali
                 }
     return 0;
 }
+
+/* ------------------------------------------------------------------------
+ * Backward of the forward above (the training direction; the pages use the
+ * operator for training, e.g. the Stable Diffusion fine-tuning of the
+ * jsqmd.com page, section 4). For a loss L with dL/dout = grad_out:
+ *   dL/dx[n,y,x,gc]  = sum over every (ho, wo, k, corner) that reads (y, x) of
+ *                      m_k * W_corner * grad_out[n,ho,wo,gc]
+ *   dL/dm_k          = sum_c grad_out[c] * sample_k[c],  sample_k = sum_corners W * x
+ *   dL/d r[k]        = m_k * s * sum_c grad_out[c] * sum_corners dW/dfx * x   (x-offset)
+ *   dL/d r[K*K + k]  = m_k * s * sum_c grad_out[c] * sum_corners dW/dfy * x   (y-offset)
+ * with W_ab = (a ? fy : 1-fy) (b ? fx : 1-fx), dW/dfy = (a ? 1 : -1)(b ? fx : 1-fx),
+ * dW/dfx = (a ? fy : 1-fy)(b ? 1 : -1), s = offset_scale (d = s*r, and
+ * fy = d - floor(d) moves one for one with d between integers). Corners
+ * outside the image take no part; a sample with a non-finite offset is
+ * outside and gets zero gradients. At an integer position the corner set of
+ * floor(d) is used, i.e. the derivative from above.
+ * grad_x: [N,H,W,C] (overwritten), grad_om: [N,Hout,Wout,G,3*K*K] (overwritten).
+ * ------------------------------------------------------------------------ */
+int oracle_dcnv4_backward(const double *x, const double *om, const double *grad_out,
+                          double *grad_x, double *grad_om,
+                          int N, int H, int W, int C, int G, int K,
+                          int stride, int pad, int dilation, float offset_scale)
+{
+    if (N < 0 || H <= 0 || W <= 0 || C <= 0 || G <= 0 || K <= 0 || C % G) return -1;
+    const int Hout = oracle_output_size(H, K, stride, pad, dilation);
+    const int Wout = oracle_output_size(W, K, stride, pad, dilation);
+    if (Hout <= 0 || Wout <= 0) return -1;
+    const int Cg = C / G, KK = K * K;
+    for (size_t i = 0; i < (size_t)N * H * W * C; ++i) grad_x[i] = 0.0;
+    for (int n = 0; n < N; ++n)
+        for (int ho = 0; ho < Hout; ++ho)
+            for (int wo = 0; wo < Wout; ++wo)
+                for (int g = 0; g < G; ++g) {
+                    const size_t unit = (((size_t)n * Hout + ho) * Wout + wo) * G + g;
+                    const double *r = om + unit * (size_t)(3 * KK);
+                    double *gr = grad_om + unit * (size_t)(3 * KK);
+                    const double *go = grad_out + (((size_t)n * Hout + ho) * Wout + wo) * (size_t)C + (size_t)g * Cg;
+                    for (int k = 0; k < KK; ++k) {
+                        const int ky = k / K, kx = k % K;
+                        const int p0y = ho * stride - pad + ky * dilation;
+                        const int p0x = wo * stride - pad + kx * dilation;
+                        const double dx = scaled_offset(offset_scale, r[k]);
+                        const double dy = scaled_offset(offset_scale, r[KK + k]);
+                        const double m = r[2 * KK + k];
+                        double g_m = 0.0, g_fx = 0.0, g_fy = 0.0;
+                        if (isfinite(dx) && isfinite(dy)) {
+                            const double fy0 = floor(dy), fx0 = floor(dx);
+                            const double ly = dy - fy0, lx = dx - fx0;
+                            const double y0 = (double)p0y + fy0, x0 = (double)p0x + fx0;
+                            for (int a = 0; a <= 1; ++a)
+                                for (int b = 0; b <= 1; ++b) {
+                                    const double yy = y0 + a, xx = x0 + b;
+                                    if (!(yy >= 0.0 && yy <= (double)(H - 1) && xx >= 0.0 && xx <= (double)(W - 1)))
+                                        continue;
+                                    const double wy = a ? ly : 1.0 - ly, wx = b ? lx : 1.0 - lx;
+                                    const double dwy = a ? 1.0 : -1.0, dwx = b ? 1.0 : -1.0;
+                                    const size_t pix = (((size_t)n * H + (size_t)yy) * W + (size_t)xx) * C + (size_t)g * Cg;
+                                    for (int c = 0; c < Cg; ++c) {
+                                        const double xv = x[pix + c];
+                                        g_m += go[c] * wy * wx * xv;
+                                        g_fy += go[c] * dwy * wx * xv;
+                                        g_fx += go[c] * wy * dwx * xv;
+                                        grad_x[pix + c] += m * wy * wx * go[c];
+                                    }
+                                }
+                        }
+                        gr[k] = m * (double)offset_scale * g_fx;
+                        gr[KK + k] = m * (double)offset_scale * g_fy;
+                        gr[2 * KK + k] = g_m;
+                    }
+                }
+    return 0;
+}
