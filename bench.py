@@ -36,6 +36,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "DCNv4 fwd sampling points/s (G/s); achieved HBM GB/s as % of B200 peak"
+METRIC_BWD = "DCNv4 bwd sampling points/s (G/s); achieved HBM GB/s as % of B200 peak"
 UNIT = "Gpoints/s"
 FALLBACK_HBM_GBS = 6650.0
 
@@ -50,6 +51,8 @@ def parse_args():
     ap.add_argument("--soak-s", type=float, default=1.0)
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--pass", dest="which", choices=["forward", "backward"], default="forward",
+                    help="forward (the headline) or the backward of the same workload")
     return ap.parse_args()
 
 
@@ -153,6 +156,19 @@ def cpu_baseline(w, x, om):
                                     "fp64 C oracle, one thread"}
 
 
+def cpu_baseline_backward(w, x, om, go):
+    """The fp64 oracle's backward, as it stands, on the whole batch (single thread)."""
+    import oracle
+    xd, omd, god = x.double().numpy(), om.double().numpy(), go.double().numpy()
+    oracle.dcnv4_backward(xd[:1], omd[:1], god[:1], **w.kwargs())  # load + warm
+    t0 = time.perf_counter()
+    oracle.dcnv4_backward(xd, omd, god, **w.kwargs())
+    dt = time.perf_counter() - t0
+    return {"value": w.points / dt / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "seconds": dt, "sample": f"the whole {w.name} batch ({w.N} images, {w.points} points), "
+                                    "fp64 C oracle backward, one thread"}
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -164,25 +180,173 @@ def run_reference(args):
     xd, omd = x.double().numpy(), om.double().numpy()
     n_s = max(1, min(w.N, 8))  # images per step: a bounded sample (~0.1 s of CPU work each)
     pts = w.points // w.N * n_s
+    if args.which == "backward":
+        from deformable_convolution_sparse_b200.workloads import workload_grad_out
+        god = workload_grad_out(w).double().numpy()
+
+        def one(b):
+            oracle.dcnv4_backward(xd[b:b + n_s], omd[b:b + n_s], god[b:b + n_s], **w.kwargs())
+    else:
+        def one(b):
+            oracle.dcnv4_forward(xd, omd, **w.kwargs(), n_begin=b, n_end=b + n_s)
     for _ in range(args.warmup):
-        oracle.dcnv4_forward(xd, omd, **w.kwargs(), n_begin=0, n_end=n_s)
+        one(0)
     t0 = time.perf_counter()
     for i in range(args.steps):
-        b = (i * n_s) % (w.N - n_s + 1)
-        oracle.dcnv4_forward(xd, omd, **w.kwargs(), n_begin=b, n_end=b + n_s)
+        one((i * n_s) % (w.N - n_s + 1))
     dt = time.perf_counter() - t0
     value = pts * args.steps / dt / 1e9
     line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "impl": "reference", "metric": METRIC_BWD if args.which == "backward" else METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": f"{w.name}: N={w.N} H=W={w.H} C={w.C} G={w.G} K={w.K} pad={w.pad} "
                                f"dilation={w.dilation}, {w.dtype} storage", "sample_images_per_step": n_s},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
-                         "sample": f"{n_s} of {w.N} images per step, fp64 C oracle, one thread"},
+                         "sample": f"{n_s} of {w.N} images per step, fp64 C oracle "
+                                   f"{args.which}, one thread"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+
+
+def time_steps(step, launches, args, dev, stream, barrier, max_over_ranks):
+    """W warm-up steps, a soak of --soak-s seconds with the clock sampler running, then exactly
+    K steps between CUDA events on `stream`, bracketed by barrier + synchronise. Returns
+    (max over ranks of the timed milliseconds, the stopped sampler, launches in the timed region)."""
+    import torch
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+    uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    sampler = ClockSampler(uuid)
+    sampler.start()
+    t_end = time.perf_counter() + args.soak_s
+    i = 0
+    while time.perf_counter() < t_end:
+        for _ in range(50):
+            step(i)
+            i += 1
+        torch.cuda.synchronize(dev)
+    barrier()
+    torch.cuda.synchronize(dev)
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    launches[0] = 0
+    ev0.record(stream)
+    for i in range(args.steps):
+        step(i)
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    sampler.stop()
+    return max_over_ranks(ev0.elapsed_time(ev1)), sampler, launches[0]
+
+
+def run_backward(args, w, dev, world, rank, barrier, max_over_ranks):
+    """The backward of the same workload: one dcnv4_backward call (a clear of grad_x plus one
+    kernel) per step, fp32 gradients, inputs rotating over resident sets larger than L2."""
+    import torch
+    import deformable_convolution_sparse_b200 as dcn
+    from deformable_convolution_sparse_b200.workloads import workload_grad_out, workload_inputs
+
+    wr = w.with_(seed=w.seed + 1000 * rank)
+    x, om = workload_inputs(wr)
+    go = workload_grad_out(wr)
+    lib = dcn.load_library()
+    dtype_code = dcn.binding.TORCH_DTYPE[x.dtype]
+    e = x.element_size()
+    nx, nom, nout = x.numel(), om.numel(), go.numel()
+    # algorithmic bytes: x, offset_mask and grad_out read once; grad_x and grad_offset_mask (fp32) written once
+    foot = (nx + nom + nout) * e + (nx + nom) * 4
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    copies = max(3, math.ceil(3 * l2 / foot))
+    sets = [(x.to(dev), om.to(dev), go.to(dev), torch.empty(x.shape, dtype=torch.float32, device=dev),
+             torch.empty(om.shape, dtype=torch.float32, device=dev)) for _ in range(copies)]
+    stream = torch.cuda.current_stream(dev)
+    sh = stream.cuda_stream
+    launches = [0]
+
+    def call(xd, omd, god, gxd, gomd):
+        rc = lib.dcnv4_backward(xd.data_ptr(), omd.data_ptr(), god.data_ptr(), gxd.data_ptr(), gomd.data_ptr(),
+                                w.N, w.H, w.W, w.C, w.G, w.K, w.stride, w.pad, w.dilation, w.offset_scale,
+                                dtype_code, sh)
+        if rc != 0:
+            raise dcn.DCNv4Error(rc, "dcnv4_backward")
+
+    def step(i):
+        call(*sets[i % copies])
+        launches[0] += 1  # one kernel (the clear of grad_x is a cudaMemsetAsync)
+
+    ms, sampler, timed_launches = time_steps(step, launches, args, dev, stream, barrier, max_over_ranks)
+    ms_step = ms / args.steps
+    value = w.points * world * args.steps / (ms / 1e3) / 1e9
+    peak, peak_kind = measured_peaks()
+    achieved = foot / (ms_step / 1e3) / 1e9
+
+    # end to end: pinned host inputs copied in, backward, both gradients copied back, one stream
+    xh, omh, goh = x.pin_memory(), om.pin_memory(), go.pin_memory()
+    gxh = torch.empty(x.shape, dtype=torch.float32).pin_memory()
+    gomh = torch.empty(om.shape, dtype=torch.float32).pin_memory()
+    xd, omd, god, gxd, gomd = sets[0]
+
+    def e2e_step():
+        xd.copy_(xh, non_blocking=True)
+        omd.copy_(omh, non_blocking=True)
+        god.copy_(goh, non_blocking=True)
+        call(xd, omd, god, gxd, gomd)
+        gxh.copy_(gxd, non_blocking=True)
+        gomh.copy_(gomd, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1))
+    e2e_value = w.points * world * args.e2e_steps / (e2e_ms / 1e3) / 1e9
+    if not torch.equal(gomh, gomd.cpu()):
+        raise SystemExit("end-to-end gradient record differs from the device-resident one")
+
+    base = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        base = cpu_baseline_backward(w, x, om, go)
+    if rank == 0:
+        line = {
+            "metric": METRIC_BWD, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic", "pass": "backward",
+            "config": {
+                "workload": f"{w.name} backward: N={w.N} per GPU, H=W={w.H}, C={w.C}, G={w.G} (C/G={w.Cg}), "
+                            f"K={w.K}, stride={w.stride}, pad={w.pad}, dilation={w.dilation}; fp32 gradients",
+                "storage_dtype": w.dtype, "accumulate": "f32", "global_batch": w.N * world,
+                "points_per_step_per_gpu": w.points, "parallelism": f"dp{world} (independent batches)",
+                "l2": f"steps rotate over {copies} resident sets, {copies * foot / 1e6:.0f} MB in total vs "
+                      f"{l2 / 1e6:.0f} MB L2",
+                "inputs": "seeded synthetic: x~N(0,1), offsets and masks as the forward, grad_out~N(0,1)",
+            },
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak,
+                         "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json)"
+                         if peak_kind == "measured" else "fallback 6.65 TB/s",
+                         "kernel": "dcnv4 backward (clear of grad_x + one kernel per step)",
+                         "algorithmic_bytes_per_launch": foot, "traffic": None},
+            "e2e": {"value": e2e_value, "unit": UNIT, "ms_per_step": e2e_ms / args.e2e_steps,
+                    "steps": args.e2e_steps, "h2d_bytes_per_step": (nx + nom + nout) * e,
+                    "d2h_bytes_per_step": (nx + nom) * 4,
+                    "path": "pinned host tensors copied in, dcnv4_backward, gradients copied out, one stream"},
+            "gpu_launches": timed_launches,
+            "clocks": sampler.summary(),
+            "cpu_baseline": base,
+        }
+        print(json.dumps(line), flush=True)
 
 
 def main():
@@ -219,6 +383,11 @@ def main():
         return float(t.item())
 
     w = WORKLOADS[args.workload or BENCH_WORKLOAD]
+    if args.which == "backward":
+        run_backward(args, w, dev, world, rank, barrier, max_over_ranks)
+        if world > 1:
+            dist.destroy_process_group()
+        return
     # weak scaling: rank r owns images [64 r, 64 (r+1)) of the global batch, drawn from seed + r
     wr = w.with_(seed=w.seed + 1000 * rank)
     x, om = workload_inputs(wr)
@@ -243,35 +412,7 @@ def main():
             raise dcn.DCNv4Error(rc, "dcnv4_forward")
         launches[0] += 1
 
-    for i in range(args.warmup):
-        step(i)
-    torch.cuda.synchronize(dev)
-
-    uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
-    sampler = ClockSampler(uuid)
-    sampler.start()
-    t_end = time.perf_counter() + args.soak_s
-    i = 0
-    while time.perf_counter() < t_end:
-        for _ in range(200):
-            step(i)
-            i += 1
-        torch.cuda.synchronize(dev)
-
-    barrier()
-    torch.cuda.synchronize(dev)
-    ev0 = torch.cuda.Event(enable_timing=True)
-    ev1 = torch.cuda.Event(enable_timing=True)
-    launches[0] = 0
-    ev0.record(stream)
-    for i in range(args.steps):
-        step(i)
-    ev1.record(stream)
-    torch.cuda.synchronize(dev)
-    barrier()
-    sampler.stop()
-    timed_launches = launches[0]
-    ms = max_over_ranks(ev0.elapsed_time(ev1))
+    ms, sampler, timed_launches = time_steps(step, launches, args, dev, stream, barrier, max_over_ranks)
     ms_step = ms / args.steps
     total_points = w.points * world * args.steps
     value = total_points / (ms / 1e3) / 1e9

@@ -27,7 +27,7 @@ STATUS = {v: k for k, v in STATUS_NAMES.items()}
 TORCH_DTYPE = {torch.float32: DCNV4_F32, torch.float16: DCNV4_F16, torch.bfloat16: DCNV4_BF16}
 
 # every symbol include/dcnv4.h declares
-EXPORTS = ("dcnv4_output_shape", "dcnv4_validate", "dcnv4_forward", "dcnv4_sampling_index",
+EXPORTS = ("dcnv4_output_shape", "dcnv4_validate", "dcnv4_forward", "dcnv4_backward", "dcnv4_sampling_index",
            "dcnv4_forward_host", "dcnv4_forward_host_noalloc", "dcnv4_device_status", "dcnv4_selftest_wait_timeout", "dcnv4_strerror",
            "dcnv4_abi_version")
 DEVSTATUS_COPY_TIMEOUT, DEVSTATUS_SELFTEST_TIMEOUT = 1, 2
@@ -59,6 +59,8 @@ def load_library():
     lib.dcnv4_validate.restype = i
     lib.dcnv4_forward.argtypes = [p, p, p] + [i] * 9 + [f, i, p]
     lib.dcnv4_forward.restype = i
+    lib.dcnv4_backward.argtypes = [p] * 5 + [i] * 9 + [f, i, p]
+    lib.dcnv4_backward.restype = i
     lib.dcnv4_sampling_index.argtypes = [p, p, p] + [i] * 8 + [f, i, p]
     lib.dcnv4_sampling_index.restype = i
     lib.dcnv4_forward_host.argtypes = [p] * 6 + [i] * 9 + [f, i, p]
@@ -168,6 +170,48 @@ def forward(x: torch.Tensor, offset_mask: torch.Tensor, G: int, K: int, stride: 
     if rc != DCNV4_OK:
         raise DCNv4Error(rc, "dcnv4_forward")
     return out
+
+
+def backward(x: torch.Tensor, offset_mask: torch.Tensor, grad_out: torch.Tensor, G: int, K: int, stride: int = 1,
+             pad: int = 0, dilation: int = 1, offset_scale: float = 1.0, grad_x: torch.Tensor | None = None,
+             grad_offset_mask: torch.Tensor | None = None, stream=None):
+    """DCNv4 backward on the GPU through ``dcnv4_backward``.
+
+    x: [N,H,W,C]; offset_mask: [N,Hout,Wout,G,3*K*K]; grad_out: [N,Hout,Wout,C],
+    all of one dtype. Returns (grad_x [N,H,W,C], grad_offset_mask
+    [N,Hout,Wout,G,3*K*K]), both fp32; the record layout of grad_offset_mask
+    is that of offset_mask. Asynchronous on ``stream`` (default: current).
+    """
+    for t, name in ((x, "x"), (offset_mask, "offset_mask"), (grad_out, "grad_out")):
+        _check_tensor(t, name)
+    if x.dim() != 4:
+        raise ValueError("x must be [N,H,W,C]")
+    if offset_mask.dtype != x.dtype or grad_out.dtype != x.dtype or offset_mask.device != x.device or \
+            grad_out.device != x.device:
+        raise ValueError("offset_mask and grad_out must match x in dtype and device")
+    N, H, W, C = x.shape
+    Hout, Wout = output_shape(H, W, K, stride, pad, dilation)
+    if tuple(offset_mask.shape) != (N, Hout, Wout, G, 3 * K * K):
+        raise ValueError(f"offset_mask shape {tuple(offset_mask.shape)} != {(N, Hout, Wout, G, 3 * K * K)}")
+    if tuple(grad_out.shape) != (N, Hout, Wout, C):
+        raise ValueError(f"grad_out shape {tuple(grad_out.shape)} != {(N, Hout, Wout, C)}")
+    outs = []
+    for t, shape, name in ((grad_x, x.shape, "grad_x"), (grad_offset_mask, offset_mask.shape, "grad_offset_mask")):
+        if t is None:
+            t = torch.empty(tuple(shape), dtype=torch.float32, device=x.device)
+        else:
+            _check_tensor(t, name)
+            if tuple(t.shape) != tuple(shape) or t.dtype != torch.float32 or t.device != x.device:
+                raise ValueError(f"{name} must be fp32 of shape {tuple(shape)} on {x.device}")
+        outs.append(t)
+    gx, gom = outs
+    with torch.cuda.device(x.device):
+        rc = load_library().dcnv4_backward(x.data_ptr(), offset_mask.data_ptr(), grad_out.data_ptr(), gx.data_ptr(),
+                                           gom.data_ptr(), N, H, W, C, G, K, stride, pad, dilation,
+                                           float(offset_scale), TORCH_DTYPE[x.dtype], _stream_handle(stream))
+    if rc != DCNV4_OK:
+        raise DCNv4Error(rc, "dcnv4_backward")
+    return gx, gom
 
 
 def forward_host(x: torch.Tensor, offset_mask: torch.Tensor, G: int, K: int, stride: int = 1, pad: int = 0,

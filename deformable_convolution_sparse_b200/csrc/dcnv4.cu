@@ -17,6 +17,7 @@
 #include "dcnv4.h"
 #include "dcnv4_kernels.cuh"
 #include "dcnv4_window.cuh"
+#include "dcnv4_backward.cuh"
 
 namespace {
 
@@ -46,6 +47,25 @@ int check_geometry(int N, int H, int W, int K, int stride, int pad, int dilation
     if (N < 0) return DCNV4_ERR_SHAPE;
     const int rc = dcnv4_output_shape(H, W, K, stride, pad, dilation, Hout, Wout);
     return rc;
+}
+
+// Checks shared by every entry point that takes the full operator signature:
+// geometry, groups, dtype, offset_scale and the 32-bit element counts of x,
+// out and offset_mask (returned through nx, nout, nom).
+int check_sizes(int N, int H, int W, int C, int G, int K, int stride, int pad, int dilation, float offset_scale,
+                int dtype, long long* nx, long long* nout, long long* nom) {
+    int Hout = 0, Wout = 0;
+    int rc = check_geometry(N, H, W, K, stride, pad, dilation, &Hout, &Wout);
+    if (rc) return rc;
+    if (C <= 0 || G <= 0) return DCNV4_ERR_SHAPE;
+    if (C % G) return DCNV4_ERR_GROUPS;
+    if (!elem_size(dtype)) return DCNV4_ERR_DTYPE;
+    if (!std::isfinite(offset_scale)) return DCNV4_ERR_SCALE;
+    *nx = static_cast<long long>(N) * H * W * C;
+    *nout = static_cast<long long>(N) * Hout * Wout * C;
+    *nom = static_cast<long long>(N) * Hout * Wout * G * 3 * K * K;
+    if (*nx >= kLimit || *nout >= kLimit || *nom >= kLimit) return DCNV4_ERR_TOO_LARGE;
+    return DCNV4_OK;
 }
 
 int launch_status() {
@@ -356,6 +376,52 @@ int launch_forward(const void* x, const void* om, void* out, FwdParams p, cudaSt
     return launch_status();
 }
 
+// Backward: grad_x is cleared on the stream, then one kernel computes every
+// gradient. Vector path (16-byte channel chunks, float4 reductions) when the
+// pointers and channel rows allow it, element path otherwise.
+template <typename T>
+int launch_backward(const void* x, const void* om, const void* go, float* gx, float* gom, FwdParams p,
+                    cudaStream_t stream) {
+    constexpr int E = sizeof(T);
+    const bool vec = aligned(x, 16) && aligned(go, 16) && aligned(gx, 16) && (p.C * E) % 16 == 0 &&
+                     (p.Cg * E) % 16 == 0;
+    const int cpl = vec ? 16 / E : 1;
+    p.chunks = p.Cg / cpl;
+    int lanes = 1;
+    while (lanes < p.chunks && lanes < 32) lanes <<= 1;
+    p.lanes = lanes;
+    // units per block: full warps, records and fp32 gradient records in shared memory
+    const size_t R = static_cast<size_t>(3) * p.KK;
+    const int step = lanes < 32 ? 32 / lanes : 1;
+    auto smem_for = [&](int upb) {
+        return ((upb * R * E + 16 + 15) & ~static_cast<size_t>(15)) + upb * R * sizeof(float);
+    };
+    int upb = kThreads / lanes;
+    while (upb > step && smem_for(upb) > 48 * 1024) upb -= step;
+    p.units_per_block = upb;
+    const size_t smem = smem_for(upb);
+    const long long blocks = (static_cast<long long>(p.units) + upb - 1) / upb;
+    if (blocks > 0x7fffffffLL) return DCNV4_ERR_TOO_LARGE;
+
+    const size_t gx_bytes = static_cast<size_t>(p.N) * p.H * p.W * p.C * sizeof(float);
+    if (cudaMemsetAsync(gx, 0, gx_bytes, stream) != cudaSuccess) return DCNV4_ERR_CUDA;
+    const T* xt = static_cast<const T*>(x);
+    const T* omt = static_cast<const T*>(om);
+    const T* got = static_cast<const T*>(go);
+    const int threads = upb * lanes;
+    auto run = [&](auto kernel) -> int {
+        if (smem > 48 * 1024 &&
+            cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+                cudaSuccess)
+            return DCNV4_ERR_LAUNCH;
+        kernel<<<static_cast<unsigned>(blocks), threads, smem, stream>>>(xt, omt, got, gx, gom, p);
+        return launch_status();
+    };
+    const bool k3 = p.K == 3;
+    if (vec) return k3 ? run(dcnv4::bwd_kernel<T, 16 / E, 3>) : run(dcnv4::bwd_kernel<T, 16 / E, 0>);
+    return k3 ? run(dcnv4::bwd_kernel<T, 1, 3>) : run(dcnv4::bwd_kernel<T, 1, 0>);
+}
+
 // Two non-blocking streams per device for the host-memory entry point,
 // created on first use and kept for the life of the process.
 constexpr int kMaxDevices = 64;
@@ -435,18 +501,10 @@ int dcnv4_output_shape(int H, int W, int K, int stride, int pad, int dilation, i
 int dcnv4_validate(const void* x, const void* offset_mask, const void* out,
                    int N, int H, int W, int C, int G, int K,
                    int stride, int pad, int dilation, float offset_scale, int dtype) {
-    int Hout = 0, Wout = 0;
-    int rc = check_geometry(N, H, W, K, stride, pad, dilation, &Hout, &Wout);
+    long long nx = 0, nout = 0, nom = 0;
+    int rc = check_sizes(N, H, W, C, G, K, stride, pad, dilation, offset_scale, dtype, &nx, &nout, &nom);
     if (rc) return rc;
-    if (C <= 0 || G <= 0) return DCNV4_ERR_SHAPE;
-    if (C % G) return DCNV4_ERR_GROUPS;
     const int e = elem_size(dtype);
-    if (!e) return DCNV4_ERR_DTYPE;
-    if (!std::isfinite(offset_scale)) return DCNV4_ERR_SCALE;
-    const long long nx = static_cast<long long>(N) * H * W * C;
-    const long long nout = static_cast<long long>(N) * Hout * Wout * C;
-    const long long nom = static_cast<long long>(N) * Hout * Wout * G * 3 * K * K;
-    if (nx >= kLimit || nout >= kLimit || nom >= kLimit) return DCNV4_ERR_TOO_LARGE;
     if (N == 0) return DCNV4_OK;
     if (!x || !offset_mask || !out) return DCNV4_ERR_NULL;
     if (!aligned(x, e) || !aligned(offset_mask, e) || !aligned(out, e)) return DCNV4_ERR_ALIGN;
@@ -469,6 +527,37 @@ int dcnv4_forward(const void* x, const void* offset_mask, void* out,
         case DCNV4_F32: return launch_forward<float>(x, offset_mask, out, p, s);
         case DCNV4_F16: return launch_forward<__half>(x, offset_mask, out, p, s);
         default: return launch_forward<__nv_bfloat16>(x, offset_mask, out, p, s);
+    }
+}
+
+int dcnv4_backward(const void* x, const void* offset_mask, const void* grad_out,
+                   float* grad_x, float* grad_offset_mask,
+                   int N, int H, int W, int C, int G, int K,
+                   int stride, int pad, int dilation, float offset_scale, int dtype,
+                   void* stream) {
+    long long nx = 0, nout = 0, nom = 0;
+    int rc = check_sizes(N, H, W, C, G, K, stride, pad, dilation, offset_scale, dtype, &nx, &nout, &nom);
+    if (rc) return rc;
+    if (N == 0) return DCNV4_OK;
+    if (!x || !offset_mask || !grad_out || !grad_x || !grad_offset_mask) return DCNV4_ERR_NULL;
+    const int e = elem_size(dtype);
+    if (!aligned(x, e) || !aligned(offset_mask, e) || !aligned(grad_out, e) || !aligned(grad_x, 4) ||
+        !aligned(grad_offset_mask, 4))
+        return DCNV4_ERR_ALIGN;
+    const void* inputs[3] = {x, offset_mask, grad_out};
+    const long long in_bytes[3] = {nx * e, nom * e, nout * e};
+    for (int i = 0; i < 3; ++i)
+        if (overlap(grad_x, nx * 4, inputs[i], in_bytes[i]) || overlap(grad_offset_mask, nom * 4, inputs[i], in_bytes[i]))
+            return DCNV4_ERR_ALIAS;
+    if (overlap(grad_x, nx * 4, grad_offset_mask, nom * 4)) return DCNV4_ERR_ALIAS;
+    int Hout = 0, Wout = 0;
+    dcnv4_output_shape(H, W, K, stride, pad, dilation, &Hout, &Wout);
+    const FwdParams p = make_params(N, H, W, C, G, K, stride, pad, dilation, offset_scale, Hout, Wout);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    switch (dtype) {
+        case DCNV4_F32: return launch_backward<float>(x, offset_mask, grad_out, grad_x, grad_offset_mask, p, s);
+        case DCNV4_F16: return launch_backward<__half>(x, offset_mask, grad_out, grad_x, grad_offset_mask, p, s);
+        default: return launch_backward<__nv_bfloat16>(x, offset_mask, grad_out, grad_x, grad_offset_mask, p, s);
     }
 }
 

@@ -1,0 +1,169 @@
+// sm_100a kernel of the DCNv4 backward: gradients of a loss with respect to
+// the input x, the offsets and the masks, given the gradient of the output.
+//
+// The forward ("不只是卷积的平替：我把DCNv4塞进Stable Diffusion的U-Net里",
+// jsqmd.com, section 1) is out[c] = sum_k m_k * S_k[c] with S_k the zero-padded
+// bilinear sample of x at grid point k moved by fl32(s * r). Its use for
+// training (section 4 of the same page) needs, for dL/dout = go:
+//   dL/dx at each in-bounds corner of each point  += m_k * W_corner * go[c]
+//   dL/dm_k                                        = sum_c go[c] * S_k[c]
+//   dL/dr (x part) = m_k * s * sum_c go[c] * dS_k[c]/dfx, likewise for y,
+// with fx, fy the fractional parts of the sample position (S is linear in each
+// of them inside a pixel cell; at an integer position the cell of floor(d) is
+// used, as in the forward).
+//
+// Design (B200): like the forward, a gather that runs on the CUDA cores. A
+// unit is one (pixel, group); `p.lanes` (a power of two <= 32) threads share
+// it, each owning 16 bytes of its channels per pass. Per point the four corner
+// vectors are loaded once and give, per channel, the top and bottom row
+// interpolants t and b: S = t + fy (b - t), dS/dfy = b - t and
+// dS/dfx = (x01 - x00) + fy ((x11 - x10) - (x01 - x00)); the three channel
+// sums are folded across the unit's lanes with xor shuffles. The x gradient is
+// a scatter: each in-bounds corner gets m W go as fp32 vector reductions
+// (`atomicAdd` on float4, resolved in L2), so its summation order, and only
+// its, is not deterministic. The offset/mask gradient of the block's units is
+// collected in shared memory and written out as one contiguous run.
+#pragma once
+
+#include "dcnv4_kernels.cuh"
+
+namespace dcnv4 {
+
+// CPL channels of storage type T at p (16 bytes when CPL > 1) -> floats
+template <typename T, int CPL>
+__device__ __forceinline__ void load_channels(const T* p, float (&v)[CPL]) {
+    if constexpr (CPL == 1) {
+        v[0] = ElemTraits<T>::to_float(__ldg(p));
+    } else {
+        static_assert(CPL * sizeof(T) == 16, "vector chunks are 16 bytes");
+        uint32_t w[4];
+        load_vec<16>(p, w);
+        if constexpr (sizeof(T) == 4) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) v[q] = __uint_as_float(w[q]);
+        } else {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float2 f = unpack2(w[q], static_cast<T*>(nullptr));
+                v[2 * q] = f.x;
+                v[2 * q + 1] = f.y;
+            }
+        }
+    }
+}
+
+// dst[0:CPL] += a * v[0:CPL] in fp32 global reductions (16-byte ones when CPL % 4 == 0)
+template <int CPL>
+__device__ __forceinline__ void scatter_add(float* dst, float a, const float (&v)[CPL]) {
+    if constexpr (CPL % 4 == 0) {
+#pragma unroll
+        for (int q = 0; q < CPL; q += 4)
+            atomicAdd(reinterpret_cast<float4*>(dst + q), make_float4(a * v[q], a * v[q + 1], a * v[q + 2], a * v[q + 3]));
+    } else {
+#pragma unroll
+        for (int q = 0; q < CPL; ++q) atomicAdd(dst + q, a * v[q]);
+    }
+}
+
+// grad_x must be zero on entry (the host clears it on the same stream);
+// grad_om is overwritten. Shared memory: the block's records (T, staged at
+// their 16-byte phase plus 16 bytes) followed, 16-byte aligned, by the block's
+// fp32 gradient records.
+template <typename T, int CPL, int KS>
+__global__ void __launch_bounds__(256)
+bwd_kernel(const T* __restrict__ x, const T* __restrict__ om, const T* __restrict__ go,
+           float* __restrict__ grad_x, float* __restrict__ grad_om, FwdParams p) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    const int K = KS > 0 ? KS : p.K;
+    const int KK = K * K;
+    const int R = 3 * KK;
+
+    const int unit0 = blockIdx.x * p.units_per_block;
+    const int nunits = min(p.units_per_block, p.units - unit0);
+    const size_t rec_area = (static_cast<size_t>(p.units_per_block) * R * sizeof(T) + 16 + 15) & ~static_cast<size_t>(15);
+    float* gbuf = reinterpret_cast<float*>(smem_raw + rec_area);
+    const T* rec_base = stage_run<T>(om + static_cast<size_t>(unit0) * R, nunits * R, smem_raw);
+    __syncthreads();
+
+    const int lu = threadIdx.x / p.lanes;
+    const int part = threadIdx.x - lu * p.lanes;
+    const bool active = lu < nunits;
+    int n = 0, ho = 0, wo = 0, g = 0;
+    if (active) unit_coords(unit0 + lu, p, n, ho, wo, g);
+    const T* rec = rec_base + (active ? lu : 0) * R;
+
+    const int rowC = p.W * p.C;
+    const T* ximg = x + static_cast<size_t>(n) * p.H * rowC;
+    float* gimg = grad_x + static_cast<size_t>(n) * p.H * rowC;
+    const T* gop = go + (static_cast<size_t>((n * p.Hout + ho) * p.Wout + wo)) * p.C + g * p.Cg;
+
+#pragma unroll (KS > 0 ? KS * KS : 1)
+    for (int k = 0; k < KK; ++k) {
+        const int ky = k / K, kx = k - (k / K) * K;
+        const int p0y = ho * p.stride - p.pad + ky * p.dilation;
+        const int p0x = wo * p.stride - p.pad + kx * p.dilation;
+        const float rx = ElemTraits<T>::to_float(rec[k]);
+        const float ry = ElemTraits<T>::to_float(rec[KK + k]);
+        const float m = ElemTraits<T>::to_float(rec[2 * KK + k]);
+        Sample s = locate(p0y, p0x, ry, rx, p.offset_scale, p.H, p.W);
+        if (!active) s.bits = 0u;
+
+        float gm = 0.f, gfx = 0.f, gfy = 0.f;
+        if (s.bits) {
+            const float ly = s.ly, lx = s.lx;
+            // mask times the corner weights, for the scatter into grad_x
+            const float a1 = m * ly, a0 = m - a1;
+            const float w01 = a0 * lx, w00 = a0 - w01, w11 = a1 * lx, w10 = a1 - w11;
+            const float wc[4] = {w00, w01, w10, w11};
+            const size_t c00 = static_cast<size_t>(s.y0 * p.W + s.x0) * p.C;
+            const size_t coff[4] = {c00, c00 + p.C, c00 + rowC, c00 + rowC + p.C};
+            for (int ch = part; ch < p.chunks; ch += p.lanes) {
+                const int c0 = g * p.Cg + ch * CPL;
+                float gv[CPL], xv[4][CPL];
+                load_channels<T, CPL>(gop + ch * CPL, gv);
+#pragma unroll
+                for (int cn = 0; cn < 4; ++cn) {
+                    if (s.bits & (1u << cn)) {
+                        load_channels<T, CPL>(ximg + coff[cn] + c0, xv[cn]);
+                    } else {
+#pragma unroll
+                        for (int q = 0; q < CPL; ++q) xv[cn][q] = 0.f;
+                    }
+                }
+#pragma unroll
+                for (int q = 0; q < CPL; ++q) {
+                    const float d0 = xv[1][q] - xv[0][q];   // along x, top row
+                    const float d1 = xv[3][q] - xv[2][q];   // along x, bottom row
+                    const float t = fmaf(lx, d0, xv[0][q]);
+                    const float b = fmaf(lx, d1, xv[2][q]);
+                    const float dfy = b - t;
+                    const float S = fmaf(ly, dfy, t);
+                    const float dfx = fmaf(ly, d1 - d0, d0);
+                    gm = fmaf(gv[q], S, gm);
+                    gfy = fmaf(gv[q], dfy, gfy);
+                    gfx = fmaf(gv[q], dfx, gfx);
+                }
+#pragma unroll
+                for (int cn = 0; cn < 4; ++cn)
+                    if (s.bits & (1u << cn)) scatter_add<CPL>(gimg + coff[cn] + c0, wc[cn], gv);
+            }
+        }
+        // every lane of the warp reaches the folds (inactive lanes carry zeros)
+        for (int o = p.lanes >> 1; o > 0; o >>= 1) {
+            gm += __shfl_xor_sync(0xffffffffu, gm, o);
+            gfx += __shfl_xor_sync(0xffffffffu, gfx, o);
+            gfy += __shfl_xor_sync(0xffffffffu, gfy, o);
+        }
+        if (active && part == 0) {
+            const float ms = m * p.offset_scale;
+            gbuf[lu * R + k] = ms * gfx;
+            gbuf[lu * R + KK + k] = ms * gfy;
+            gbuf[lu * R + 2 * KK + k] = gm;
+        }
+    }
+    __syncthreads();
+    float* dst = grad_om + static_cast<size_t>(unit0) * R;
+    for (int i = threadIdx.x; i < nunits * R; i += blockDim.x) dst[i] = gbuf[i];
+}
+
+}  // namespace dcnv4

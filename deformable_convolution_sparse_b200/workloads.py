@@ -1,4 +1,4 @@
-"""Seeded synthetic inputs for the DCNv4 forward aggregation.
+"""Seeded synthetic inputs for the DCNv4 aggregation (forward and backward).
 
 This module only draws random numbers in the shapes the operator takes. It
 holds none of the operator's arithmetic: the output extent of every named
@@ -20,7 +20,9 @@ and for the predictor's offsets and masks):
 x ~ N(0,1) everywhere. Draw order on one CPU torch.Generator: x [N,H,W,C],
 then offsets [N,Hout,Wout,G,2*K*K], then masks [N,Hout,Wout,G,K*K], all
 fp32; offsets and masks are concatenated on the last axis and the tensors are
-then rounded to the storage dtype.
+then rounded to the storage dtype. The backward's upstream gradient
+dL/dout ~ N(0,1) [N,Hout,Wout,C] comes from a second generator seeded with
+1000 + seed.
 """
 from __future__ import annotations
 
@@ -128,3 +130,20 @@ def workload_inputs(w: Workload):
     """Seeded inputs of a named workload (CPU tensors in its storage dtype)."""
     return make_inputs(w.N, w.H, w.W, w.C, w.G, w.K, w.Hout, w.Wout, w.dtype,
                        w.offsets, w.masks, seed=w.seed)
+
+
+def make_grad_out(N: int, Hout: int, Wout: int, C: int, dtype: str = "f32", seed: int = 0,
+                  dist=("normal", 0.0, 1.0)) -> torch.Tensor:
+    """Seeded upstream gradient dL/dout [N,Hout,Wout,C] (CPU tensor in ``dtype``) for the backward.
+
+    Drawn on its own generator, seeded with 1000 + seed, so that it does not
+    shift the draws of ``make_inputs``.
+    """
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(1000 + int(seed))
+    return _draw(gen, (N, Hout, Wout, C), dist).to(DTYPES[dtype]).contiguous()
+
+
+def workload_grad_out(w: Workload) -> torch.Tensor:
+    """Seeded dL/dout of a named workload (CPU tensor in its storage dtype)."""
+    return make_grad_out(w.N, w.Hout, w.Wout, w.C, w.dtype, seed=w.seed)

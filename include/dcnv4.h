@@ -1,6 +1,6 @@
 /*
  * dcnv4.h -- C ABI of libdcnv4.so, the B200 (sm_100a) DCNv4 forward spatial
- * aggregation.
+ * aggregation and its backward.
  *
  * The operation (sources by page title and section):
  *   "不只是卷积的平替：我把DCNv4塞进Stable Diffusion的U-Net里" (jsqmd.com),
@@ -124,6 +124,41 @@ DCNV4_API int dcnv4_forward(const void *x, const void *offset_mask, void *out,
                   int N, int H, int W, int C, int G, int K,
                   int stride, int pad, int dilation, float offset_scale, int dtype,
                   void *stream);
+
+/* The backward of dcnv4_forward, for training with the operator ("不只是卷积的
+ * 平替：我把DCNv4塞进Stable Diffusion的U-Net里", jsqmd.com: section 1 defines the
+ * forward, section 4 fine-tunes through it). For a loss L with
+ * dL/dout = grad_out it writes
+ *   grad_x[n,y,x,c]   = sum over the in-bounds corners (y, x) of every point
+ *                       that reads them of m_k * W_corner * grad_out[...,c],
+ *   grad_offset_mask  = per (n, ho, wo, g) record, the same layout as
+ *                       offset_mask: [m_k*s*dL/dfx_k (K*K) | m_k*s*dL/dfy_k
+ *                       (K*K) | dL/dm_k (K*K)], dL/dm_k being the sum over
+ *                       the group's channels of grad_out times the bilinear
+ *                       sample, and dL/dfx_k, dL/dfy_k the derivatives of that
+ *                       sum with respect to the fractional parts of the
+ *                       sample position (s = offset_scale). At an integer
+ *                       position the cell of floor(s*r) is used (the
+ *                       derivative from above); a point whose offset is not
+ *                       finite or that has no corner inside gets zero offset
+ *                       and mask gradients and adds nothing to grad_x.
+ * x: device, T [N,H,W,C]; offset_mask: device, T [N,Hout,Wout,G,3*K*K];
+ * grad_out: device, T [N,Hout,Wout,C] (read only, may overlap x or
+ * offset_mask); grad_x: device, fp32 [N,H,W,C], fully overwritten (cleared on
+ * `stream` first); grad_offset_mask: device, fp32 [N,Hout,Wout,G,3*K*K],
+ * fully overwritten. All buffers are caller-owned; nothing is allocated or
+ * kept. Arithmetic is fp32. grad_x sums its contributions with fp32
+ * reductions whose order is not fixed, so it can differ in the last bits
+ * from run to run; grad_offset_mask is deterministic.
+ * Checks as dcnv4_validate (with grad_out in place of out), plus: grad_x and
+ * grad_offset_mask non-NULL and 4-byte aligned, overlapping neither each
+ * other nor any input (DCNV4_ERR_ALIAS). On success a clear and one kernel
+ * are queued on `stream` (nothing when N == 0) and DCNV4_OK is returned. */
+DCNV4_API int dcnv4_backward(const void *x, const void *offset_mask, const void *grad_out,
+                   float *grad_x, float *grad_offset_mask,
+                   int N, int H, int W, int C, int G, int K,
+                   int stride, int pad, int dilation, float offset_scale, int dtype,
+                   void *stream);
 
 /* The integer half of the forward, exposed so that it can be compared bit for
  * bit: for every sampling point (n, ho, wo, g, k) it writes the top-left

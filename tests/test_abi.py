@@ -128,3 +128,40 @@ def test_binding_refuses_cpu_tensors():
     om = torch.zeros(1, 8, 8, 2, 27)
     with pytest.raises(ValueError, match="CUDA"):
         B.forward(x, om, G=2, K=3, pad=1)
+
+
+GX, GOM = 0x40000000, 0x50000000
+
+
+def _bw(x=X, om=OM, go=OUT, gx=GX, gom=GOM, **kw):
+    a = dict(GOOD)
+    a.update(kw)
+    return B.load_library().dcnv4_backward(x, om, go, gx, gom, a["N"], a["H"], a["W"], a["C"], a["G"], a["K"],
+                                           a["stride"], a["pad"], a["dilation"], a["offset_scale"], a["dtype"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(x=0), "DCNV4_ERR_NULL"), (dict(go=0), "DCNV4_ERR_NULL"), (dict(gx=0), "DCNV4_ERR_NULL"),
+    (dict(gom=0), "DCNV4_ERR_NULL"),
+    (dict(N=-1), "DCNV4_ERR_SHAPE"), (dict(K=17), "DCNV4_ERR_SHAPE"), (dict(C=18, G=4), "DCNV4_ERR_GROUPS"),
+    (dict(dtype=7), "DCNV4_ERR_DTYPE"), (dict(offset_scale=float("nan")), "DCNV4_ERR_SCALE"),
+    (dict(go=OUT + 1), "DCNV4_ERR_ALIGN"), (dict(gx=GX + 2), "DCNV4_ERR_ALIGN"), (dict(gom=GOM + 2), "DCNV4_ERR_ALIGN"),
+    # outputs may not overlap any input nor each other
+    (dict(gx=X), "DCNV4_ERR_ALIAS"), (dict(gx=OUT + 64), "DCNV4_ERR_ALIAS"), (dict(gom=OM + 16), "DCNV4_ERR_ALIAS"),
+    (dict(gom=GX + 64), "DCNV4_ERR_ALIAS"),
+    (dict(N=1 << 20, H=64, W=64, C=64, G=4), "DCNV4_ERR_TOO_LARGE"),
+])
+def test_backward_reports_each_error_class_before_any_cuda_call(kw, status):
+    assert _bw(**kw) == B.STATUS[status]
+
+
+def test_backward_empty_batch_touches_nothing():
+    assert _bw(x=0, om=0, go=0, gx=0, gom=0, N=0) == B.DCNV4_OK
+
+
+def test_backward_binding_refuses_cpu_tensors():
+    import torch
+    x = torch.zeros(1, 8, 8, 16)
+    om = torch.zeros(1, 8, 8, 2, 27)
+    with pytest.raises(ValueError, match="CUDA"):
+        B.backward(x, om, torch.zeros(1, 8, 8, 16), G=2, K=3, pad=1)
