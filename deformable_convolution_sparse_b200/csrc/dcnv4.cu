@@ -377,15 +377,14 @@ int launch_forward(const void* x, const void* om, void* out, FwdParams p, cudaSt
 }
 
 // Backward: grad_x is cleared on the stream, then one kernel computes every
-// gradient. Vector path (16-byte channel chunks, float4 reductions) when the
-// pointers and channel rows allow it, element path otherwise.
+// gradient. Vector path (4 channels per thread, float4 reductions) when the
+// pointers and channel counts allow it, element path otherwise.
 template <typename T>
 int launch_backward(const void* x, const void* om, const void* go, float* gx, float* gom, FwdParams p,
                     cudaStream_t stream) {
     constexpr int E = sizeof(T);
-    const bool vec = aligned(x, 16) && aligned(go, 16) && aligned(gx, 16) && (p.C * E) % 16 == 0 &&
-                     (p.Cg * E) % 16 == 0;
-    const int cpl = vec ? 16 / E : 1;
+    const bool vec = aligned(x, 4 * E) && aligned(go, 4 * E) && aligned(gx, 16) && p.C % 4 == 0 && p.Cg % 4 == 0;
+    const int cpl = vec ? 4 : 1;
     p.chunks = p.Cg / cpl;
     int lanes = 1;
     while (lanes < p.chunks && lanes < 32) lanes <<= 1;
@@ -418,7 +417,7 @@ int launch_backward(const void* x, const void* om, const void* go, float* gx, fl
         return launch_status();
     };
     const bool k3 = p.K == 3;
-    if (vec) return k3 ? run(dcnv4::bwd_kernel<T, 16 / E, 3>) : run(dcnv4::bwd_kernel<T, 16 / E, 0>);
+    if (vec) return k3 ? run(dcnv4::bwd_kernel<T, 4, 3>) : run(dcnv4::bwd_kernel<T, 4, 0>);
     return k3 ? run(dcnv4::bwd_kernel<T, 1, 3>) : run(dcnv4::bwd_kernel<T, 1, 0>);
 }
 

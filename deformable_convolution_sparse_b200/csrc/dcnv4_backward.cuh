@@ -14,14 +14,20 @@
 //
 // Design (B200): like the forward, a gather that runs on the CUDA cores. A
 // unit is one (pixel, group); `p.lanes` (a power of two <= 32) threads share
-// it, each owning 16 bytes of its channels per pass. Per point the four corner
+// it, each owning 4 of its channels per pass (one float4 of the gradient). Per point the four corner
 // vectors are loaded once and give, per channel, the top and bottom row
 // interpolants t and b: S = t + fy (b - t), dS/dfy = b - t and
 // dS/dfx = (x01 - x00) + fy ((x11 - x10) - (x01 - x00)); the three channel
 // sums are folded across the unit's lanes with xor shuffles. The x gradient is
 // a scatter: each in-bounds corner gets m W go as fp32 vector reductions
 // (`atomicAdd` on float4, resolved in L2), so its summation order, and only
-// its, is not deterministic. The offset/mask gradient of the block's units is
+// its, is not deterministic. These reductions bound the kernel: the requests
+// they send from L1 to the L2 keep that path nearly saturated, so one warp
+// instruction covers a unit's whole group slice of a corner (its lanes write
+// adjacent float4s, which leave L1 as one request per 128-byte line).
+// Accumulating a tile's contributions in shared memory first was tried and is
+// several times slower: fp32 reductions into shared memory cost more than
+// these L2 ones. The offset/mask gradient of the block's units is
 // collected in shared memory and written out as one contiguous run.
 #pragma once
 
@@ -29,11 +35,18 @@
 
 namespace dcnv4 {
 
-// CPL channels of storage type T at p (16 bytes when CPL > 1) -> floats
+// CPL channels of storage type T at p (8 or 16 bytes when CPL > 1) -> floats
 template <typename T, int CPL>
 __device__ __forceinline__ void load_channels(const T* p, float (&v)[CPL]) {
     if constexpr (CPL == 1) {
         v[0] = ElemTraits<T>::to_float(__ldg(p));
+    } else if constexpr (CPL * sizeof(T) == 8) {
+        const uint2 w = __ldg(reinterpret_cast<const uint2*>(p));
+        const float2 a = unpack2(w.x, static_cast<T*>(nullptr)), b = unpack2(w.y, static_cast<T*>(nullptr));
+        v[0] = a.x;
+        v[1] = a.y;
+        v[2] = b.x;
+        v[3] = b.y;
     } else {
         static_assert(CPL * sizeof(T) == 16, "vector chunks are 16 bytes");
         uint32_t w[4];
