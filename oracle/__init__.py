@@ -57,6 +57,8 @@ def _load():
         lib.oracle_dcnv4_sampling_index.restype = i
         lib.oracle_dcnv4_backward.argtypes = [p] * 5 + [i] * 9 + [f]
         lib.oracle_dcnv4_backward.restype = i
+        lib.oracle_dcnv4_forward_variants.argtypes = [p] * 4 + [i] * 9 + [f, i, i, i]
+        lib.oracle_dcnv4_forward_variants.restype = i
         _lib = lib
     return _lib
 
@@ -100,6 +102,38 @@ def dcnv4_forward(x, offset_mask, G: int, K: int, stride: int = 1, pad: int = 0,
                                              stride, pad, dilation, float(offset_scale),
                                              0 if n_begin is None else n_begin,
                                              N if n_end is None else n_end)
+    if rc != 0:
+        raise ValueError("oracle rejected the arguments")
+    return out
+
+
+def dcnv4_forward_variants(x, offset_mask, G: int, K: int, stride: int = 1, pad: int = 0, dilation: int = 1,
+                           offset_scale: float = 1.0, softmax: bool = False, remove_center: bool = False,
+                           center_logit=None) -> np.ndarray:
+    """fp64 forward with the variant switches (see dcnv4_oracle.c for the readings).
+
+    softmax: DCNv3-style softmax over each unit's masks; remove_center: P = K*K-1
+    points per unit, record [N,Hout,Wout,G,3*P]; center_logit [N,Hout,Wout,G]:
+    centre feature scaling with gate sigmoid(center_logit) (None: off).
+    """
+    x = _f64(x)
+    om = _f64(offset_mask)
+    N, H, W, C = x.shape
+    Hout, Wout = output_size(H, K, stride, pad, dilation), output_size(W, K, stride, pad, dilation)
+    P = K * K - (1 if remove_center else 0)
+    if om.shape != (N, Hout, Wout, G, 3 * P):
+        raise ValueError(f"offset_mask shape {om.shape} != {(N, Hout, Wout, G, 3 * P)}")
+    z = None
+    if center_logit is not None:
+        z = _f64(center_logit)
+        if z.shape != (N, Hout, Wout, G):
+            raise ValueError("center_logit must be [N,Hout,Wout,G]")
+    out = np.zeros((N, Hout, Wout, C), dtype=np.float64)
+    if N == 0:
+        return out
+    rc = _load().oracle_dcnv4_forward_variants(_ptr(x), _ptr(om), None if z is None else _ptr(z), _ptr(out),
+                                               N, H, W, C, G, K, stride, pad, dilation, float(offset_scale),
+                                               int(bool(softmax)), int(bool(remove_center)), int(z is not None))
     if rc != 0:
         raise ValueError("oracle rejected the arguments")
     return out

@@ -193,6 +193,100 @@ int oracle_dcnv4_sampling_index(const double *om, int32_t *corner, uint8_t *vali
 }
 
 /* ------------------------------------------------------------------------
+ * Variants of the forward. "掌握DCNv4技术" (pwwt.cn), section on advanced
+ * tuning and extension: DCNv4 also offers centre feature scaling (a sigmoid
+ * that weighs the feature at the centre against the aggregate) and the
+ * removal of the centre point. "不只是卷积的平替" (jsqmd.com), section 1:
+ * DCNv3 normalised the K*K aggregation weights with a softmax, which DCNv4
+ * drops; the flag below restores it for comparison.
+ *
+ * Readings taken here (the pages give no formulas):
+ *  - softmax: per (n, ho, wo, g), m'_j = exp(m_j - max) / sum_i exp(m_i - max)
+ *    over the unit's points, then the aggregation of the forward with m';
+ *  - remove_center (K odd, K >= 3): the unit has P = K*K - 1 points, its
+ *    record is [dx_0..dx_{P-1} | dy_0..dy_{P-1} | m_0..m_{P-1}], and point j
+ *    sits on grid index k = j for j < (K*K-1)/2 and k = j + 1 after it (the
+ *    centre grid index (K*K-1)/2 is skipped);
+ *  - centre feature scaling: with a logit z[n,ho,wo,g] given as input,
+ *    s = 1 / (1 + exp(-z)) and out = (1 - s) * aggregate + s * x_c, where
+ *    x_c is x at the centre grid position (ho*stride - pad + (K/2)*dilation,
+ *    wo*stride - pad + (K/2)*dilation) of channel g*Cg + c, zero outside the
+ *    image (for stride 1 and pad = dilation*(K-1)/2 that is the output pixel
+ *    itself).
+ * center_logit: [N,Hout,Wout,G] (read only when center_scale != 0).
+ * ------------------------------------------------------------------------ */
+int oracle_dcnv4_forward_variants(const double *x, const double *om, const double *center_logit, double *out,
+                                  int N, int H, int W, int C, int G, int K,
+                                  int stride, int pad, int dilation, float offset_scale,
+                                  int softmax, int remove_center, int center_scale)
+{
+    if (N < 0 || H <= 0 || W <= 0 || C <= 0 || G <= 0 || K <= 0 || K > 16 || C % G) return -1;
+    if (remove_center && (K % 2 == 0 || K < 3)) return -1;
+    if (center_scale && !center_logit) return -1;
+    const int Hout = oracle_output_size(H, K, stride, pad, dilation);
+    const int Wout = oracle_output_size(W, K, stride, pad, dilation);
+    if (Hout <= 0 || Wout <= 0) return -1;
+    const int Cg = C / G, KK = K * K;
+    const int centre = (KK - 1) / 2;
+    const int P = remove_center ? KK - 1 : KK;
+    double mk[256];
+    for (int n = 0; n < N; ++n)
+        for (int ho = 0; ho < Hout; ++ho)
+            for (int wo = 0; wo < Wout; ++wo)
+                for (int g = 0; g < G; ++g) {
+                    const size_t unit = (((size_t)n * Hout + ho) * Wout + wo) * G + g;
+                    const double *r = om + unit * (size_t)(3 * P);
+                    double *o = out + (((size_t)n * Hout + ho) * Wout + wo) * (size_t)C + (size_t)g * Cg;
+                    /* the aggregation weights, optionally through a softmax over the unit's points */
+                    if (softmax) {
+                        double mx = r[2 * P];
+                        for (int j = 1; j < P; ++j)
+                            if (r[2 * P + j] > mx) mx = r[2 * P + j];
+                        double sum = 0.0;
+                        for (int j = 0; j < P; ++j) sum += exp(r[2 * P + j] - mx);
+                        for (int j = 0; j < P; ++j) mk[j] = exp(r[2 * P + j] - mx) / sum;
+                    } else {
+                        for (int j = 0; j < P; ++j) mk[j] = r[2 * P + j];
+                    }
+                    for (int c = 0; c < Cg; ++c) o[c] = 0.0;
+                    for (int j = 0; j < P; ++j) {
+                        const int k = (remove_center && j >= centre) ? j + 1 : j;
+                        const int ky = k / K, kx = k % K;
+                        const int p0y = ho * stride - pad + ky * dilation;
+                        const int p0x = wo * stride - pad + kx * dilation;
+                        const double dx = scaled_offset(offset_scale, r[j]);
+                        const double dy = scaled_offset(offset_scale, r[P + j]);
+                        if (!isfinite(dx) || !isfinite(dy)) continue;
+                        const double fy0 = floor(dy), fx0 = floor(dx);
+                        const double ly = dy - fy0, lx = dx - fx0;
+                        const double y0 = (double)p0y + fy0, x0 = (double)p0x + fx0;
+                        for (int a = 0; a <= 1; ++a)
+                            for (int b = 0; b <= 1; ++b) {
+                                const double yy = y0 + a, xx = x0 + b;
+                                if (!(yy >= 0.0 && yy <= (double)(H - 1) && xx >= 0.0 && xx <= (double)(W - 1)))
+                                    continue;
+                                const double w = mk[j] * (a ? ly : 1.0 - ly) * (b ? lx : 1.0 - lx);
+                                const double *px = x + ((((size_t)n * H + (size_t)yy) * W + (size_t)xx) * C) + (size_t)g * Cg;
+                                for (int c = 0; c < Cg; ++c) o[c] += w * px[c];
+                            }
+                    }
+                    if (center_scale) {
+                        const double sg = 1.0 / (1.0 + exp(-center_logit[unit]));
+                        const int cy = ho * stride - pad + (K / 2) * dilation;
+                        const int cx = wo * stride - pad + (K / 2) * dilation;
+                        const int inside = cy >= 0 && cy < H && cx >= 0 && cx < W;
+                        const double *px = x + ((((size_t)n * H + (size_t)(inside ? cy : 0)) * W +
+                                                 (size_t)(inside ? cx : 0)) * C) + (size_t)g * Cg;
+                        for (int c = 0; c < Cg; ++c) {
+                            const double xc = inside ? px[c] : 0.0;
+                            o[c] = (1.0 - sg) * o[c] + sg * xc;
+                        }
+                    }
+                }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------
  * Backward of the forward above (the training direction; the pages use the
  * operator for training, e.g. the Stable Diffusion fine-tuning of the
  * jsqmd.com page, section 4). For a loss L with dL/dout = grad_out:
