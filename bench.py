@@ -17,6 +17,10 @@ exceeds the L2 cache, so no step starts with its inputs in L2.
 
 --impl reference times the fp64 CPU oracle (the reference arm of this
 repository: there is no other implementation to install) on the host cores.
+
+Secondary lines (not the headline): --pass backward times dcnv4_backward on
+the same workload; --variant softmax|remove_center|center_scale|all times
+dcnv4_forward_ex with those variant flags.
 """
 from __future__ import annotations
 
@@ -53,6 +57,9 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--pass", dest="which", choices=["forward", "backward"], default="forward",
                     help="forward (the headline) or the backward of the same workload")
+    ap.add_argument("--variant", choices=["none", "softmax", "remove_center", "center_scale", "all"],
+                    default="none", help="forward variant flags (DCNv3 softmax, centre point removed, "
+                                         "centre feature scaling, or all three)")
     return ap.parse_args()
 
 
@@ -349,6 +356,128 @@ def run_backward(args, w, dev, world, rank, barrier, max_over_ranks):
         print(json.dumps(line), flush=True)
 
 
+VARIANT_FLAGS = {"softmax": 1, "remove_center": 2, "center_scale": 4, "all": 7}
+
+
+def run_variant(args, w, dev, world, rank, barrier, max_over_ranks):
+    """The forward with variant flags (dcnv4_forward_ex), inputs rotating over resident sets larger than L2."""
+    import torch
+    import deformable_convolution_sparse_b200 as dcn
+    from deformable_convolution_sparse_b200.workloads import make_center_logit, make_inputs
+
+    flags = VARIANT_FLAGS[args.variant]
+    P = w.K * w.K - (1 if flags & 2 else 0)
+    wr = w.with_(seed=w.seed + 1000 * rank)
+    x, om = make_inputs(w.N, w.H, w.W, w.C, w.G, w.K, w.Hout, w.Wout, w.dtype, w.offsets, w.masks, seed=wr.seed,
+                        points=P)
+    z = make_center_logit(w.N, w.Hout, w.Wout, w.G, w.dtype, seed=wr.seed)
+    lib = dcn.load_library()
+    dtype_code = dcn.binding.TORCH_DTYPE[x.dtype]
+    e = x.element_size()
+    nout = w.N * w.Hout * w.Wout * w.C
+    # algorithmic bytes: x, offset_mask (and the gate logits) read once, out written once
+    foot = (x.numel() + om.numel() + nout + (z.numel() if flags & 4 else 0)) * e
+    points = w.N * w.Hout * w.Wout * w.G * P
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    copies = max(3, math.ceil(3 * l2 / foot))
+    sets = [(x.to(dev), om.to(dev), z.to(dev), torch.empty((w.N, w.Hout, w.Wout, w.C), dtype=x.dtype, device=dev))
+            for _ in range(copies)]
+    stream = torch.cuda.current_stream(dev)
+    sh = stream.cuda_stream
+    launches = [0]
+
+    def call(xd, omd, zd, od):
+        rc = lib.dcnv4_forward_ex(xd.data_ptr(), omd.data_ptr(), zd.data_ptr(), od.data_ptr(), w.N, w.H, w.W, w.C,
+                                  w.G, w.K, w.stride, w.pad, w.dilation, w.offset_scale, dtype_code, flags, sh)
+        if rc != 0:
+            raise dcn.DCNv4Error(rc, "dcnv4_forward_ex")
+
+    def step(i):
+        call(*sets[i % copies])
+        launches[0] += 1
+
+    ms, sampler, timed_launches = time_steps(step, launches, args, dev, stream, barrier, max_over_ranks)
+    ms_step = ms / args.steps
+    value = points * world * args.steps / (ms / 1e3) / 1e9
+    peak, peak_kind = measured_peaks()
+    achieved = foot / (ms_step / 1e3) / 1e9
+
+    xh, omh, zh = x.pin_memory(), om.pin_memory(), z.pin_memory()
+    oh = torch.empty((w.N, w.Hout, w.Wout, w.C), dtype=x.dtype).pin_memory()
+    xd, omd, zd, od = sets[0]
+
+    def e2e_step():
+        xd.copy_(xh, non_blocking=True)
+        omd.copy_(omh, non_blocking=True)
+        if flags & 4:
+            zd.copy_(zh, non_blocking=True)
+        call(xd, omd, zd, od)
+        oh.copy_(od, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1))
+    e2e_value = points * world * args.e2e_steps / (e2e_ms / 1e3) / 1e9
+    if not torch.equal(oh, od.cpu()):
+        raise SystemExit("end-to-end result differs from the device-resident result")
+
+    base = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        xd64, omd64, z64 = x[:1].double().numpy(), om[:1].double().numpy(), z[:1].double().numpy()
+        kw = dict(G=w.G, K=w.K, stride=w.stride, pad=w.pad, dilation=w.dilation, offset_scale=w.offset_scale,
+                  softmax=bool(flags & 1), remove_center=bool(flags & 2), center_logit=z64 if flags & 4 else None)
+        oracle.dcnv4_forward_variants(xd64, omd64, **kw)
+        n_s = min(w.N, 8)
+        kw["center_logit"] = z[:n_s].double().numpy() if flags & 4 else None
+        xs64, oms64 = x[:n_s].double().numpy(), om[:n_s].double().numpy()
+        t0 = time.perf_counter()
+        oracle.dcnv4_forward_variants(xs64, oms64, **kw)
+        dt = time.perf_counter() - t0
+        base = {"value": points // w.N * n_s / dt / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
+                "seconds": dt, "sample": f"{n_s} of {w.N} images, fp64 C oracle ({args.variant}), one thread"}
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic", "variant": args.variant,
+            "config": {
+                "workload": f"{w.name} forward, variant {args.variant}: N={w.N} per GPU, H=W={w.H}, C={w.C}, "
+                            f"G={w.G}, K={w.K}, {P} points per unit",
+                "storage_dtype": w.dtype, "accumulate": "f32", "global_batch": w.N * world,
+                "points_per_step_per_gpu": points, "parallelism": f"dp{world} (independent batches)",
+                "l2": f"steps rotate over {copies} resident sets, {copies * foot / 1e6:.0f} MB in total vs "
+                      f"{l2 / 1e6:.0f} MB L2",
+                "inputs": "seeded synthetic as the plain forward; gate logits ~N(0,1.5^2)",
+            },
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak,
+                         "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json)"
+                         if peak_kind == "measured" else "fallback 6.65 TB/s",
+                         "kernel": "dcnv4 forward with variant flags (one launch per step)",
+                         "algorithmic_bytes_per_launch": foot, "traffic": None},
+            "e2e": {"value": e2e_value, "unit": UNIT, "ms_per_step": e2e_ms / args.e2e_steps,
+                    "steps": args.e2e_steps,
+                    "h2d_bytes_per_step": (x.numel() + om.numel() + (z.numel() if flags & 4 else 0)) * e,
+                    "d2h_bytes_per_step": nout * e,
+                    "path": "pinned host tensors copied in, dcnv4_forward_ex, result copied out, one stream"},
+            "gpu_launches": timed_launches,
+            "clocks": sampler.summary(),
+            "cpu_baseline": base,
+        }
+        print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
@@ -383,8 +512,11 @@ def main():
         return float(t.item())
 
     w = WORKLOADS[args.workload or BENCH_WORKLOAD]
-    if args.which == "backward":
-        run_backward(args, w, dev, world, rank, barrier, max_over_ranks)
+    if args.which == "backward" or args.variant != "none":
+        if args.which == "backward":
+            run_backward(args, w, dev, world, rank, barrier, max_over_ranks)
+        else:
+            run_variant(args, w, dev, world, rank, barrier, max_over_ranks)
         if world > 1:
             dist.destroy_process_group()
         return

@@ -22,12 +22,16 @@ STATUS_NAMES = {
     0: "DCNV4_OK", 1: "DCNV4_ERR_NULL", 2: "DCNV4_ERR_SHAPE", 3: "DCNV4_ERR_GROUPS",
     4: "DCNV4_ERR_DTYPE", 5: "DCNV4_ERR_ALIGN", 6: "DCNV4_ERR_ALIAS", 7: "DCNV4_ERR_SCALE",
     8: "DCNV4_ERR_TOO_LARGE", 9: "DCNV4_ERR_LAUNCH", 10: "DCNV4_ERR_CUDA", 11: "DCNV4_ERR_STAGING",
+    12: "DCNV4_ERR_FLAGS",
 }
+# variant switches of dcnv4_forward_ex
+FLAG_SOFTMAX, FLAG_REMOVE_CENTER, FLAG_CENTER_SCALE = 1, 2, 4
 STATUS = {v: k for k, v in STATUS_NAMES.items()}
 TORCH_DTYPE = {torch.float32: DCNV4_F32, torch.float16: DCNV4_F16, torch.bfloat16: DCNV4_BF16}
 
 # every symbol include/dcnv4.h declares
-EXPORTS = ("dcnv4_output_shape", "dcnv4_validate", "dcnv4_forward", "dcnv4_backward", "dcnv4_sampling_index",
+EXPORTS = ("dcnv4_output_shape", "dcnv4_validate", "dcnv4_validate_ex", "dcnv4_forward", "dcnv4_forward_ex",
+           "dcnv4_backward", "dcnv4_sampling_index",
            "dcnv4_forward_host", "dcnv4_forward_host_noalloc", "dcnv4_device_status", "dcnv4_selftest_wait_timeout", "dcnv4_strerror",
            "dcnv4_abi_version")
 DEVSTATUS_COPY_TIMEOUT, DEVSTATUS_SELFTEST_TIMEOUT = 1, 2
@@ -59,6 +63,10 @@ def load_library():
     lib.dcnv4_validate.restype = i
     lib.dcnv4_forward.argtypes = [p, p, p] + [i] * 9 + [f, i, p]
     lib.dcnv4_forward.restype = i
+    lib.dcnv4_validate_ex.argtypes = [p] * 4 + [i] * 9 + [f, i, ctypes.c_uint]
+    lib.dcnv4_validate_ex.restype = i
+    lib.dcnv4_forward_ex.argtypes = [p] * 4 + [i] * 9 + [f, i, ctypes.c_uint, p]
+    lib.dcnv4_forward_ex.restype = i
     lib.dcnv4_backward.argtypes = [p] * 5 + [i] * 9 + [f, i, p]
     lib.dcnv4_backward.restype = i
     lib.dcnv4_sampling_index.argtypes = [p, p, p] + [i] * 8 + [f, i, p]
@@ -139,12 +147,17 @@ def _check_tensor(t: torch.Tensor, name: str):
 
 def forward(x: torch.Tensor, offset_mask: torch.Tensor, G: int, K: int, stride: int = 1, pad: int = 0,
             dilation: int = 1, offset_scale: float = 1.0, out: torch.Tensor | None = None,
-            stream=None) -> torch.Tensor:
-    """DCNv4 forward aggregation on the GPU through ``dcnv4_forward``.
+            stream=None, softmax: bool = False, remove_center: bool = False,
+            center_logit: torch.Tensor | None = None) -> torch.Tensor:
+    """DCNv4 forward aggregation on the GPU through ``dcnv4_forward`` / ``dcnv4_forward_ex``.
 
-    x: [N,H,W,C]; offset_mask: [N,Hout,Wout,G,3*K*K] (per group: K*K x-offsets,
-    K*K y-offsets, K*K masks); returns out [N,Hout,Wout,C] in x's dtype. The
-    launch is asynchronous on ``stream`` (default: the current stream).
+    x: [N,H,W,C]; offset_mask: [N,Hout,Wout,G,3*P] (per group: P x-offsets,
+    P y-offsets, P masks; P = K*K, or K*K-1 with ``remove_center``); returns
+    out [N,Hout,Wout,C] in x's dtype. Variants: ``softmax`` (DCNv3-style
+    softmax over each unit's masks), ``remove_center`` (the centre grid point
+    is left out), ``center_logit`` [N,Hout,Wout,G] (centre feature scaling with
+    gate sigmoid(center_logit)). The launch is asynchronous on ``stream``
+    (default: the current stream).
     """
     _check_tensor(x, "x")
     _check_tensor(offset_mask, "offset_mask")
@@ -154,9 +167,19 @@ def forward(x: torch.Tensor, offset_mask: torch.Tensor, G: int, K: int, stride: 
         raise ValueError("offset_mask must match x in dtype and device")
     N, H, W, C = x.shape
     Hout, Wout = output_shape(H, W, K, stride, pad, dilation)
-    want = (N, Hout, Wout, G, 3 * K * K)
+    P = K * K - (1 if remove_center else 0)
+    want = (N, Hout, Wout, G, 3 * P)
     if tuple(offset_mask.shape) != want:
         raise ValueError(f"offset_mask shape {tuple(offset_mask.shape)} != {want}")
+    flags = (FLAG_SOFTMAX if softmax else 0) | (FLAG_REMOVE_CENTER if remove_center else 0)
+    zp = 0
+    if center_logit is not None:
+        _check_tensor(center_logit, "center_logit")
+        if tuple(center_logit.shape) != (N, Hout, Wout, G) or center_logit.dtype != x.dtype or \
+                center_logit.device != x.device:
+            raise ValueError(f"center_logit must be [N,Hout,Wout,G] = {(N, Hout, Wout, G)} in x's dtype and device")
+        flags |= FLAG_CENTER_SCALE
+        zp = center_logit.data_ptr()
     if out is None:
         out = torch.empty((N, Hout, Wout, C), dtype=x.dtype, device=x.device)
     else:
@@ -164,11 +187,17 @@ def forward(x: torch.Tensor, offset_mask: torch.Tensor, G: int, K: int, stride: 
         if tuple(out.shape) != (N, Hout, Wout, C) or out.dtype != x.dtype or out.device != x.device:
             raise ValueError("out has the wrong shape, dtype or device")
     with torch.cuda.device(x.device):
-        rc = load_library().dcnv4_forward(x.data_ptr(), offset_mask.data_ptr(), out.data_ptr(), N, H, W, C, G, K,
-                                          stride, pad, dilation, float(offset_scale), TORCH_DTYPE[x.dtype],
-                                          _stream_handle(stream))
+        lib = load_library()
+        if flags:
+            rc = lib.dcnv4_forward_ex(x.data_ptr(), offset_mask.data_ptr(), zp, out.data_ptr(), N, H, W, C, G, K,
+                                      stride, pad, dilation, float(offset_scale), TORCH_DTYPE[x.dtype], flags,
+                                      _stream_handle(stream))
+        else:
+            rc = lib.dcnv4_forward(x.data_ptr(), offset_mask.data_ptr(), out.data_ptr(), N, H, W, C, G, K,
+                                   stride, pad, dilation, float(offset_scale), TORCH_DTYPE[x.dtype],
+                                   _stream_handle(stream))
     if rc != DCNV4_OK:
-        raise DCNv4Error(rc, "dcnv4_forward")
+        raise DCNv4Error(rc, "dcnv4_forward_ex" if flags else "dcnv4_forward")
     return out
 
 

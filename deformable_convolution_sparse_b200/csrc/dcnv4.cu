@@ -140,7 +140,7 @@ bool plan_tile(const void* x, const void* om, const void* out, const FwdParams& 
     if (const char* n = std::getenv("DCNV4_NREC")) forceNrec = (std::atoi(n) == 2 || std::atoi(n) == 3) ? std::atoi(n) : 0;
     if (const char* t = std::getenv("DCNV4_TILE")) std::sscanf(t, "%dx%d", &forceTH, &forceTW);
     if (const char* g = std::getenv("DCNV4_GS")) forceGS = std::atoi(g);
-    const int R3 = 3 * f.KK;
+    const int R3 = 3 * f.npts;
     const int nsm = sm_count();
     if (nsm <= 0) return false;
 
@@ -264,9 +264,9 @@ bool f16_exact_from_env() {
     return v && *v == '1';
 }
 
-template <typename T, int Q, int KS, bool HW, int PBC>
+template <typename T, int Q, int KS, bool HW, int PBC, bool VF = false>
 int launch_tile_q(const T* x, const T* om, T* out, const TilePlan& plan, cudaStream_t stream) {
-    auto kern = dcnv4::fwd_tile_kernel<T, Q, KS, HW, PBC>;
+    auto kern = dcnv4::fwd_tile_kernel<T, Q, KS, HW, PBC, VF>;
     static std::once_flag once;
     static cudaError_t attr = cudaSuccess;
     std::call_once(once, [&] {
@@ -282,17 +282,24 @@ int launch_tile_q(const T* x, const T* om, T* out, const TilePlan& plan, cudaStr
     return launch_status();
 }
 
-template <typename T, int Q, bool HW>
-int launch_tile_k(const T* x, const T* om, T* out, const TilePlan& plan, cudaStream_t s) {
+template <typename T, int Q, bool HW, bool VF>
+int launch_tile_v(const T* x, const T* om, T* out, const TilePlan& plan, cudaStream_t s) {
     // a 128-byte window pixel (the common case) as a compile-time stride
     if constexpr (Q != 5) {
         if (plan.p.PB == 128) {
-            if (plan.p.f.K == 3) return launch_tile_q<T, Q, 3, HW, 128>(x, om, out, plan, s);
-            return launch_tile_q<T, Q, 0, HW, 128>(x, om, out, plan, s);
+            if (plan.p.f.K == 3) return launch_tile_q<T, Q, 3, HW, 128, VF>(x, om, out, plan, s);
+            return launch_tile_q<T, Q, 0, HW, 128, VF>(x, om, out, plan, s);
         }
     }
-    if (plan.p.f.K == 3) return launch_tile_q<T, Q, 3, HW, 0>(x, om, out, plan, s);
-    return launch_tile_q<T, Q, 0, HW, 0>(x, om, out, plan, s);
+    if (plan.p.f.K == 3) return launch_tile_q<T, Q, 3, HW, 0, VF>(x, om, out, plan, s);
+    return launch_tile_q<T, Q, 0, HW, 0, VF>(x, om, out, plan, s);
+}
+
+template <typename T, int Q, bool HW>
+int launch_tile_k(const T* x, const T* om, T* out, const TilePlan& plan, cudaStream_t s) {
+    // the variant flags get their own instantiations, so that the plain forward carries none of their code
+    if (plan.p.f.flags != 0) return launch_tile_v<T, Q, HW, true>(x, om, out, plan, s);
+    return launch_tile_v<T, Q, HW, false>(x, om, out, plan, s);
 }
 
 template <typename T, int Q>
@@ -327,7 +334,7 @@ int launch_forward(const void* x, const void* om, void* out, FwdParams p, cudaSt
     const int row_bytes = p.Cg * E;
     const bool a16 = aligned(x, 16) && aligned(out, 16) && (p.C * E) % 16 == 0;
     const bool a32 = aligned(x, 32) && aligned(out, 32) && (p.C * E) % 32 == 0;
-    const size_t rec_bytes = static_cast<size_t>(3) * p.KK * E;
+    const size_t rec_bytes = static_cast<size_t>(3) * p.npts * E;
 
     int lane_bytes = 0, vec_bytes = 0;
     if (a16 && row_bytes % 16 == 0) {
@@ -446,15 +453,24 @@ int host_pipe(HostPipe** out) {
 }
 
 FwdParams make_params(int N, int H, int W, int C, int G, int K, int stride, int pad, int dilation,
-                      float offset_scale, int Hout, int Wout) {
+                      float offset_scale, int Hout, int Wout, unsigned flags = 0u,
+                      const void* center_logit = nullptr) {
     FwdParams p{};
     p.N = N; p.H = H; p.W = W; p.C = C; p.G = G; p.K = K; p.KK = K * K; p.Cg = C / G;
     p.stride = stride; p.pad = pad; p.dilation = dilation;
     p.Hout = Hout; p.Wout = Wout;
     p.units = N * Hout * Wout * G;
     p.offset_scale = offset_scale;
+    p.flags = static_cast<int>(flags);
+    const bool rc = (flags & DCNV4_FLAG_REMOVE_CENTER) != 0u;
+    p.npts = p.KK - (rc ? 1 : 0);
+    p.kc = rc ? (p.KK - 1) / 2 : p.KK;
+    p.center_logit = center_logit;
     return p;
 }
+
+// Points per unit for a flag set (K*K, or K*K - 1 without the centre).
+int points_per_unit(int K, unsigned flags) { return K * K - ((flags & DCNV4_FLAG_REMOVE_CENTER) ? 1 : 0); }
 
 }  // namespace
 
@@ -476,6 +492,7 @@ const char* dcnv4_strerror(int status) {
         case DCNV4_ERR_LAUNCH: return "kernel launch failed";
         case DCNV4_ERR_CUDA: return "CUDA runtime call failed";
         case DCNV4_ERR_STAGING: return "one image does not fit half of the static staging area";
+        case DCNV4_ERR_FLAGS: return "unknown variant flag";
         default: return "unknown status";
     }
 }
@@ -497,36 +514,62 @@ int dcnv4_output_shape(int H, int W, int K, int stride, int pad, int dilation, i
     return DCNV4_OK;
 }
 
-int dcnv4_validate(const void* x, const void* offset_mask, const void* out,
-                   int N, int H, int W, int C, int G, int K,
-                   int stride, int pad, int dilation, float offset_scale, int dtype) {
+int dcnv4_validate_ex(const void* x, const void* offset_mask, const void* center_logit, const void* out,
+                      int N, int H, int W, int C, int G, int K,
+                      int stride, int pad, int dilation, float offset_scale, int dtype, unsigned flags) {
     long long nx = 0, nout = 0, nom = 0;
     int rc = check_sizes(N, H, W, C, G, K, stride, pad, dilation, offset_scale, dtype, &nx, &nout, &nom);
     if (rc) return rc;
+    if (flags & ~static_cast<unsigned>(DCNV4_FLAG_SOFTMAX | DCNV4_FLAG_REMOVE_CENTER | DCNV4_FLAG_CENTER_SCALE))
+        return DCNV4_ERR_FLAGS;
+    if ((flags & DCNV4_FLAG_REMOVE_CENTER) && (K % 2 == 0 || K < 3)) return DCNV4_ERR_SHAPE;
+    nom = nom / (3LL * K * K) * 3LL * points_per_unit(K, flags);
+    const long long ngate = nout / C * G;
     const int e = elem_size(dtype);
     if (N == 0) return DCNV4_OK;
-    if (!x || !offset_mask || !out) return DCNV4_ERR_NULL;
-    if (!aligned(x, e) || !aligned(offset_mask, e) || !aligned(out, e)) return DCNV4_ERR_ALIGN;
-    if (overlap(out, nout * e, x, nx * e) || overlap(out, nout * e, offset_mask, nom * e)) return DCNV4_ERR_ALIAS;
+    const bool cs = (flags & DCNV4_FLAG_CENTER_SCALE) != 0u;
+    if (!x || !offset_mask || !out || (cs && !center_logit)) return DCNV4_ERR_NULL;
+    if (!aligned(x, e) || !aligned(offset_mask, e) || !aligned(out, e) || (cs && !aligned(center_logit, e)))
+        return DCNV4_ERR_ALIGN;
+    if (overlap(out, nout * e, x, nx * e) || overlap(out, nout * e, offset_mask, nom * e) ||
+        (cs && overlap(out, nout * e, center_logit, ngate * e)))
+        return DCNV4_ERR_ALIAS;
     return DCNV4_OK;
 }
 
-int dcnv4_forward(const void* x, const void* offset_mask, void* out,
-                  int N, int H, int W, int C, int G, int K,
-                  int stride, int pad, int dilation, float offset_scale, int dtype,
-                  void* stream) {
-    const int rc = dcnv4_validate(x, offset_mask, out, N, H, W, C, G, K, stride, pad, dilation, offset_scale, dtype);
+int dcnv4_validate(const void* x, const void* offset_mask, const void* out,
+                   int N, int H, int W, int C, int G, int K,
+                   int stride, int pad, int dilation, float offset_scale, int dtype) {
+    return dcnv4_validate_ex(x, offset_mask, nullptr, out, N, H, W, C, G, K, stride, pad, dilation, offset_scale,
+                             dtype, 0u);
+}
+
+int dcnv4_forward_ex(const void* x, const void* offset_mask, const void* center_logit, void* out,
+                     int N, int H, int W, int C, int G, int K,
+                     int stride, int pad, int dilation, float offset_scale, int dtype, unsigned flags,
+                     void* stream) {
+    const int rc = dcnv4_validate_ex(x, offset_mask, center_logit, out, N, H, W, C, G, K, stride, pad, dilation,
+                                     offset_scale, dtype, flags);
     if (rc) return rc;
     if (N == 0) return DCNV4_OK;
     int Hout = 0, Wout = 0;
     dcnv4_output_shape(H, W, K, stride, pad, dilation, &Hout, &Wout);
-    const FwdParams p = make_params(N, H, W, C, G, K, stride, pad, dilation, offset_scale, Hout, Wout);
+    const FwdParams p = make_params(N, H, W, C, G, K, stride, pad, dilation, offset_scale, Hout, Wout, flags,
+                                    (flags & DCNV4_FLAG_CENTER_SCALE) ? center_logit : nullptr);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     switch (dtype) {
         case DCNV4_F32: return launch_forward<float>(x, offset_mask, out, p, s);
         case DCNV4_F16: return launch_forward<__half>(x, offset_mask, out, p, s);
         default: return launch_forward<__nv_bfloat16>(x, offset_mask, out, p, s);
     }
+}
+
+int dcnv4_forward(const void* x, const void* offset_mask, void* out,
+                  int N, int H, int W, int C, int G, int K,
+                  int stride, int pad, int dilation, float offset_scale, int dtype,
+                  void* stream) {
+    return dcnv4_forward_ex(x, offset_mask, nullptr, out, N, H, W, C, G, K, stride, pad, dilation, offset_scale,
+                            dtype, 0u, stream);
 }
 
 int dcnv4_backward(const void* x, const void* offset_mask, const void* grad_out,

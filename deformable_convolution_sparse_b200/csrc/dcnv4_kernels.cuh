@@ -25,8 +25,13 @@
 
 namespace dcnv4 {
 
+// Variant switches (the DCNV4_FLAG_* bits of the C ABI).
+constexpr int kFlagSoftmax = 1;       // DCNv3: softmax over each unit's masks
+constexpr int kFlagRemoveCenter = 2;  // K*K - 1 points: the centre grid point is left out
+constexpr int kFlagCenterScale = 4;   // blend with the centre feature through a sigmoid gate
+
 struct FwdParams {
-    int N, H, W, C, G, K, KK, Cg;
+    int N, H, W, C, G, K, KK, Cg;   // KK = K*K grid points
     int stride, pad, dilation;
     int Hout, Wout;
     int units;          // N * Hout * Wout * G
@@ -34,6 +39,10 @@ struct FwdParams {
     int chunks;         // channel chunks per unit (a chunk is what one thread covers per pass)
     int units_per_block;
     float offset_scale;
+    int npts;           // points per unit (record: 3 * npts elements): KK, or KK - 1 without the centre
+    int kc;             // grid index left out (the centre), KK when none is
+    int flags;          // kFlag* bits
+    const void* center_logit;  // [N,Hout,Wout,G] gate logits (kFlagCenterScale), storage type of x
 };
 
 // ---------------------------------------------------------------- elements ---
@@ -182,6 +191,41 @@ __device__ __forceinline__ Sample locate(int p0y, int p0x, float ry, float rx, f
     return s;
 }
 
+// ------------------------------------------------------------ variants ---
+
+// The masks a unit aggregates with: raw (DCNv4), or softmax-normalised over
+// the unit's points (DCNv3, kFlagSoftmax): m'_j = exp(m_j - max) / sum.
+struct MaskNorm {
+    float mmax, inv;
+    bool on;
+};
+template <typename T>
+__device__ __forceinline__ MaskNorm mask_norm(const T* masks, int np, int flags) {
+    MaskNorm r{0.f, 1.f, (flags & kFlagSoftmax) != 0};
+    if (r.on) {
+        float mx = -INFINITY;
+        for (int j = 0; j < np; ++j) mx = fmaxf(mx, ElemTraits<T>::to_float(masks[j]));
+        float sum = 0.f;
+        for (int j = 0; j < np; ++j) sum += expf(ElemTraits<T>::to_float(masks[j]) - mx);
+        r.mmax = mx;
+        r.inv = 1.f / sum;
+    }
+    return r;
+}
+__device__ __forceinline__ float mask_value(float raw, const MaskNorm& n) {
+    return n.on ? expf(raw - n.mmax) * n.inv : raw;
+}
+
+// Gate of the centre feature scaling: sigmoid of the unit's logit.
+template <typename T>
+__device__ __forceinline__ float center_gate(const FwdParams& p, size_t unit) {
+    const float z = ElemTraits<T>::to_float(static_cast<const T*>(p.center_logit)[unit]);
+    return 1.f / (1.f + expf(-z));
+}
+
+// Grid index of point j of a unit (the centre, when left out, is skipped).
+__device__ __forceinline__ int grid_index(int j, int kc) { return j + (j >= kc ? 1 : 0); }
+
 __device__ __forceinline__ void unit_coords(int unit, const FwdParams& p, int& n, int& ho, int& wo, int& g) {
     g = unit % p.G;
     int pix = unit / p.G;
@@ -206,7 +250,8 @@ fwd_vector_kernel(const T* __restrict__ x, const T* __restrict__ om, T* __restri
     constexpr int CPL = LB / E;         // channels per thread per pass
     const int K = KS > 0 ? KS : p.K;
     const int KK = K * K;
-    const int R = 3 * KK;
+    const int NP = p.npts;
+    const int R = 3 * NP;
 
     const int unit0 = blockIdx.x * p.units_per_block;
     const int nunits = min(p.units_per_block, p.units - unit0);
@@ -224,6 +269,7 @@ fwd_vector_kernel(const T* __restrict__ x, const T* __restrict__ om, T* __restri
     const int rowC = p.W * p.C;
     const T* ximg = x + static_cast<size_t>(n) * p.H * rowC;
     T* o = out + (static_cast<size_t>((n * p.Hout + ho) * p.Wout + wo)) * p.C + g * p.Cg;
+    const MaskNorm mn = mask_norm(rec + 2 * NP, NP, p.flags);
 
     for (int ch = part; ch < p.chunks; ch += p.lanes) {
         const int c0 = g * p.Cg + ch * CPL;   // first channel of this thread's slice
@@ -233,12 +279,14 @@ fwd_vector_kernel(const T* __restrict__ x, const T* __restrict__ om, T* __restri
 
 #pragma unroll (KS > 0 ? KS * KS : 1)
         for (int k = 0; k < KK; ++k) {
+            if (k == p.kc) continue;
+            const int jp = k - (k > p.kc ? 1 : 0);  // point index in the record
             const int ky = k / K, kx = k - (k / K) * K;
             const int p0y = ho * p.stride - p.pad + ky * p.dilation;
             const int p0x = wo * p.stride - p.pad + kx * p.dilation;
-            const float rx = ElemTraits<T>::to_float(rec[k]);
-            const float ry = ElemTraits<T>::to_float(rec[KK + k]);
-            const float m = ElemTraits<T>::to_float(rec[2 * KK + k]);
+            const float rx = ElemTraits<T>::to_float(rec[jp]);
+            const float ry = ElemTraits<T>::to_float(rec[NP + jp]);
+            const float m = mask_value(ElemTraits<T>::to_float(rec[2 * NP + jp]), mn);
             const Sample s = locate(p0y, p0x, ry, rx, p.offset_scale, p.H, p.W);
             if (s.bits == 0u) continue;
 
@@ -283,6 +331,34 @@ fwd_vector_kernel(const T* __restrict__ x, const T* __restrict__ om, T* __restri
             }
         }
 
+        if (p.flags & kFlagCenterScale) {
+            // out = (1 - s) * aggregate + s * x at the centre grid position (zero outside)
+            const float sg = center_gate<T>(p, static_cast<size_t>(unit));
+            const int cy = ho * p.stride - p.pad + (K / 2) * p.dilation;
+            const int cx = wo * p.stride - p.pad + (K / 2) * p.dilation;
+            uint32_t cw[NW];
+#pragma unroll
+            for (int q = 0; q < NW; ++q) cw[q] = 0u;
+            if (cy >= 0 && cy < p.H && cx >= 0 && cx < p.W) {
+#pragma unroll
+                for (int jv = 0; jv < NV; ++jv) {
+                    uint32_t t[VB / 4];
+                    load_vec<VB>(ximg + (cy * p.W + cx) * p.C + c0 + jv * (VB / E), t);
+#pragma unroll
+                    for (int q = 0; q < VB / 4; ++q) cw[jv * (VB / 4) + q] = t[q];
+                }
+            }
+#pragma unroll
+            for (int q = 0; q < NW; ++q) {
+                if constexpr (E == 4) {
+                    acc[q] = fmaf(sg, __uint_as_float(cw[q]), (1.f - sg) * acc[q]);
+                } else {
+                    const float2 f = unpack2(cw[q], static_cast<T*>(nullptr));
+                    acc[2 * q] = fmaf(sg, f.x, (1.f - sg) * acc[2 * q]);
+                    acc[2 * q + 1] = fmaf(sg, f.y, (1.f - sg) * acc[2 * q + 1]);
+                }
+            }
+        }
         uint32_t ow[NW];
         if constexpr (E == 4) {
 #pragma unroll
@@ -311,7 +387,8 @@ fwd_scalar_kernel(const T* __restrict__ x, const T* __restrict__ om, T* __restri
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const int K = KS > 0 ? KS : p.K;
     const int KK = K * K;
-    const int R = 3 * KK;
+    const int NP = p.npts;
+    const int R = 3 * NP;
     const int unit0 = blockIdx.x * p.units_per_block;
     const int nunits = min(p.units_per_block, p.units - unit0);
     const T* rec_base = stage_run<T>(om + static_cast<size_t>(unit0) * R, nunits * R, smem_raw);
@@ -327,16 +404,19 @@ fwd_scalar_kernel(const T* __restrict__ x, const T* __restrict__ om, T* __restri
     const int rowC = p.W * p.C;
     const T* ximg = x + static_cast<size_t>(n) * p.H * rowC;
     T* o = out + (static_cast<size_t>((n * p.Hout + ho) * p.Wout + wo)) * p.C + g * p.Cg;
+    const MaskNorm mn = mask_norm(rec + 2 * NP, NP, p.flags);
 
     for (int c = part; c < p.Cg; c += p.lanes) {
         float acc = 0.f;
         for (int k = 0; k < KK; ++k) {
+            if (k == p.kc) continue;
+            const int jp = k - (k > p.kc ? 1 : 0);  // point index in the record
             const int ky = k / K, kx = k - (k / K) * K;
             const int p0y = ho * p.stride - p.pad + ky * p.dilation;
             const int p0x = wo * p.stride - p.pad + kx * p.dilation;
-            const float rx = ElemTraits<T>::to_float(rec[k]);
-            const float ry = ElemTraits<T>::to_float(rec[KK + k]);
-            const float m = ElemTraits<T>::to_float(rec[2 * KK + k]);
+            const float rx = ElemTraits<T>::to_float(rec[jp]);
+            const float ry = ElemTraits<T>::to_float(rec[NP + jp]);
+            const float m = mask_value(ElemTraits<T>::to_float(rec[2 * NP + jp]), mn);
             const Sample s = locate(p0y, p0x, ry, rx, p.offset_scale, p.H, p.W);
             if (s.bits == 0u) continue;
             const float wy0 = 1.f - s.ly, wx0 = 1.f - s.lx;
@@ -345,6 +425,14 @@ fwd_scalar_kernel(const T* __restrict__ x, const T* __restrict__ om, T* __restri
             if (s.bits & 2u) acc = fmaf(m * wy0 * s.lx, ElemTraits<T>::to_float(c00[p.C]), acc);
             if (s.bits & 4u) acc = fmaf(m * s.ly * wx0, ElemTraits<T>::to_float(c00[rowC]), acc);
             if (s.bits & 8u) acc = fmaf(m * s.ly * s.lx, ElemTraits<T>::to_float(c00[rowC + p.C]), acc);
+        }
+        if (p.flags & kFlagCenterScale) {
+            const float sg = center_gate<T>(p, static_cast<size_t>(unit));
+            const int cy = ho * p.stride - p.pad + (K / 2) * p.dilation;
+            const int cx = wo * p.stride - p.pad + (K / 2) * p.dilation;
+            const float xc = (cy >= 0 && cy < p.H && cx >= 0 && cx < p.W)
+                                 ? ElemTraits<T>::to_float(ximg[(cy * p.W + cx) * p.C + g * p.Cg + c]) : 0.f;
+            acc = fmaf(sg, xc, (1.f - sg) * acc);
         }
         if constexpr (sizeof(T) == 4) o[c] = acc;
         else if constexpr (std::is_same<T, __half>::value) o[c] = __float2half_rn(acc);

@@ -185,6 +185,27 @@ __device__ __forceinline__ void fma_chunk(float2* acc, float w, const uint4& v) 
     }
 }
 
+// acc = (1 - s) * acc + s * x over one 16-byte chunk (centre feature scaling)
+template <typename T>
+__device__ __forceinline__ void blend_chunk(float2* acc, float s, const uint4& v) {
+    const float r = 1.f - s;
+    const uint32_t vw[4] = {v.x, v.y, v.z, v.w};
+    if constexpr (sizeof(T) == 4) {
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+            acc[q].x = fmaf(s, __uint_as_float(vw[2 * q]), r * acc[q].x);
+            acc[q].y = fmaf(s, __uint_as_float(vw[2 * q + 1]), r * acc[q].y);
+        }
+    } else {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float2 f = unpack2(vw[q], static_cast<T*>(nullptr));
+            acc[q].x = fmaf(s, f.x, r * acc[q].x);
+            acc[q].y = fmaf(s, f.y, r * acc[q].y);
+        }
+    }
+}
+
 template <typename T>
 __device__ __forceinline__ uint4 pack_chunk(const float2* a) {
     uint4 v;
@@ -234,8 +255,8 @@ __device__ __forceinline__ const unsigned char* run_src(const TileParams& p, con
     const int px = row_runs ? 0 : r - py * c.nw;
     const size_t first_unit = (static_cast<size_t>((c.n * f.Hout + c.ho0 + py) * f.Wout + c.wo0 + px)) * f.G +
                               static_cast<size_t>(c.gsub) * p.GS;
-    *count = (row_runs ? c.nw * f.G : p.GS) * 3 * f.KK;
-    return reinterpret_cast<const unsigned char*>(om + first_unit * 3 * f.KK);
+    *count = (row_runs ? c.nw * f.G : p.GS) * 3 * f.npts;
+    return reinterpret_cast<const unsigned char*>(om + first_unit * 3 * f.npts);
 }
 
 __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
@@ -344,7 +365,9 @@ __device__ __forceinline__ void fma_chunk_h(float2* acc, uint32_t w2, const uint
 // producer after letting its copies in flight land).
 //
 // PBC: the window's pixel stride as a compile-time constant (0: p.PB).
-template <typename T, int Q, int KS, bool HW, int PBC>
+// VF: the variant flags of p.f may be set (softmax over the masks, centre
+// point removed, centre feature scaling); false compiles them out.
+template <typename T, int Q, int KS, bool HW, int PBC, bool VF>
 __global__ void __launch_bounds__(544, 1)
 fwd_tile_kernel(const __grid_constant__ CUtensorMap xmap, const T* __restrict__ x, const T* __restrict__ om,
                 T* __restrict__ out, TileParams p) {
@@ -355,7 +378,9 @@ fwd_tile_kernel(const __grid_constant__ CUtensorMap xmap, const T* __restrict__ 
     const FwdParams& f = p.f;
     const int K = KS > 0 ? KS : f.K;
     const int KK = K * K;
-    const int R3 = 3 * KK;
+    const int NP = VF ? f.npts : KK;   // points per unit
+    const int kcs = VF ? f.kc : KK;    // grid index left out (none: KK)
+    const int R3 = 3 * NP;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int nc = static_cast<int>(blockDim.x >> 5) - 1;  // consumer warps
     const bool row_runs = p.GS == f.G;
@@ -472,14 +497,17 @@ fwd_tile_kernel(const __grid_constant__ CUtensorMap xmap, const T* __restrict__ 
             const int by = ho * f.stride - f.pad;  // grid row of ky = 0 (image coordinates)
             const int bx = wo * f.stride - f.pad;
             const float fwy = static_cast<float>(by - c.wy0), fwx = static_cast<float>(bx - c.wx0);
-            unsigned long long slow = 0ull;  // points left for the global-memory pass (K*K <= 64)
+            unsigned long long slow = 0ull;  // grid points left for the global-memory pass (K*K <= 64)
+            const MaskNorm mn = VF ? mask_norm(rec + 2 * NP, NP, f.flags) : MaskNorm{0.f, 1.f, false};
 
 #pragma unroll (KS > 0 ? KS * KS : 1)
             for (int k = 0; k < KK; ++k) {
+                if (k == kcs) continue;
+                const int jp = k - (k > kcs ? 1 : 0);  // point index in the record
                 const int ky = k / K, kx = k - (k / K) * K;
-                const float rx = ElemTraits<T>::to_float(rec[k]);
-                const float ry = ElemTraits<T>::to_float(rec[KK + k]);
-                const float m = ElemTraits<T>::to_float(rec[2 * KK + k]);
+                const float rx = ElemTraits<T>::to_float(rec[jp]);
+                const float ry = ElemTraits<T>::to_float(rec[NP + jp]);
+                const float m = mask_value(ElemTraits<T>::to_float(rec[2 * NP + jp]), mn);
                 const float dy = __fmul_rn(f.offset_scale, ry);
                 const float dx = __fmul_rn(f.offset_scale, rx);
                 const float fy0 = floorf(dy), fx0 = floorf(dx);
@@ -542,10 +570,11 @@ fwd_tile_kernel(const __grid_constant__ CUtensorMap xmap, const T* __restrict__ 
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
                         const int k = kk[h] < 0 ? kk[0] : kk[h];
+                        const int jp = k - (k > kcs ? 1 : 0);
                         const int ky = k / K, kx = k - (k / K) * K;
-                        const float rx = ElemTraits<T>::to_float(rec[k]);
-                        const float ry = ElemTraits<T>::to_float(rec[KK + k]);
-                        const float m = ElemTraits<T>::to_float(rec[2 * KK + k]);
+                        const float rx = ElemTraits<T>::to_float(rec[jp]);
+                        const float ry = ElemTraits<T>::to_float(rec[NP + jp]);
+                        const float m = mask_value(ElemTraits<T>::to_float(rec[2 * NP + jp]), mn);
                         Sample s = locate(by + ky * f.dilation, bx + kx * f.dilation, ry, rx, f.offset_scale, f.H, f.W);
                         if (kk[h] < 0) s.bits = 0u;
                         // the same weight arithmetic as the window path
@@ -581,10 +610,11 @@ fwd_tile_kernel(const __grid_constant__ CUtensorMap xmap, const T* __restrict__ 
                 while (slow) {
                     const int k = __ffsll(static_cast<long long>(slow)) - 1;
                     slow &= slow - 1ull;
+                    const int jp = k - (k > kcs ? 1 : 0);
                     const int ky = k / K, kx = k - (k / K) * K;
-                    const float rx = ElemTraits<T>::to_float(rec[k]);
-                    const float ry = ElemTraits<T>::to_float(rec[KK + k]);
-                    const float m = ElemTraits<T>::to_float(rec[2 * KK + k]);
+                    const float rx = ElemTraits<T>::to_float(rec[jp]);
+                    const float ry = ElemTraits<T>::to_float(rec[NP + jp]);
+                    const float m = mask_value(ElemTraits<T>::to_float(rec[2 * NP + jp]), mn);
                     const Sample s = locate(by + ky * f.dilation, bx + kx * f.dilation, ry, rx, f.offset_scale, f.H, f.W);
                     if (s.bits == 0u) continue;
                     // the same weight arithmetic as the window path
@@ -610,6 +640,15 @@ fwd_tile_kernel(const __grid_constant__ CUtensorMap xmap, const T* __restrict__ 
                 }
             }
 
+            if (VF && (f.flags & kFlagCenterScale)) {
+                // out = (1 - s) * aggregate + s * x at the centre grid position, read from the
+                // window (which holds zeros outside the image)
+                const float sg = center_gate<T>(f, (static_cast<size_t>((c.n * f.Hout + ho) * f.Wout + wo)) * f.G + g);
+                const int cyw = by + (K / 2) * f.dilation - c.wy0, cxw = bx + (K / 2) * f.dilation - c.wx0;
+                const unsigned char* pcx = ubase + (cyw * p.WW + cxw) * PB;
+#pragma unroll
+                for (int j = 0; j < Q; ++j) blend_chunk<T>(acc[j], sg, *reinterpret_cast<const uint4*>(pcx + (choff[j] << 4)));
+            }
             T* o = out + (static_cast<size_t>((c.n * f.Hout + ho) * f.Wout + wo)) * f.C + g * f.Cg;
 #pragma unroll
             for (int j = 0; j < Q; ++j) {

@@ -114,13 +114,17 @@ def _draw(gen: torch.Generator, shape, dist) -> torch.Tensor:
 
 def make_inputs(N: int, H: int, W: int, C: int, G: int, K: int, Hout: int, Wout: int,
                 dtype: str = "f32", offsets=("normal", 0.0, 1.0), masks=("normal", 0.0, 1.0),
-                x_dist=("normal", 0.0, 1.0), seed: int = 0):
-    """Return (x [N,H,W,C], offset_mask [N,Hout,Wout,G,3*K*K]) as CPU tensors in ``dtype``."""
+                x_dist=("normal", 0.0, 1.0), seed: int = 0, points: int | None = None):
+    """Return (x [N,H,W,C], offset_mask [N,Hout,Wout,G,3*P]) as CPU tensors in ``dtype``.
+
+    P = ``points`` (default K*K; K*K - 1 for the variant without the centre point).
+    """
+    P = K * K if points is None else int(points)
     gen = torch.Generator(device="cpu")
     gen.manual_seed(int(seed))
     x = _draw(gen, (N, H, W, C), x_dist)
-    off = _draw(gen, (N, Hout, Wout, G, 2 * K * K), offsets)
-    msk = _draw(gen, (N, Hout, Wout, G, K * K), masks)
+    off = _draw(gen, (N, Hout, Wout, G, 2 * P), offsets)
+    msk = _draw(gen, (N, Hout, Wout, G, P), masks)
     om = torch.cat([off, msk], dim=-1)
     t = DTYPES[dtype]
     return x.to(t).contiguous(), om.to(t).contiguous()
@@ -147,3 +151,11 @@ def make_grad_out(N: int, Hout: int, Wout: int, C: int, dtype: str = "f32", seed
 def workload_grad_out(w: Workload) -> torch.Tensor:
     """Seeded dL/dout of a named workload (CPU tensor in its storage dtype)."""
     return make_grad_out(w.N, w.Hout, w.Wout, w.C, w.dtype, seed=w.seed)
+
+
+def make_center_logit(N: int, Hout: int, Wout: int, G: int, dtype: str = "f32", seed: int = 0,
+                      dist=("normal", 0.0, 1.5)) -> torch.Tensor:
+    """Seeded gate logits [N,Hout,Wout,G] for centre feature scaling (own generator, seed 2000 + seed)."""
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(2000 + int(seed))
+    return _draw(gen, (N, Hout, Wout, G), dist).to(DTYPES[dtype]).contiguous()

@@ -91,9 +91,31 @@ typedef enum {
     DCNV4_ERR_TOO_LARGE = 8, /* an element count reaches 2^31                           */
     DCNV4_ERR_LAUNCH = 9,    /* the kernel launch failed (CUDA error after launch)      */
     DCNV4_ERR_CUDA = 10,     /* a CUDA runtime call other than a launch failed          */
-    DCNV4_ERR_STAGING = 11   /* dcnv4_forward_host_noalloc: one image does not fit its  */
+    DCNV4_ERR_STAGING = 11,  /* dcnv4_forward_host_noalloc: one image does not fit its  */
                              /* half of the library's static staging area               */
+    DCNV4_ERR_FLAGS = 12     /* dcnv4_forward_ex: a flag bit that is not defined        */
 } dcnv4_status_t;
+
+/* Variant switches of dcnv4_forward_ex / dcnv4_validate_ex (bitwise or).
+ * Sources: "掌握DCNv4技术" (pwwt.cn), section on advanced tuning and extension
+ * (DCNv4 also offers centre feature scaling, a sigmoid that weighs the centre
+ * feature, and removal of the centre point); "不只是卷积的平替" (jsqmd.com),
+ * section 1 (DCNv3 normalised the aggregation weights with a softmax, which
+ * DCNv4 removed). The pages give no formulas; the readings are:
+ *   DCNV4_FLAG_SOFTMAX: per (n, ho, wo, g) the masks are replaced by
+ *     m'_j = exp(m_j - max) / sum_i exp(m_i - max) over the unit's points
+ *     (fp32, expf), then aggregated as usual;
+ *   DCNV4_FLAG_REMOVE_CENTER: K odd and >= 3; each unit has P = K*K - 1
+ *     points, offset_mask is [N,Hout,Wout,G,3*P] with per group P x-offsets,
+ *     P y-offsets, P masks, and point j sits on grid index j before the
+ *     centre (K*K-1)/2 and j + 1 after it;
+ *   DCNV4_FLAG_CENTER_SCALE: with s = 1/(1 + exp(-center_logit[n,ho,wo,g])),
+ *     out = (1 - s) * aggregate + s * x_c, x_c being x at the centre grid
+ *     position (ho*stride - pad + (K/2)*dilation, wo*stride - pad +
+ *     (K/2)*dilation), channels of group g, zero outside the image. */
+#define DCNV4_FLAG_SOFTMAX 1u
+#define DCNV4_FLAG_REMOVE_CENTER 2u
+#define DCNV4_FLAG_CENTER_SCALE 4u
 
 #define DCNV4_MAX_K 16
 #define DCNV4_MAX_EXTENT (1 << 22)
@@ -124,6 +146,27 @@ DCNV4_API int dcnv4_forward(const void *x, const void *offset_mask, void *out,
                   int N, int H, int W, int C, int G, int K,
                   int stride, int pad, int dilation, float offset_scale, int dtype,
                   void *stream);
+
+/* dcnv4_validate with the variant flags above: additionally DCNV4_ERR_FLAGS
+ * for an unknown bit, DCNV4_ERR_SHAPE for DCNV4_FLAG_REMOVE_CENTER with an
+ * even K or K < 3, and, with DCNV4_FLAG_CENTER_SCALE, center_logit (type
+ * dtype, [N,Hout,Wout,G]) non-NULL, aligned and not overlapping out.
+ * center_logit is ignored (may be NULL) without DCNV4_FLAG_CENTER_SCALE.
+ * offset_mask's size follows the flags (3*(K*K-1) per group without the
+ * centre). Host only. */
+DCNV4_API int dcnv4_validate_ex(const void *x, const void *offset_mask, const void *center_logit,
+                      const void *out, int N, int H, int W, int C, int G, int K,
+                      int stride, int pad, int dilation, float offset_scale, int dtype,
+                      unsigned int flags);
+
+/* dcnv4_forward with the variant flags above (flags == 0 is dcnv4_forward).
+ * center_logit: device, read only, [N,Hout,Wout,G] of type dtype, used only
+ * with DCNV4_FLAG_CENTER_SCALE. Same launch, ownership and error behaviour
+ * as dcnv4_forward, after dcnv4_validate_ex. */
+DCNV4_API int dcnv4_forward_ex(const void *x, const void *offset_mask, const void *center_logit, void *out,
+                     int N, int H, int W, int C, int G, int K,
+                     int stride, int pad, int dilation, float offset_scale, int dtype,
+                     unsigned int flags, void *stream);
 
 /* The backward of dcnv4_forward, for training with the operator ("不只是卷积的
  * 平替：我把DCNv4塞进Stable Diffusion的U-Net里", jsqmd.com: section 1 defines the

@@ -165,3 +165,38 @@ def test_backward_binding_refuses_cpu_tensors():
     om = torch.zeros(1, 8, 8, 2, 27)
     with pytest.raises(ValueError, match="CUDA"):
         B.backward(x, om, torch.zeros(1, 8, 8, 16), G=2, K=3, pad=1)
+
+
+def _vex(x=X, om=OM, z=0x60000000, out=OUT, flags=0, **kw):
+    a = dict(GOOD)
+    a.update(kw)
+    return B.load_library().dcnv4_validate_ex(x, om, z, out, a["N"], a["H"], a["W"], a["C"], a["G"], a["K"],
+                                              a["stride"], a["pad"], a["dilation"], a["offset_scale"], a["dtype"],
+                                              flags)
+
+
+def test_validate_ex_checks_the_variant_flags():
+    assert _vex(flags=0) == B.DCNV4_OK
+    assert _vex(flags=B.FLAG_SOFTMAX | B.FLAG_REMOVE_CENTER | B.FLAG_CENTER_SCALE) == B.DCNV4_OK
+    assert _vex(flags=8) == B.STATUS["DCNV4_ERR_FLAGS"]
+    assert _vex(flags=0x80000000) == B.STATUS["DCNV4_ERR_FLAGS"]
+    # no centre to remove for an even kernel or K = 1
+    assert _vex(flags=B.FLAG_REMOVE_CENTER, K=2, pad=0) == B.STATUS["DCNV4_ERR_SHAPE"]
+    assert _vex(flags=B.FLAG_REMOVE_CENTER, K=1, pad=0) == B.STATUS["DCNV4_ERR_SHAPE"]
+    # the gate logits are needed, aligned and disjoint from out only with centre scaling
+    assert _vex(z=0, flags=B.FLAG_CENTER_SCALE) == B.STATUS["DCNV4_ERR_NULL"]
+    assert _vex(z=0, flags=B.FLAG_SOFTMAX) == B.DCNV4_OK
+    assert _vex(z=0x60000001, flags=B.FLAG_CENTER_SCALE) == B.STATUS["DCNV4_ERR_ALIGN"]
+    assert _vex(z=OUT + 64, flags=B.FLAG_CENTER_SCALE) == B.STATUS["DCNV4_ERR_ALIAS"]
+    assert _vex(z=OUT + 64, flags=B.FLAG_SOFTMAX) == B.DCNV4_OK
+
+
+def test_forward_ex_returns_flag_errors_before_any_cuda_call():
+    lib = B.load_library()
+    a = dict(GOOD)
+    rc = lib.dcnv4_forward_ex(X, OM, 0, OUT, a["N"], a["H"], a["W"], 16, 2, 3, 1, 1, 1, 1.0, a["dtype"], 16, None)
+    assert rc == B.STATUS["DCNV4_ERR_FLAGS"]
+    rc = lib.dcnv4_forward_ex(X, OM, 0, OUT, a["N"], a["H"], a["W"], 16, 2, 4, 1, 1, 1, 1.0, a["dtype"],
+                              B.FLAG_REMOVE_CENTER, None)
+    assert rc == B.STATUS["DCNV4_ERR_SHAPE"]
+    assert lib.dcnv4_forward_ex(0, 0, 0, 0, 0, 8, 8, 16, 2, 3, 1, 1, 1, 1.0, a["dtype"], 7, None) == B.DCNV4_OK
