@@ -59,6 +59,8 @@ def _load():
         lib.oracle_dcnv4_backward.restype = i
         lib.oracle_dcnv4_forward_variants.argtypes = [p] * 4 + [i] * 9 + [f, i, i, i]
         lib.oracle_dcnv4_forward_variants.restype = i
+        lib.oracle_dcnv4_predictor.argtypes = [p] * 4 + [i] * 4
+        lib.oracle_dcnv4_predictor.restype = i
         _lib = lib
     return _lib
 
@@ -137,6 +139,30 @@ def dcnv4_forward_variants(x, offset_mask, G: int, K: int, stride: int = 1, pad:
     if rc != 0:
         raise ValueError("oracle rejected the arguments")
     return out
+
+
+def dcnv4_predictor(y, weight, bias, G: int, P: int) -> np.ndarray:
+    """fp64 1x1 projection + repacking into offset_mask records.
+
+    y: [..., C] (any leading pixel shape), weight: [3*G*P, C] in the pages'
+    channel order (all groups' offsets, (g, comp, point), then all groups'
+    masks, (g, point)), bias: [3*G*P] or None. Returns [..., G, 3*P].
+    """
+    y = _f64(y)
+    w = _f64(weight)
+    lead, C = y.shape[:-1], y.shape[-1]
+    M = int(np.prod(lead)) if lead else 1
+    if w.shape != (3 * G * P, C):
+        raise ValueError(f"weight shape {w.shape} != {(3 * G * P, C)}")
+    b = None if bias is None else _f64(bias)
+    if b is not None and b.shape != (3 * G * P,):
+        raise ValueError("bias must be [3*G*P]")
+    rec = np.zeros((M, G, 3 * P), dtype=np.float64)
+    if M:
+        rc = _load().oracle_dcnv4_predictor(_ptr(y), _ptr(w), None if b is None else _ptr(b), _ptr(rec), M, C, G, P)
+        if rc != 0:
+            raise ValueError("oracle rejected the arguments")
+    return rec.reshape(*lead, G, 3 * P)
 
 
 def sampling_index(offset_mask, H: int, W: int, G: int, K: int, stride: int = 1, pad: int = 0,

@@ -287,6 +287,44 @@ int oracle_dcnv4_forward_variants(const double *x, const double *om, const doubl
 }
 
 /* ------------------------------------------------------------------------
+ * The offset/mask predictor's last step. "不只是卷积的平替" (jsqmd.com),
+ * section 2, U-Net block listing: a depthwise 3x3 convolution followed by a
+ * 1x1 convolution to 3*groups*9 channels predicts the parameters; the first
+ * 2*groups*9 channels are the offsets and the rest the masks, and section 1's
+ * listing reads them as offset.reshape(N, G, 2, K*K, ...) and
+ * mask.reshape(N, G, K*K, ...). This function is that 1x1 convolution on
+ * channels-last input followed by the repacking into this library's
+ * offset_mask record:
+ *   params[m, o] = bias[o] + sum_c W[o, c] * y[m, c]      (o < 3*G*P)
+ *   o = g*2P + comp*P + j  (o < 2GP)  ->  record[m, g, comp*P + j]
+ *   o = 2GP + g*P + j                 ->  record[m, g, 2P + j]
+ * y: [M, C] (M pixels), W: [3GP, C], bias: [3GP] (NULL: none),
+ * record: [M, G, 3P]. P = points per group (K*K, or K*K - 1 without the
+ * centre).
+ * ------------------------------------------------------------------------ */
+int oracle_dcnv4_predictor(const double *y, const double *w, const double *bias, double *record,
+                           int M, int C, int G, int P)
+{
+    if (M < 0 || C <= 0 || G <= 0 || P <= 0) return -1;
+    const int NO = 3 * G * P;
+    for (int m = 0; m < M; ++m)
+        for (int o = 0; o < NO; ++o) {
+            double acc = bias ? bias[o] : 0.0;
+            for (int c = 0; c < C; ++c) acc += w[(size_t)o * C + c] * y[(size_t)m * C + c];
+            int g, slot;
+            if (o < 2 * G * P) {
+                g = o / (2 * P);
+                slot = o % (2 * P);          /* comp * P + j */
+            } else {
+                g = (o - 2 * G * P) / P;
+                slot = 2 * P + (o - 2 * G * P) % P;
+            }
+            record[((size_t)m * G + g) * (size_t)(3 * P) + slot] = acc;
+        }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------
  * Backward of the forward above (the training direction; the pages use the
  * operator for training, e.g. the Stable Diffusion fine-tuning of the
  * jsqmd.com page, section 4). For a loss L with dL/dout = grad_out:
