@@ -19,8 +19,10 @@ exceeds the L2 cache, so no step starts with its inputs in L2.
 repository: there is no other implementation to install) on the host cores.
 
 Secondary lines (not the headline): --pass backward times dcnv4_backward on
-the same workload; --variant softmax|remove_center|center_scale|all times
-dcnv4_forward_ex with those variant flags.
+the same workload; --pass predictor times dcnv4_predictor (the tcgen05
+projection that produces the workload's offset_mask records); --variant
+softmax|remove_center|center_scale|all times dcnv4_forward_ex with those
+variant flags.
 """
 from __future__ import annotations
 
@@ -41,6 +43,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "DCNv4 fwd sampling points/s (G/s); achieved HBM GB/s as % of B200 peak"
 METRIC_BWD = "DCNv4 bwd sampling points/s (G/s); achieved HBM GB/s as % of B200 peak"
+METRIC_PRED = "DCNv4 offset/mask predictor records/s (G pixel-group records/s); achieved HBM GB/s as % of B200 peak"
 UNIT = "Gpoints/s"
 FALLBACK_HBM_GBS = 6650.0
 
@@ -55,8 +58,9 @@ def parse_args():
     ap.add_argument("--soak-s", type=float, default=1.0)
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--pass", dest="which", choices=["forward", "backward"], default="forward",
-                    help="forward (the headline) or the backward of the same workload")
+    ap.add_argument("--pass", dest="which", choices=["forward", "backward", "predictor"], default="forward",
+                    help="forward (the headline), the backward of the same workload, or the offset/mask "
+                         "predictor's projection that produces its records")
     ap.add_argument("--variant", choices=["none", "softmax", "remove_center", "center_scale", "all"],
                     default="none", help="forward variant flags (DCNv3 softmax, centre point removed, "
                                          "centre feature scaling, or all three)")
@@ -478,6 +482,117 @@ def run_variant(args, w, dev, world, rank, barrier, max_over_ranks):
         print(json.dumps(line), flush=True)
 
 
+def run_predictor(args, w, dev, world, rank, barrier, max_over_ranks):
+    """The offset/mask predictor's 1x1 projection + packing (dcnv4_predictor) for the workload's records:
+    y [N*Hout*Wout, C] -> offset_mask [N*Hout*Wout, G, 3*K*K], fp16/bf16 on the tensor cores."""
+    import torch
+    import deformable_convolution_sparse_b200 as dcn
+
+    M, P = w.N * w.Hout * w.Wout, w.K * w.K
+    NO = 3 * w.G * P
+    gen = torch.Generator().manual_seed(w.seed + 1000 * rank)
+    td = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}[w.dtype]
+    y = torch.randn(M, w.C, generator=gen).to(td)
+    wt = (torch.randn(NO, w.C, generator=gen) * w.C ** -0.5).to(td)
+    b = torch.randn(NO, generator=gen)
+    lib = dcn.load_library()
+    dtype_code = dcn.binding.TORCH_DTYPE[td]
+    e = y.element_size()
+    foot = (y.numel() + wt.numel() + M * NO) * e + b.numel() * 4
+    flops = 2.0 * M * NO * w.C
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    copies = max(3, math.ceil(3 * l2 / foot))
+    sets = [(y.to(dev), torch.empty(M, w.G, 3 * P, dtype=td, device=dev)) for _ in range(copies)]
+    wd, bd = wt.to(dev), b.to(dev)
+    stream = torch.cuda.current_stream(dev)
+    sh = stream.cuda_stream
+    launches = [0]
+
+    def call(yd, od):
+        rc = lib.dcnv4_predictor(yd.data_ptr(), wd.data_ptr(), bd.data_ptr(), od.data_ptr(), M, w.C, w.G, w.K, 0,
+                                 dtype_code, sh)
+        if rc != 0:
+            raise dcn.DCNv4Error(rc, "dcnv4_predictor")
+
+    def step(i):
+        call(*sets[i % copies])
+        launches[0] += 1
+
+    ms, sampler, timed_launches = time_steps(step, launches, args, dev, stream, barrier, max_over_ranks)
+    ms_step = ms / args.steps
+    units = M * w.G
+    value = units * world * args.steps / (ms / 1e3) / 1e9
+    peak, peak_kind = measured_peaks()
+    achieved = foot / (ms_step / 1e3) / 1e9
+
+    yh = y.pin_memory()
+    oh = torch.empty(M, w.G, 3 * P, dtype=td).pin_memory()
+    yd0, od0 = sets[0]
+
+    def e2e_step():
+        yd0.copy_(yh, non_blocking=True)
+        call(yd0, od0)
+        oh.copy_(od0, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1))
+    if not torch.equal(oh, od0.cpu()):
+        raise SystemExit("end-to-end records differ from the device-resident ones")
+
+    base = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        n_s = min(M, 8 * w.Hout * w.Wout)
+        ys, ws, bs = y[:n_s].double().numpy(), wt.double().numpy(), b.double().numpy()
+        oracle.dcnv4_predictor(ys[:16], ws, bs, G=w.G, P=P)
+        t0 = time.perf_counter()
+        oracle.dcnv4_predictor(ys, ws, bs, G=w.G, P=P)
+        dt = time.perf_counter() - t0
+        base = {"value": n_s * w.G / dt / 1e9, "unit": "Grecords/s", "cores": 1, "kind": "oracle", "seconds": dt,
+                "sample": f"{n_s} of {M} pixels (8 images), fp64 C oracle predictor, one thread"}
+    if rank == 0:
+        line = {
+            "metric": METRIC_PRED, "value": value, "unit": "Grecords/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": w.dtype, "data": "synthetic", "pass": "predictor",
+            "config": {
+                "workload": f"{w.name} predictor: y [{M}, {w.C}] x W [{NO}, {w.C}] + bias -> offset_mask "
+                            f"[{M}, {w.G}, {3 * P}] (the records of the {w.name} aggregation)",
+                "storage_dtype": w.dtype, "accumulate": "f32 (tensor memory)", "global_batch": w.N * world,
+                "parallelism": f"dp{world} (independent batches)",
+                "l2": f"steps rotate over {copies} resident sets, {copies * foot / 1e6:.0f} MB in total vs "
+                      f"{l2 / 1e6:.0f} MB L2",
+                "inputs": "seeded synthetic: y~N(0,1), W~N(0,1/C), bias~N(0,1)",
+                "tensor_tflops": flops / (ms_step / 1e3) / 1e12,
+            },
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak,
+                         "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json)"
+                         if peak_kind == "measured" else "fallback 6.65 TB/s",
+                         "kernel": "dcnv4 predictor (tcgen05 GEMM + packing epilogue, one launch per step)",
+                         "algorithmic_bytes_per_launch": foot, "flops_per_launch": flops, "traffic": None},
+            "e2e": {"value": units * world * args.e2e_steps / (e2e_ms / 1e3) / 1e9, "unit": "Grecords/s",
+                    "ms_per_step": e2e_ms / args.e2e_steps, "steps": args.e2e_steps,
+                    "h2d_bytes_per_step": y.numel() * e, "d2h_bytes_per_step": M * NO * e,
+                    "path": "pinned y copied in, dcnv4_predictor, records copied out, one stream"},
+            "gpu_launches": timed_launches,
+            "clocks": sampler.summary(),
+            "cpu_baseline": base,
+        }
+        print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
@@ -512,9 +627,11 @@ def main():
         return float(t.item())
 
     w = WORKLOADS[args.workload or BENCH_WORKLOAD]
-    if args.which == "backward" or args.variant != "none":
+    if args.which != "forward" or args.variant != "none":
         if args.which == "backward":
             run_backward(args, w, dev, world, rank, barrier, max_over_ranks)
+        elif args.which == "predictor":
+            run_predictor(args, w, dev, world, rank, barrier, max_over_ranks)
         else:
             run_variant(args, w, dev, world, rank, barrier, max_over_ranks)
         if world > 1:

@@ -31,7 +31,7 @@ TORCH_DTYPE = {torch.float32: DCNV4_F32, torch.float16: DCNV4_F16, torch.bfloat1
 
 # every symbol include/dcnv4.h declares
 EXPORTS = ("dcnv4_output_shape", "dcnv4_validate", "dcnv4_validate_ex", "dcnv4_forward", "dcnv4_forward_ex",
-           "dcnv4_backward", "dcnv4_sampling_index",
+           "dcnv4_backward", "dcnv4_predictor", "dcnv4_sampling_index",
            "dcnv4_forward_host", "dcnv4_forward_host_noalloc", "dcnv4_device_status", "dcnv4_selftest_wait_timeout", "dcnv4_strerror",
            "dcnv4_abi_version")
 DEVSTATUS_COPY_TIMEOUT, DEVSTATUS_SELFTEST_TIMEOUT = 1, 2
@@ -67,6 +67,8 @@ def load_library():
     lib.dcnv4_validate_ex.restype = i
     lib.dcnv4_forward_ex.argtypes = [p] * 4 + [i] * 9 + [f, i, ctypes.c_uint, p]
     lib.dcnv4_forward_ex.restype = i
+    lib.dcnv4_predictor.argtypes = [p] * 4 + [i] * 4 + [ctypes.c_uint, i, p]
+    lib.dcnv4_predictor.restype = i
     lib.dcnv4_backward.argtypes = [p] * 5 + [i] * 9 + [f, i, p]
     lib.dcnv4_backward.restype = i
     lib.dcnv4_sampling_index.argtypes = [p, p, p] + [i] * 8 + [f, i, p]
@@ -241,6 +243,47 @@ def backward(x: torch.Tensor, offset_mask: torch.Tensor, grad_out: torch.Tensor,
     if rc != DCNV4_OK:
         raise DCNv4Error(rc, "dcnv4_backward")
     return gx, gom
+
+
+def predictor(y: torch.Tensor, weight: torch.Tensor, bias: torch.Tensor | None, G: int, K: int,
+              remove_center: bool = False, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Offset/mask predictor step through ``dcnv4_predictor``: 1x1 projection + packing.
+
+    y: [..., C] channels-last (leading dims are the pixels); weight: [3*G*P, C]
+    in the pages' channel order (all groups' offsets, then all groups'
+    masks); bias: fp32 [3*G*P] or None. Returns offset_mask [..., G, 3*P] in
+    y's dtype (P = K*K, or K*K-1 with ``remove_center``).
+    """
+    _check_tensor(y, "y")
+    _check_tensor(weight, "weight")
+    P = K * K - (1 if remove_center else 0)
+    C = y.shape[-1]
+    if weight.dtype != y.dtype or weight.device != y.device or tuple(weight.shape) != (3 * G * P, C):
+        raise ValueError(f"weight must be [{3 * G * P}, {C}] in y's dtype and device")
+    bp = 0
+    if bias is not None:
+        _check_tensor(bias, "bias")
+        if bias.dtype != torch.float32 or tuple(bias.shape) != (3 * G * P,) or bias.device != y.device:
+            raise ValueError(f"bias must be fp32 [{3 * G * P}] on y's device")
+        bp = bias.data_ptr()
+    lead = tuple(y.shape[:-1])
+    M = 1
+    for d in lead:
+        M *= d
+    shape = lead + (G, 3 * P)
+    if out is None:
+        out = torch.empty(shape, dtype=y.dtype, device=y.device)
+    else:
+        _check_tensor(out, "out")
+        if tuple(out.shape) != shape or out.dtype != y.dtype or out.device != y.device:
+            raise ValueError("out has the wrong shape, dtype or device")
+    with torch.cuda.device(y.device):
+        rc = load_library().dcnv4_predictor(y.data_ptr(), weight.data_ptr(), bp, out.data_ptr(), M, C, G, K,
+                                            FLAG_REMOVE_CENTER if remove_center else 0, TORCH_DTYPE[y.dtype],
+                                            _stream_handle(stream))
+    if rc != DCNV4_OK:
+        raise DCNv4Error(rc, "dcnv4_predictor")
+    return out
 
 
 def forward_host(x: torch.Tensor, offset_mask: torch.Tensor, G: int, K: int, stride: int = 1, pad: int = 0,

@@ -18,6 +18,7 @@
 #include "dcnv4_kernels.cuh"
 #include "dcnv4_window.cuh"
 #include "dcnv4_backward.cuh"
+#include "dcnv4_predictor.cuh"
 
 namespace {
 
@@ -428,6 +429,103 @@ int launch_backward(const void* x, const void* om, const void* go, float* gx, fl
     return k3 ? run(dcnv4::bwd_kernel<T, 1, 3>) : run(dcnv4::bwd_kernel<T, 1, 0>);
 }
 
+// Offset/mask predictor: the tensor-core kernel for fp16/bf16 with C a multiple
+// of 64 and at most 256 output channels (DCNV4_PRED_VARIANT=plain forces the
+// CUDA-core kernel), the CUDA-core kernel otherwise.
+template <typename T>
+int launch_predictor(const void* y, const void* w, const float* bias, void* rec, dcnv4::PredParams p,
+                     cudaStream_t stream) {
+    constexpr int E = sizeof(T);
+    const char* pv = std::getenv("DCNV4_PRED_VARIANT");
+    const bool force_plain = pv && std::strcmp(pv, "plain") == 0;
+    bool tc = !force_plain && E == 2 && p.C % 64 == 0 && p.NO <= 256 && aligned(y, 16) && aligned(w, 16) &&
+              aligned(rec, 16) && p.M > 0;
+    if constexpr (E == 2) {
+        if (tc) {
+            p.NP = (p.NO + 15) / 16 * 16;
+            p.kblocks = p.C / 64;
+            p.tiles = (p.M + 127) / 128;
+            unsigned cols = 32;
+            while (cols < 2u * static_cast<unsigned>(p.NP)) cols <<= 1;
+            p.tmem_cols = cols;
+            p.a_fmt = std::is_same<T, __half>::value ? 0 : 1;
+            const size_t b_bytes = static_cast<size_t>(p.kblocks) * p.NP * 128;
+            const size_t a_stage = static_cast<size_t>(p.kblocks) * 128 * 128;
+            const size_t meta = static_cast<size_t>(p.NO) * 8 + 8 + 8 * 16 + 16;
+            // two output staging buffers (store of tile i overlaps the epilogue of tile i+1) when they fit
+            size_t o_bytes = 0, fixed = 0;
+            int stages = 0;
+            for (int ob = 2; ob >= 1 && stages < 2; --ob) {
+                o_bytes = (static_cast<size_t>(ob) * 128 * p.NO * E + 15) / 16 * 16;
+                fixed = 1024 + b_bytes + o_bytes + meta;
+                stages = 4;
+                while (stages >= 2 && fixed + stages * a_stage > kTileSmemLimit) --stages;
+                p.out_bufs = ob;
+            }
+            tc = stages >= 2;
+            if (tc) {
+                p.stages = stages;
+                p.smem_b = 0;
+                p.smem_a = static_cast<unsigned>(b_bytes);
+                p.smem_o = static_cast<unsigned>(b_bytes + stages * a_stage);
+                p.smem_meta = static_cast<unsigned>(p.smem_o + o_bytes);
+                const size_t smem = fixed + stages * a_stage;
+                auto encode = tensor_map_encoder();
+                CUtensorMap amap, bmap;
+                const cuuint32_t estr[2] = {1u, 1u};
+                const cuuint64_t adims[2] = {static_cast<cuuint64_t>(p.C), static_cast<cuuint64_t>(p.M)};
+                const cuuint64_t astr[1] = {static_cast<cuuint64_t>(p.C) * E};
+                const cuuint32_t abox[2] = {64u, 128u};
+                const cuuint64_t bdims[2] = {static_cast<cuuint64_t>(p.C), static_cast<cuuint64_t>(p.NO)};
+                const cuuint32_t bbox[2] = {64u, static_cast<cuuint32_t>(p.NP)};
+                tc = encode &&
+                     encode(&amap, tma_dtype<T>(), 2, const_cast<void*>(y), adims, astr, abox, estr,
+                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS &&
+                     encode(&bmap, tma_dtype<T>(), 2, const_cast<void*>(w), bdims, astr, bbox, estr,
+                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+                if (tc) {
+                    auto kern = dcnv4::predictor_tc_kernel<T>;
+                    static std::once_flag once;
+                    static cudaError_t attr = cudaSuccess;
+                    std::call_once(once, [&] {
+                        attr = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                    static_cast<int>(kTileSmemLimit));
+                    });
+                    if (attr != cudaSuccess) return DCNV4_ERR_LAUNCH;
+                    const int nsm = sm_count();
+                    if (nsm <= 0) return DCNV4_ERR_CUDA;
+                    const unsigned grid = static_cast<unsigned>(std::min(p.tiles, nsm));
+                    if (std::getenv("DCNV4_DEBUG"))
+                        std::fprintf(stderr, "dcnv4 predictor: tcgen05 NP %d kblocks %d stages %d out bufs %d tiles %d "
+                                     "grid %u smem %zu tmem cols %u\n", p.NP, p.kblocks, p.stages, p.out_bufs, p.tiles,
+                                     grid, smem, p.tmem_cols);
+                    kern<<<grid, dcnv4::kPredThreads, smem, stream>>>(amap, bmap, bias, static_cast<T*>(rec), p);
+                    return launch_status();
+                }
+            }
+        }
+    }
+    // 8 warps per block, 4 pixels per warp; the pixels' inputs staged as fp32 in shared memory
+    const size_t psmem = static_cast<size_t>(32) * p.C * sizeof(float);
+    if (psmem > kTileSmemLimit) return DCNV4_ERR_SHAPE;
+    if (psmem > 48 * 1024) {
+        static std::once_flag once;
+        static cudaError_t attr = cudaSuccess;
+        std::call_once(once, [&] {
+            attr = cudaFuncSetAttribute(dcnv4::predictor_plain_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        static_cast<int>(kTileSmemLimit));
+        });
+        if (attr != cudaSuccess) return DCNV4_ERR_LAUNCH;
+    }
+    const long long wblocks = (static_cast<long long>(p.M) + 31) / 32;
+    const unsigned blocks = static_cast<unsigned>(std::min<long long>(wblocks, 148LL * 8));
+    dcnv4::predictor_plain_kernel<T><<<blocks, 256, psmem, stream>>>(
+        static_cast<const T*>(y), static_cast<const T*>(w), bias, static_cast<T*>(rec), p);
+    return launch_status();
+}
+
 // Two non-blocking streams per device for the host-memory entry point,
 // created on first use and kept for the life of the process.
 constexpr int kMaxDevices = 64;
@@ -600,6 +698,34 @@ int dcnv4_backward(const void* x, const void* offset_mask, const void* grad_out,
         case DCNV4_F32: return launch_backward<float>(x, offset_mask, grad_out, grad_x, grad_offset_mask, p, s);
         case DCNV4_F16: return launch_backward<__half>(x, offset_mask, grad_out, grad_x, grad_offset_mask, p, s);
         default: return launch_backward<__nv_bfloat16>(x, offset_mask, grad_out, grad_x, grad_offset_mask, p, s);
+    }
+}
+
+int dcnv4_predictor(const void* y, const void* weight, const float* bias, void* offset_mask,
+                    int M, int C, int G, int K, unsigned flags, int dtype, void* stream) {
+    if (M < 0 || C <= 0 || G <= 0 || K <= 0 || K > DCNV4_MAX_K) return DCNV4_ERR_SHAPE;
+    if (flags & ~static_cast<unsigned>(DCNV4_FLAG_REMOVE_CENTER)) return DCNV4_ERR_FLAGS;
+    if ((flags & DCNV4_FLAG_REMOVE_CENTER) && (K % 2 == 0 || K < 3)) return DCNV4_ERR_SHAPE;
+    const int e = elem_size(dtype);
+    if (!e) return DCNV4_ERR_DTYPE;
+    const long long P = points_per_unit(K, flags);
+    const long long NO = 3LL * G * P;
+    const long long ny = static_cast<long long>(M) * C, nw = NO * C, nrec = static_cast<long long>(M) * NO;
+    if (ny >= kLimit || nw >= kLimit || nrec >= kLimit) return DCNV4_ERR_TOO_LARGE;
+    if (M == 0) return DCNV4_OK;
+    if (!y || !weight || !offset_mask) return DCNV4_ERR_NULL;
+    if (!aligned(y, e) || !aligned(weight, e) || !aligned(offset_mask, e) || (bias && !aligned(bias, 4)))
+        return DCNV4_ERR_ALIGN;
+    if (overlap(offset_mask, nrec * e, y, ny * e) || overlap(offset_mask, nrec * e, weight, nw * e) ||
+        (bias && overlap(offset_mask, nrec * e, bias, NO * 4)))
+        return DCNV4_ERR_ALIAS;
+    dcnv4::PredParams p{};
+    p.M = M; p.C = C; p.G = G; p.P = static_cast<int>(P); p.NO = static_cast<int>(NO);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    switch (dtype) {
+        case DCNV4_F32: return launch_predictor<float>(y, weight, bias, offset_mask, p, s);
+        case DCNV4_F16: return launch_predictor<__half>(y, weight, bias, offset_mask, p, s);
+        default: return launch_predictor<__nv_bfloat16>(y, weight, bias, offset_mask, p, s);
     }
 }
 

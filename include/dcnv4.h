@@ -203,6 +203,31 @@ DCNV4_API int dcnv4_backward(const void *x, const void *offset_mask, const void 
                    int stride, int pad, int dilation, float offset_scale, int dtype,
                    void *stream);
 
+/* The offset/mask predictor's last step: the 1x1 projection of the block's
+ * parameter network, packed into offset_mask records. "不只是卷积的平替"
+ * (jsqmd.com), section 2: a depthwise 3x3 convolution then a 1x1 convolution
+ * to 3*groups*9 channels predict the parameters, the first 2*groups*9 being
+ * the offsets and the rest the masks; section 1's listing reads them as
+ * offset.reshape(N, G, 2, K*K, ...) and mask.reshape(N, G, K*K, ...). With
+ * P = K*K points per group (K*K - 1 with DCNV4_FLAG_REMOVE_CENTER, the only
+ * flag taken here) and NO = 3*G*P:
+ *   params[m, o] = bias[o] + sum_c weight[o, c] * y[m, c]
+ *   offset_mask[m, g, comp*P + j] = params[m, g*2P + comp*P + j]  (comp 0: x, 1: y)
+ *   offset_mask[m, g, 2P + j]     = params[m, 2GP + g*P + j]
+ * y: device, dtype, [M, C] (M pixels, e.g. N*Hout*Wout, channels-last: the
+ * depthwise convolution's output); weight: device, dtype, [NO, C];
+ * bias: device fp32 [NO] or NULL; offset_mask: device, dtype, [M, G, 3P],
+ * fully overwritten. fp32 sums, one rounding to dtype. fp16/bf16 with C a
+ * multiple of 64, NO <= 256 and 16-byte aligned pointers run on the tensor
+ * cores (tcgen05.mma, fp32 accumulators in tensor memory); other shapes and
+ * fp32 run a CUDA-core kernel. Errors: DCNV4_ERR_SHAPE (M < 0, C, G or K out
+ * of range, no centre to remove), DCNV4_ERR_FLAGS, DCNV4_ERR_DTYPE,
+ * DCNV4_ERR_TOO_LARGE (an element count >= 2^31), DCNV4_ERR_NULL,
+ * DCNV4_ERR_ALIGN, DCNV4_ERR_ALIAS (offset_mask overlaps an input).
+ * Asynchronous on `stream`; nothing is launched when M == 0. */
+DCNV4_API int dcnv4_predictor(const void *y, const void *weight, const float *bias, void *offset_mask,
+                    int M, int C, int G, int K, unsigned int flags, int dtype, void *stream);
+
 /* The integer half of the forward, exposed so that it can be compared bit for
  * bit: for every sampling point (n, ho, wo, g, k) it writes the top-left
  * corner (y0, x0) into corner[2*p], corner[2*p+1] and a 4-bit mask of the

@@ -200,3 +200,24 @@ def test_forward_ex_returns_flag_errors_before_any_cuda_call():
                               B.FLAG_REMOVE_CENTER, None)
     assert rc == B.STATUS["DCNV4_ERR_SHAPE"]
     assert lib.dcnv4_forward_ex(0, 0, 0, 0, 0, 8, 8, 16, 2, 3, 1, 1, 1, 1.0, a["dtype"], 7, None) == B.DCNV4_OK
+
+
+def _pred(y=X, w=OM, b=0, rec=OUT, M=1000, C=64, G=4, K=3, flags=0, dtype=B.DCNV4_F16):
+    return B.load_library().dcnv4_predictor(y, w, b, rec, M, C, G, K, flags, dtype, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(M=-1), "DCNV4_ERR_SHAPE"), (dict(C=0), "DCNV4_ERR_SHAPE"), (dict(G=0), "DCNV4_ERR_SHAPE"),
+    (dict(K=17), "DCNV4_ERR_SHAPE"), (dict(K=2, flags=B.FLAG_REMOVE_CENTER), "DCNV4_ERR_SHAPE"),
+    (dict(flags=B.FLAG_SOFTMAX), "DCNV4_ERR_FLAGS"), (dict(dtype=9), "DCNV4_ERR_DTYPE"),
+    (dict(y=0), "DCNV4_ERR_NULL"), (dict(w=0), "DCNV4_ERR_NULL"), (dict(rec=0), "DCNV4_ERR_NULL"),
+    (dict(y=X + 1), "DCNV4_ERR_ALIGN"), (dict(b=0x70000002), "DCNV4_ERR_ALIGN"),
+    (dict(rec=X + 64), "DCNV4_ERR_ALIAS"), (dict(rec=OM), "DCNV4_ERR_ALIAS"), (dict(b=OUT + 16), "DCNV4_ERR_ALIAS"),
+    (dict(M=1 << 25, C=128), "DCNV4_ERR_TOO_LARGE"),
+])
+def test_predictor_reports_each_error_class_before_any_cuda_call(kw, status):
+    assert _pred(**kw) == B.STATUS[status]
+
+
+def test_predictor_empty_batch_touches_nothing():
+    assert _pred(y=0, w=0, rec=0, M=0) == B.DCNV4_OK
