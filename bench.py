@@ -77,19 +77,27 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def kernel_sources_sha() -> str:
+# the source files that define each profiled kernel and its launch configuration
+KERNEL_SOURCES = {
+    "forward": ("dcnv4_kernels.cuh", "dcnv4_window.cuh", "dcnv4_host_common.inl", "dcnv4_launch_forward.inl"),
+    "backward": ("dcnv4_kernels.cuh", "dcnv4_backward.cuh", "dcnv4_host_common.inl", "dcnv4_launch_backward.inl"),
+    "predictor": ("dcnv4_kernels.cuh", "dcnv4_window.cuh", "dcnv4_predictor.cuh", "dcnv4_host_common.inl",
+                  "dcnv4_launch_predictor.inl"),
+}
+
+
+def kernel_sources_sha(kind: str = "forward") -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "deformable_convolution_sparse_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(csrc, f), "rb") as fh:
-                h.update(f.encode() + b"\0" + fh.read())
+    for f in KERNEL_SOURCES[kind]:
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode() + b"\0" + fh.read())
     return h.hexdigest()
 
 
-def profiled_traffic(workload: str):
+def profiled_traffic(workload: str, kind: str = "forward"):
     """DRAM bytes per launch from a committed ncu summary, if it was taken on the current kernel sources."""
-    sha = kernel_sources_sha()
+    sha = kernel_sources_sha(kind)
     for path in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md"))):
         fields = {}
         with open(path) as f:
@@ -97,8 +105,8 @@ def profiled_traffic(workload: str):
                 if ":" in line and line.startswith("- "):
                     k, v = line[2:].split(":", 1)
                     fields[k.strip()] = v.strip().strip("`")
-        if fields.get("workload") == workload and fields.get("kernel_sources_sha256") == sha \
-                and "dram_bytes_per_launch" in fields:
+        if fields.get("workload") == workload and fields.get("pass", "forward") == kind \
+                and fields.get("kernel_sources_sha256") == sha and "dram_bytes_per_launch" in fields:
             return int(float(fields["dram_bytes_per_launch"])), os.path.relpath(path, ROOT)
     return None, None
 
@@ -294,6 +302,7 @@ def run_backward(args, w, dev, world, rank, barrier, max_over_ranks):
     value = w.points * world * args.steps / (ms / 1e3) / 1e9
     peak, peak_kind = measured_peaks()
     achieved = foot / (ms_step / 1e3) / 1e9
+    traffic, traffic_src = profiled_traffic(w.name, "backward")
 
     # end to end: pinned host inputs copied in, backward, both gradients copied back, one stream
     xh, omh, goh = x.pin_memory(), om.pin_memory(), go.pin_memory()
@@ -348,7 +357,7 @@ def run_backward(args, w, dev, world, rank, barrier, max_over_ranks):
                          "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json)"
                          if peak_kind == "measured" else "fallback 6.65 TB/s",
                          "kernel": "dcnv4 backward (clear of grad_x + one kernel per step)",
-                         "algorithmic_bytes_per_launch": foot, "traffic": None},
+                         "algorithmic_bytes_per_launch": foot, "traffic": traffic, "traffic_source": traffic_src},
             "e2e": {"value": e2e_value, "unit": UNIT, "ms_per_step": e2e_ms / args.e2e_steps,
                     "steps": args.e2e_steps, "h2d_bytes_per_step": (nx + nom + nout) * e,
                     "d2h_bytes_per_step": (nx + nom) * 4,
@@ -524,6 +533,7 @@ def run_predictor(args, w, dev, world, rank, barrier, max_over_ranks):
     value = units * world * args.steps / (ms / 1e3) / 1e9
     peak, peak_kind = measured_peaks()
     achieved = foot / (ms_step / 1e3) / 1e9
+    traffic, traffic_src = profiled_traffic(w.name, "predictor")
 
     yh = y.pin_memory()
     oh = torch.empty(M, w.G, 3 * P, dtype=td).pin_memory()
@@ -581,7 +591,8 @@ def run_predictor(args, w, dev, world, rank, barrier, max_over_ranks):
                          "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json)"
                          if peak_kind == "measured" else "fallback 6.65 TB/s",
                          "kernel": "dcnv4 predictor (tcgen05 GEMM + packing epilogue, one launch per step)",
-                         "algorithmic_bytes_per_launch": foot, "flops_per_launch": flops, "traffic": None},
+                         "algorithmic_bytes_per_launch": foot, "flops_per_launch": flops,
+                         "traffic": traffic, "traffic_source": traffic_src},
             "e2e": {"value": units * world * args.e2e_steps / (e2e_ms / 1e3) / 1e9, "unit": "Grecords/s",
                     "ms_per_step": e2e_ms / args.e2e_steps, "steps": args.e2e_steps,
                     "h2d_bytes_per_step": y.numel() * e, "d2h_bytes_per_step": M * NO * e,

@@ -24,507 +24,13 @@ namespace {
 
 using dcnv4::FwdParams;
 
-int elem_size(int dtype) {
-    switch (dtype) {
-        case DCNV4_F32: return 4;
-        case DCNV4_F16: return 2;
-        case DCNV4_BF16: return 2;
-        default: return 0;
-    }
-}
+#include "dcnv4_host_common.inl"
 
-bool aligned(const void* p, int a) { return (reinterpret_cast<uintptr_t>(p) % static_cast<uintptr_t>(a)) == 0; }
+#include "dcnv4_launch_forward.inl"
 
-bool overlap(const void* a, long long abytes, const void* b, long long bbytes) {
-    if (abytes <= 0 || bbytes <= 0) return false;
-    const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
-    return a0 < b0 + static_cast<uintptr_t>(bbytes) && b0 < a0 + static_cast<uintptr_t>(abytes);
-}
+#include "dcnv4_launch_backward.inl"
 
-constexpr long long kLimit = 1LL << 31;  // element counts stay below 2^31 (32-bit indexing)
-
-// Shape checks shared by the forward and the index dump. Fills Hout/Wout.
-int check_geometry(int N, int H, int W, int K, int stride, int pad, int dilation, int* Hout, int* Wout) {
-    if (N < 0) return DCNV4_ERR_SHAPE;
-    const int rc = dcnv4_output_shape(H, W, K, stride, pad, dilation, Hout, Wout);
-    return rc;
-}
-
-// Checks shared by every entry point that takes the full operator signature:
-// geometry, groups, dtype, offset_scale and the 32-bit element counts of x,
-// out and offset_mask (returned through nx, nout, nom).
-int check_sizes(int N, int H, int W, int C, int G, int K, int stride, int pad, int dilation, float offset_scale,
-                int dtype, long long* nx, long long* nout, long long* nom) {
-    int Hout = 0, Wout = 0;
-    int rc = check_geometry(N, H, W, K, stride, pad, dilation, &Hout, &Wout);
-    if (rc) return rc;
-    if (C <= 0 || G <= 0) return DCNV4_ERR_SHAPE;
-    if (C % G) return DCNV4_ERR_GROUPS;
-    if (!elem_size(dtype)) return DCNV4_ERR_DTYPE;
-    if (!std::isfinite(offset_scale)) return DCNV4_ERR_SCALE;
-    *nx = static_cast<long long>(N) * H * W * C;
-    *nout = static_cast<long long>(N) * Hout * Wout * C;
-    *nom = static_cast<long long>(N) * Hout * Wout * G * 3 * K * K;
-    if (*nx >= kLimit || *nout >= kLimit || *nom >= kLimit) return DCNV4_ERR_TOO_LARGE;
-    return DCNV4_OK;
-}
-
-int launch_status() {
-    const cudaError_t e = cudaGetLastError();
-    return e == cudaSuccess ? DCNV4_OK : DCNV4_ERR_LAUNCH;
-}
-
-// ------------------------------------------------------------ dispatch ---
-
-constexpr int kThreads = 256;
-
-// Kernel choice: DCNV4_VARIANT=gather forces the global-gather kernel (A/B
-// comparisons); unset or anything else selects the persistent shared-memory
-// tile kernel whenever the shape allows it. DCNV4_HALO overrides the window
-// halo (pixels) and DCNV4_TILE=<TH>x<TW> the output tile, for tuning runs.
-enum class Variant { Auto, Gather };
-
-Variant variant_from_env() {
-    const char* v = std::getenv("DCNV4_VARIANT");
-    if (v && std::strcmp(v, "gather") == 0) return Variant::Gather;
-    return Variant::Auto;
-}
-
-constexpr size_t kTileSmemLimit = 226 * 1024;  // dynamic shared memory per CTA (sm_100: 227 KB with the static part)
-constexpr int kTileUnitsMax = 512;  // consumer threads (16 warps) per CTA, plus one producer warp
-
-PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void* ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-    });
-    return fn;
-}
-
-template <typename T> CUtensorMapDataType tma_dtype();
-template <> CUtensorMapDataType tma_dtype<float>() { return CU_TENSOR_MAP_DATA_TYPE_FLOAT32; }
-template <> CUtensorMapDataType tma_dtype<__half>() { return CU_TENSOR_MAP_DATA_TYPE_FLOAT16; }
-template <> CUtensorMapDataType tma_dtype<__nv_bfloat16>() { return CU_TENSOR_MAP_DATA_TYPE_BFLOAT16; }
-
-struct TilePlan {
-    dcnv4::TileParams p;
-    CUtensorMap map;
-    size_t smem;
-    int threads;
-};
-
-int sm_count() {
-    int dev = 0, n = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-        return 0;
-    return n;
-}
-
-// Chooses group subset, tile and halo for the tile kernel and encodes the
-// tensor map of x; false when the shape or the alignment does not suit it.
-template <typename T>
-bool plan_tile(const void* x, const void* om, const void* out, const FwdParams& f, TilePlan* plan) {
-    constexpr int E = sizeof(T);
-    const int row_bytes = f.Cg * E;
-    if (!aligned(x, 16) || !aligned(out, 16) || (f.C * E) % 16 || row_bytes % 16) return false;
-    const int Q = row_bytes / 16;
-    if (!(Q == 1 || Q == 2 || Q == 4 || Q == 5 || Q == 8)) return false;
-    if (f.KK > 64) return false;  // the per-unit mask of points outside the window has 64 bits
-    int R = 5;
-    if (const char* h = std::getenv("DCNV4_HALO")) R = std::atoi(h) > 0 ? std::atoi(h) : R;
-    int forceTH = 0, forceTW = 0, forceGS = 0, forceNrec = 0;
-    if (const char* n = std::getenv("DCNV4_NREC")) forceNrec = (std::atoi(n) == 2 || std::atoi(n) == 3) ? std::atoi(n) : 0;
-    if (const char* t = std::getenv("DCNV4_TILE")) std::sscanf(t, "%dx%d", &forceTH, &forceTW);
-    if (const char* g = std::getenv("DCNV4_GS")) forceGS = std::atoi(g);
-    const int R3 = 3 * f.npts;
-    const int nsm = sm_count();
-    if (nsm <= 0) return false;
-
-    static const int THs[] = {1, 2, 4, 7, 8, 14, 16, 28, 32};
-    static const int TWs[] = {1, 2, 4, 7, 8, 14, 16, 28, 32};
-    double best = -1.0;
-    dcnv4::TileParams bp{};
-    int best_threads = 0, best_c2 = 0;
-    size_t best_smem = 0;
-    for (int GS = 1; GS <= f.G; ++GS) {
-        if (f.G % GS || (forceGS && GS != forceGS)) continue;
-        const int PB = GS * row_bytes;
-        const int sub_ch = GS * f.Cg;
-        int c2 = 0;
-        for (int d = std::min(sub_ch, 256); d >= 1; --d)
-            if (sub_ch % d == 0 && (d * E) % 16 == 0) { c2 = d; break; }
-        if (c2 == 0 || sub_ch / c2 > 256) continue;
-        // a pixel stride that is a multiple of 128 bytes keeps the gathers free of
-        // bank conflicts (see the kernel); other strides pay for some
-        const double banks = (PB % 128 == 0) ? 1.0 : 0.6;
-        const bool row_runs = GS == f.G;
-        for (int TH : THs) {
-            for (int TW : TWs) {
-                if (forceTH && (TH != forceTH || TW != forceTW)) continue;
-                const int units = TH * TW * GS;
-                if (units > kTileUnitsMax || units < 32) continue;
-                if (TH > f.Hout + 7 || TW > f.Wout + 7) continue;
-                const int WH = (TH - 1) * f.stride + (f.K - 1) * f.dilation + 2 * R + 1;
-                const int WW = (TW - 1) * f.stride + (f.K - 1) * f.dilation + 2 * R + 1;
-                if (WH > 256 || WW > 256) continue;
-                const int nruns = row_runs ? TH : TH * TW;
-                const int count = (row_runs ? TW * f.G : GS) * R3;
-                const int slot = (count * E + 32 + 15) / 16 * 16;
-                const size_t rec = (static_cast<size_t>(nruns) * slot + 127) / 128 * 128;
-                const size_t win = (static_cast<size_t>(WH) * WW * PB + 127) / 128 * 128;
-                // records get a third buffer (a longer lead for their DRAM reads) when it fits
-                int nrec = (2 * win + 3 * rec <= kTileSmemLimit) ? 3 : 2;
-                if (forceNrec) nrec = forceNrec;
-                const size_t smem = 2 * win + nrec * rec;
-                if (smem > kTileSmemLimit) continue;
-                const int threads = (units + 31) / 32 * 32 + 32;  // consumers + the producer warp
-                const int tiles_y = (f.Hout + TH - 1) / TH, tiles_x = (f.Wout + TW - 1) / TW;
-                const long long tiles = static_cast<long long>(f.N) * tiles_y * tiles_x * (f.G / GS);
-                // the choice must not depend on N: an image's result (which samples take
-                // the window path) then never depends on the batch it comes in. The wave
-                // balance is judged for a nominal batch of 64 images.
-                const long long tiles_nominal = 64LL * tiles_y * tiles_x * (f.G / GS);
-                const int per_sm = std::max(1, static_cast<int>(std::min<size_t>(
-                                                   (kTileSmemLimit + 2048) / (smem + 1024), 2048 / threads)));
-                const double slots = static_cast<double>(nsm) * per_sm;
-                const double waves = static_cast<double>(tiles_nominal) / slots;
-                const double balance = waves / std::ceil(waves);
-                const double useful =
-                    static_cast<double>(f.Hout) * f.Wout / (static_cast<double>(tiles_y) * TH * tiles_x * TW);
-                const double reuse = static_cast<double>(TH * TW) / (static_cast<double>(WH) * WW);
-                const double fill = static_cast<double>(units) / (threads - 32);
-                const double occ = std::min(1.0, per_sm * (threads - 32) / 384.0);
-                const double depth = nrec == 3 ? 1.0 : 0.9;
-                // a ragged tile loses threads and still loads a full window: useful counts twice
-                const double score = useful * useful * balance * fill * occ * banks * depth * std::sqrt(reuse);
-                if (score > best) {
-                    best = score;
-                    bp.TH = TH; bp.TW = TW; bp.tiles_x = tiles_x; bp.tiles_y = tiles_y;
-                    bp.WH = WH; bp.WW = WW; bp.run_slot = slot; bp.rec_bytes = static_cast<int>(rec);
-                    bp.win_bytes = static_cast<int>(win);
-                    bp.nrec = nrec;
-                    bp.tiles = static_cast<int>(tiles); bp.units = units;
-                    bp.GS = GS; bp.PB = PB; bp.cblk = sub_ch / c2;
-                    best_threads = threads;
-                    best_smem = smem;
-                    best_c2 = c2;
-                }
-            }
-        }
-    }
-    if (best < 0) return false;
-    const int GS = bp.GS, PB = bp.PB, c2 = best_c2;
-    bp.f = f;
-    bp.nsub = f.G / GS;
-    bp.R = R;
-    const size_t om_bytes = static_cast<size_t>(f.N) * f.Hout * f.Wout * f.G * R3 * E;
-    bp.om_lo = reinterpret_cast<unsigned long long>(om);
-    bp.om_hi = bp.om_lo + om_bytes;
-    bp.div_tw_gs = dcnv4::make_fastdiv(bp.TW * GS);
-    bp.div_gs = dcnv4::make_fastdiv(GS);
-    bp.div_nsub = dcnv4::make_fastdiv(bp.nsub);
-    bp.div_tx = dcnv4::make_fastdiv(bp.tiles_x);
-    bp.div_ty = dcnv4::make_fastdiv(bp.tiles_y);
-
-    auto encode = tensor_map_encoder();
-    if (!encode) return false;
-    const cuuint64_t dims[5] = {static_cast<cuuint64_t>(c2), static_cast<cuuint64_t>(f.C / c2),
-                                static_cast<cuuint64_t>(f.W), static_cast<cuuint64_t>(f.H),
-                                static_cast<cuuint64_t>(f.N)};
-    const cuuint64_t strides[4] = {static_cast<cuuint64_t>(c2) * E, static_cast<cuuint64_t>(f.C) * E,
-                                   static_cast<cuuint64_t>(f.W) * f.C * E,
-                                   static_cast<cuuint64_t>(f.H) * f.W * f.C * E};
-    const cuuint32_t box[5] = {static_cast<cuuint32_t>(c2), static_cast<cuuint32_t>(bp.cblk),
-                               static_cast<cuuint32_t>(bp.WW), static_cast<cuuint32_t>(bp.WH), 1u};
-    const cuuint32_t estr[5] = {1u, 1u, 1u, 1u, 1u};
-    if (encode(&plan->map, tma_dtype<T>(), 5, const_cast<void*>(x), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-        return false;
-    plan->p = bp;
-    plan->smem = best_smem;
-    plan->threads = best_threads;
-    if (const char* d = std::getenv("DCNV4_DEBUG"); d && *d == '1')
-        std::fprintf(stderr,
-                     "dcnv4 tile plan: tile %dx%d GS %d (nsub %d) R %d window %dx%d PB %d cblk %d tiles %d units %d "
-                     "threads %d nrec %d smem %zu\n",
-                     bp.TH, bp.TW, GS, bp.nsub, R, bp.WH, bp.WW, PB, bp.cblk, bp.tiles, bp.units, best_threads,
-                     bp.nrec, best_smem);
-    return true;
-}
-
-// fp16 storage: weights rounded to fp16 for the mixed-precision FMA (default)
-// or kept in fp32 (DCNV4_F16_EXACT=1, for comparisons).
-bool f16_exact_from_env() {
-    const char* v = std::getenv("DCNV4_F16_EXACT");
-    return v && *v == '1';
-}
-
-template <typename T, int Q, int KS, bool HW, int PBC, bool VF = false>
-int launch_tile_q(const T* x, const T* om, T* out, const TilePlan& plan, cudaStream_t stream) {
-    auto kern = dcnv4::fwd_tile_kernel<T, Q, KS, HW, PBC, VF>;
-    static std::once_flag once;
-    static cudaError_t attr = cudaSuccess;
-    std::call_once(once, [&] {
-        attr = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kTileSmemLimit));
-    });
-    if (attr != cudaSuccess) return DCNV4_ERR_LAUNCH;
-    int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, plan.threads, plan.smem) != cudaSuccess || per_sm < 1)
-        return DCNV4_ERR_LAUNCH;
-    const long long slots = static_cast<long long>(sm_count()) * per_sm;
-    const unsigned grid = static_cast<unsigned>(std::min<long long>(plan.p.tiles, slots));
-    kern<<<grid, plan.threads, plan.smem, stream>>>(plan.map, x, om, out, plan.p);
-    return launch_status();
-}
-
-template <typename T, int Q, bool HW, bool VF>
-int launch_tile_v(const T* x, const T* om, T* out, const TilePlan& plan, cudaStream_t s) {
-    // a 128-byte window pixel (the common case) as a compile-time stride
-    if constexpr (Q != 5) {
-        if (plan.p.PB == 128) {
-            if (plan.p.f.K == 3) return launch_tile_q<T, Q, 3, HW, 128, VF>(x, om, out, plan, s);
-            return launch_tile_q<T, Q, 0, HW, 128, VF>(x, om, out, plan, s);
-        }
-    }
-    if (plan.p.f.K == 3) return launch_tile_q<T, Q, 3, HW, 0, VF>(x, om, out, plan, s);
-    return launch_tile_q<T, Q, 0, HW, 0, VF>(x, om, out, plan, s);
-}
-
-template <typename T, int Q, bool HW>
-int launch_tile_k(const T* x, const T* om, T* out, const TilePlan& plan, cudaStream_t s) {
-    // the variant flags get their own instantiations, so that the plain forward carries none of their code
-    if (plan.p.f.flags != 0) return launch_tile_v<T, Q, HW, true>(x, om, out, plan, s);
-    return launch_tile_v<T, Q, HW, false>(x, om, out, plan, s);
-}
-
-template <typename T, int Q>
-int launch_tile_k(const T* x, const T* om, T* out, const TilePlan& plan, cudaStream_t s) {
-    if constexpr (std::is_same<T, __half>::value) {
-        if (!f16_exact_from_env()) return launch_tile_k<T, Q, true>(x, om, out, plan, s);
-    }
-    return launch_tile_k<T, Q, false>(x, om, out, plan, s);
-}
-
-template <typename T>
-int launch_tile(const void* x, const void* om, void* out, const TilePlan& plan, cudaStream_t s) {
-    const T* xt = static_cast<const T*>(x);
-    const T* omt = static_cast<const T*>(om);
-    T* ot = static_cast<T*>(out);
-    switch (plan.p.f.Cg * static_cast<int>(sizeof(T)) / 16) {
-        case 1: return launch_tile_k<T, 1>(xt, omt, ot, plan, s);
-        case 2: return launch_tile_k<T, 2>(xt, omt, ot, plan, s);
-        case 4: return launch_tile_k<T, 4>(xt, omt, ot, plan, s);
-        case 5: return launch_tile_k<T, 5>(xt, omt, ot, plan, s);
-        default: return launch_tile_k<T, 8>(xt, omt, ot, plan, s);
-    }
-}
-
-template <typename T>
-int launch_forward(const void* x, const void* om, void* out, FwdParams p, cudaStream_t stream) {
-    constexpr int E = sizeof(T);
-    if (variant_from_env() == Variant::Auto) {
-        TilePlan plan;
-        if (plan_tile<T>(x, om, out, p, &plan)) return launch_tile<T>(x, om, out, plan, stream);
-    }
-    const int row_bytes = p.Cg * E;
-    const bool a16 = aligned(x, 16) && aligned(out, 16) && (p.C * E) % 16 == 0;
-    const bool a32 = aligned(x, 32) && aligned(out, 32) && (p.C * E) % 32 == 0;
-    const size_t rec_bytes = static_cast<size_t>(3) * p.npts * E;
-
-    int lane_bytes = 0, vec_bytes = 0;
-    if (a16 && row_bytes % 16 == 0) {
-        if (a32 && row_bytes % 32 == 0) {
-            vec_bytes = 32;
-            lane_bytes = (E == 4 && row_bytes % 64 == 0) ? 64 : 32;
-        } else {
-            vec_bytes = 16;
-            lane_bytes = 16;
-        }
-    }
-    if (lane_bytes) {
-        p.chunks = row_bytes / lane_bytes;
-        p.lanes = p.chunks < kThreads ? p.chunks : kThreads;
-    } else {
-        p.chunks = p.Cg;
-        p.lanes = p.Cg < kThreads ? p.Cg : kThreads;
-    }
-    int upb = kThreads / p.lanes;
-    const size_t smem_cap = 40 * 1024;
-    while (upb > 1 && upb * rec_bytes + 16 > smem_cap) --upb;
-    p.units_per_block = upb;
-    const size_t smem = upb * rec_bytes + 16;
-    const int threads = upb * p.lanes;
-    const long long blocks = (static_cast<long long>(p.units) + upb - 1) / upb;
-    if (blocks > 0x7fffffffLL) return DCNV4_ERR_TOO_LARGE;
-    const dim3 grid(static_cast<unsigned>(blocks));
-
-    const T* xt = static_cast<const T*>(x);
-    const T* omt = static_cast<const T*>(om);
-    T* ot = static_cast<T*>(out);
-    const bool k3 = p.K == 3;
-    if (lane_bytes == 64) {
-        if (k3) dcnv4::fwd_vector_kernel<T, 32, 64, 3><<<grid, threads, smem, stream>>>(xt, omt, ot, p);
-        else dcnv4::fwd_vector_kernel<T, 32, 64, 0><<<grid, threads, smem, stream>>>(xt, omt, ot, p);
-    } else if (lane_bytes == 32) {
-        if (k3) dcnv4::fwd_vector_kernel<T, 32, 32, 3><<<grid, threads, smem, stream>>>(xt, omt, ot, p);
-        else dcnv4::fwd_vector_kernel<T, 32, 32, 0><<<grid, threads, smem, stream>>>(xt, omt, ot, p);
-    } else if (lane_bytes == 16) {
-        if (k3) dcnv4::fwd_vector_kernel<T, 16, 16, 3><<<grid, threads, smem, stream>>>(xt, omt, ot, p);
-        else dcnv4::fwd_vector_kernel<T, 16, 16, 0><<<grid, threads, smem, stream>>>(xt, omt, ot, p);
-    } else {
-        if (k3) dcnv4::fwd_scalar_kernel<T, 3><<<grid, threads, smem, stream>>>(xt, omt, ot, p);
-        else dcnv4::fwd_scalar_kernel<T, 0><<<grid, threads, smem, stream>>>(xt, omt, ot, p);
-    }
-    return launch_status();
-}
-
-// Backward: grad_x is cleared on the stream, then one kernel computes every
-// gradient. Vector path (4 channels per thread, float4 reductions) when the
-// pointers and channel counts allow it, element path otherwise.
-template <typename T>
-int launch_backward(const void* x, const void* om, const void* go, float* gx, float* gom, FwdParams p,
-                    cudaStream_t stream) {
-    constexpr int E = sizeof(T);
-    const bool vec = aligned(x, 4 * E) && aligned(go, 4 * E) && aligned(gx, 16) && p.C % 4 == 0 && p.Cg % 4 == 0;
-    const int cpl = vec ? 4 : 1;
-    p.chunks = p.Cg / cpl;
-    int lanes = 1;
-    while (lanes < p.chunks && lanes < 32) lanes <<= 1;
-    p.lanes = lanes;
-    // units per block: full warps, records and fp32 gradient records in shared memory
-    const size_t R = static_cast<size_t>(3) * p.KK;
-    const int step = lanes < 32 ? 32 / lanes : 1;
-    auto smem_for = [&](int upb) {
-        return ((upb * R * E + 16 + 15) & ~static_cast<size_t>(15)) + upb * R * sizeof(float);
-    };
-    int upb = kThreads / lanes;
-    while (upb > step && smem_for(upb) > 48 * 1024) upb -= step;
-    p.units_per_block = upb;
-    const size_t smem = smem_for(upb);
-    const long long blocks = (static_cast<long long>(p.units) + upb - 1) / upb;
-    if (blocks > 0x7fffffffLL) return DCNV4_ERR_TOO_LARGE;
-
-    const size_t gx_bytes = static_cast<size_t>(p.N) * p.H * p.W * p.C * sizeof(float);
-    if (cudaMemsetAsync(gx, 0, gx_bytes, stream) != cudaSuccess) return DCNV4_ERR_CUDA;
-    const T* xt = static_cast<const T*>(x);
-    const T* omt = static_cast<const T*>(om);
-    const T* got = static_cast<const T*>(go);
-    const int threads = upb * lanes;
-    auto run = [&](auto kernel) -> int {
-        if (smem > 48 * 1024 &&
-            cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
-                cudaSuccess)
-            return DCNV4_ERR_LAUNCH;
-        kernel<<<static_cast<unsigned>(blocks), threads, smem, stream>>>(xt, omt, got, gx, gom, p);
-        return launch_status();
-    };
-    const bool k3 = p.K == 3;
-    if (vec) return k3 ? run(dcnv4::bwd_kernel<T, 4, 3>) : run(dcnv4::bwd_kernel<T, 4, 0>);
-    return k3 ? run(dcnv4::bwd_kernel<T, 1, 3>) : run(dcnv4::bwd_kernel<T, 1, 0>);
-}
-
-// Offset/mask predictor: the tensor-core kernel for fp16/bf16 with C a multiple
-// of 64 and at most 256 output channels (DCNV4_PRED_VARIANT=plain forces the
-// CUDA-core kernel), the CUDA-core kernel otherwise.
-template <typename T>
-int launch_predictor(const void* y, const void* w, const float* bias, void* rec, dcnv4::PredParams p,
-                     cudaStream_t stream) {
-    constexpr int E = sizeof(T);
-    const char* pv = std::getenv("DCNV4_PRED_VARIANT");
-    const bool force_plain = pv && std::strcmp(pv, "plain") == 0;
-    bool tc = !force_plain && E == 2 && p.C % 64 == 0 && p.NO <= 256 && aligned(y, 16) && aligned(w, 16) &&
-              aligned(rec, 16) && p.M > 0;
-    if constexpr (E == 2) {
-        if (tc) {
-            p.NP = (p.NO + 15) / 16 * 16;
-            p.kblocks = p.C / 64;
-            p.tiles = (p.M + 127) / 128;
-            unsigned cols = 32;
-            while (cols < 2u * static_cast<unsigned>(p.NP)) cols <<= 1;
-            p.tmem_cols = cols;
-            p.a_fmt = std::is_same<T, __half>::value ? 0 : 1;
-            const size_t b_bytes = static_cast<size_t>(p.kblocks) * p.NP * 128;
-            const size_t a_stage = static_cast<size_t>(p.kblocks) * 128 * 128;
-            const size_t meta = static_cast<size_t>(p.NO) * 8 + 8 + 8 * 16 + 16;
-            // two output staging buffers (store of tile i overlaps the epilogue of tile i+1) when they fit
-            size_t o_bytes = 0, fixed = 0;
-            int stages = 0;
-            for (int ob = 2; ob >= 1 && stages < 2; --ob) {
-                o_bytes = (static_cast<size_t>(ob) * 128 * p.NO * E + 15) / 16 * 16;
-                fixed = 1024 + b_bytes + o_bytes + meta;
-                stages = 4;
-                while (stages >= 2 && fixed + stages * a_stage > kTileSmemLimit) --stages;
-                p.out_bufs = ob;
-            }
-            tc = stages >= 2;
-            if (tc) {
-                p.stages = stages;
-                p.smem_b = 0;
-                p.smem_a = static_cast<unsigned>(b_bytes);
-                p.smem_o = static_cast<unsigned>(b_bytes + stages * a_stage);
-                p.smem_meta = static_cast<unsigned>(p.smem_o + o_bytes);
-                const size_t smem = fixed + stages * a_stage;
-                auto encode = tensor_map_encoder();
-                CUtensorMap amap, bmap;
-                const cuuint32_t estr[2] = {1u, 1u};
-                const cuuint64_t adims[2] = {static_cast<cuuint64_t>(p.C), static_cast<cuuint64_t>(p.M)};
-                const cuuint64_t astr[1] = {static_cast<cuuint64_t>(p.C) * E};
-                const cuuint32_t abox[2] = {64u, 128u};
-                const cuuint64_t bdims[2] = {static_cast<cuuint64_t>(p.C), static_cast<cuuint64_t>(p.NO)};
-                const cuuint32_t bbox[2] = {64u, static_cast<cuuint32_t>(p.NP)};
-                tc = encode &&
-                     encode(&amap, tma_dtype<T>(), 2, const_cast<void*>(y), adims, astr, abox, estr,
-                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS &&
-                     encode(&bmap, tma_dtype<T>(), 2, const_cast<void*>(w), bdims, astr, bbox, estr,
-                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-                if (tc) {
-                    auto kern = dcnv4::predictor_tc_kernel<T>;
-                    static std::once_flag once;
-                    static cudaError_t attr = cudaSuccess;
-                    std::call_once(once, [&] {
-                        attr = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                    static_cast<int>(kTileSmemLimit));
-                    });
-                    if (attr != cudaSuccess) return DCNV4_ERR_LAUNCH;
-                    const int nsm = sm_count();
-                    if (nsm <= 0) return DCNV4_ERR_CUDA;
-                    const unsigned grid = static_cast<unsigned>(std::min(p.tiles, nsm));
-                    if (std::getenv("DCNV4_DEBUG"))
-                        std::fprintf(stderr, "dcnv4 predictor: tcgen05 NP %d kblocks %d stages %d out bufs %d tiles %d "
-                                     "grid %u smem %zu tmem cols %u\n", p.NP, p.kblocks, p.stages, p.out_bufs, p.tiles,
-                                     grid, smem, p.tmem_cols);
-                    kern<<<grid, dcnv4::kPredThreads, smem, stream>>>(amap, bmap, bias, static_cast<T*>(rec), p);
-                    return launch_status();
-                }
-            }
-        }
-    }
-    // 8 warps per block, 4 pixels per warp; the pixels' inputs staged as fp32 in shared memory
-    const size_t psmem = static_cast<size_t>(32) * p.C * sizeof(float);
-    if (psmem > kTileSmemLimit) return DCNV4_ERR_SHAPE;
-    if (psmem > 48 * 1024) {
-        static std::once_flag once;
-        static cudaError_t attr = cudaSuccess;
-        std::call_once(once, [&] {
-            attr = cudaFuncSetAttribute(dcnv4::predictor_plain_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        static_cast<int>(kTileSmemLimit));
-        });
-        if (attr != cudaSuccess) return DCNV4_ERR_LAUNCH;
-    }
-    const long long wblocks = (static_cast<long long>(p.M) + 31) / 32;
-    const unsigned blocks = static_cast<unsigned>(std::min<long long>(wblocks, 148LL * 8));
-    dcnv4::predictor_plain_kernel<T><<<blocks, 256, psmem, stream>>>(
-        static_cast<const T*>(y), static_cast<const T*>(w), bias, static_cast<T*>(rec), p);
-    return launch_status();
-}
+#include "dcnv4_launch_predictor.inl"
 
 // Two non-blocking streams per device for the host-memory entry point,
 // created on first use and kept for the life of the process.
