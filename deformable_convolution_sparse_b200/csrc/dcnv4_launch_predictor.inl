@@ -57,12 +57,21 @@ int launch_predictor(const void* y, const void* w, const float* bias, void* rec,
                             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
                 if (tc) {
-                    auto kern = dcnv4::predictor_tc_kernel<T>;
+                    // epilogue warps: DCNV4_PRED_EPI=8 or 16 (tuning runs); default 16
+                    int epw = 16;
+                    if (const char* e = std::getenv("DCNV4_PRED_EPI")) epw = std::atoi(e) == 8 ? 8 : 16;
+                    auto kern = epw == 8 ? dcnv4::predictor_tc_kernel<T, 8> : dcnv4::predictor_tc_kernel<T, 16>;
+                    const int threads = 64 + 32 * epw;
                     static std::once_flag once;
                     static cudaError_t attr = cudaSuccess;
                     std::call_once(once, [&] {
-                        attr = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                        attr = cudaFuncSetAttribute(dcnv4::predictor_tc_kernel<T, 8>,
+                                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                     static_cast<int>(kTileSmemLimit));
+                        if (attr == cudaSuccess)
+                            attr = cudaFuncSetAttribute(dcnv4::predictor_tc_kernel<T, 16>,
+                                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                        static_cast<int>(kTileSmemLimit));
                     });
                     if (attr != cudaSuccess) return DCNV4_ERR_LAUNCH;
                     const int nsm = sm_count();
@@ -70,9 +79,9 @@ int launch_predictor(const void* y, const void* w, const float* bias, void* rec,
                     const unsigned grid = static_cast<unsigned>(std::min(p.tiles, nsm));
                     if (std::getenv("DCNV4_DEBUG"))
                         std::fprintf(stderr, "dcnv4 predictor: tcgen05 NP %d kblocks %d stages %d out bufs %d tiles %d "
-                                     "grid %u smem %zu tmem cols %u\n", p.NP, p.kblocks, p.stages, p.out_bufs, p.tiles,
-                                     grid, smem, p.tmem_cols);
-                    kern<<<grid, dcnv4::kPredThreads, smem, stream>>>(amap, bmap, bias, static_cast<T*>(rec), p);
+                                     "grid %u smem %zu tmem cols %u epilogue warps %d\n", p.NP, p.kblocks, p.stages,
+                                     p.out_bufs, p.tiles, grid, smem, p.tmem_cols, epw);
+                    kern<<<grid, threads, smem, stream>>>(amap, bmap, bias, static_cast<T*>(rec), p);
                     return launch_status();
                 }
             }

@@ -20,8 +20,8 @@
 // Warp 1 (one lane) issues tcgen05.mma (M = 128, N = NP = NO rounded up to 16,
 // K = 16 per instruction, fp32 accumulators in tensor memory, two accumulator
 // buffers) and commits each tile to mbarriers that free its activation stage
-// and hand its accumulator to the epilogue. Warps 2..9 (two per 32-lane quarter
-// of tensor memory, alternate 16-column chunks) read their rows with tcgen05.ld
+// and hand its accumulator to the epilogue. The epilogue warps (EPW / 4 per
+// 32-lane quarter of tensor memory, interleaved 16-column chunks) read their rows with tcgen05.ld
 // (up to four loads in flight per wait), add the bias, round to the
 // storage type, place every channel at its record slot in a shared-memory
 // staging tile, and one thread writes the tile -- 128 consecutive records,
@@ -146,12 +146,10 @@ __device__ __forceinline__ T from_float(float v) {
     else return __float2bfloat16_rn(v);
 }
 
-constexpr int kPredEpiWarps = 8;                         // two per 32-lane quarter of tensor memory
-constexpr int kPredThreads = 64 + 32 * kPredEpiWarps;    // + the load warp and the MMA warp
-
-// kPredThreads threads: warp 0 loads, warp 1 issues the MMAs, warps 2.. run the epilogue.
-template <typename T>
-__global__ void __launch_bounds__(kPredThreads, 1)
+// 64 + 32 * EPW threads: warp 0 loads, warp 1 issues the MMAs, EPW epilogue
+// warps (a multiple of 4: EPW / 4 per 32-lane quarter of tensor memory).
+template <typename T, int EPW>
+__global__ void __launch_bounds__(64 + 32 * EPW, 1)
 predictor_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap bmap,
                     const float* __restrict__ bias, T* __restrict__ rec, PredParams p) {
     extern __shared__ unsigned char pred_smem_raw[];
@@ -188,7 +186,7 @@ predictor_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_const
         mbar_init(b_full, 1);
         for (int b = 0; b < 2; ++b) {
             mbar_init(&acc_full[b], 1);
-            mbar_init(&acc_empty[b], 32 * kPredEpiWarps);
+            mbar_init(&acc_empty[b], 32 * EPW);
         }
         fence_barrier_init();
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&amap)) : "memory");
@@ -283,10 +281,11 @@ predictor_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_const
         }
     } else {
         // ------------------------------------------------------------ epilogue
-        constexpr int NE = 32 * kPredEpiWarps;    // epilogue threads
+        constexpr int NE = 32 * EPW;              // epilogue threads
+        constexpr int EPQ = EPW / 4;              // epilogue warps per quarter
         const int et = tid - 64;                  // 0 .. NE-1
         const int quarter = warp & 3;             // tensor-memory lanes 32*quarter .. +31
-        const int half = (warp - 2) >> 2;         // which 16-column chunks: half, half + 2, ...
+        const int part = (warp - 2) >> 2;         // which 16-column chunks: part, part + EPQ, ...
         const int row = quarter * 32 + lane;      // row of the tile (pixel)
         const int nch = p.NP / 16;
         const size_t rec_tile = static_cast<size_t>(128) * p.NO;  // elements per full tile
@@ -310,12 +309,12 @@ predictor_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_const
                                    static_cast<uint32_t>(b * p.NP);
             T* orow = ob + static_cast<size_t>(row) * p.NO;
             // up to four 16-column loads in flight before one wait
-            for (int c = half; c < nch; c += 8) {
+            for (int c = part; c < nch; c += 4 * EPQ) {
                 float v[4][16];
                 int n = 0;
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
-                    const int cc = c + 2 * q;
+                    const int cc = c + EPQ * q;
                     if (cc < nch) {
                         tmem_ld16_nowait(taddr + static_cast<uint32_t>(cc * 16), v[q]);
                         n = q + 1;
@@ -325,7 +324,7 @@ predictor_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_const
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
                     if (q >= n) break;
-                    const int c0 = (c + 2 * q) * 16;  // columns are record slots
+                    const int c0 = (c + EPQ * q) * 16;  // columns are record slots
                     if (p.NO % 2 == 0) {
                         // pairs of slots as one 32-bit store (row * NO and c0 are even)
 #pragma unroll
