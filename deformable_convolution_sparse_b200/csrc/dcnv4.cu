@@ -36,7 +36,7 @@ using dcnv4::FwdParams;
 // created on first use and kept for the life of the process.
 constexpr int kMaxDevices = 64;
 struct HostPipe {
-    cudaStream_t s[2] = {nullptr, nullptr};
+    cudaStream_t s[3] = {nullptr, nullptr, nullptr};
     bool ready = false;
 };
 HostPipe g_pipes[kMaxDevices];
@@ -48,7 +48,7 @@ int host_pipe(HostPipe** out) {
     std::lock_guard<std::mutex> lock(g_pipe_mutex);
     HostPipe& p = g_pipes[dev];
     if (!p.ready) {
-        for (int i = 0; i < 2; ++i)
+        for (int i = 0; i < 3; ++i)
             if (cudaStreamCreateWithFlags(&p.s[i], cudaStreamNonBlocking) != cudaSuccess) return DCNV4_ERR_CUDA;
         p.ready = true;
     }
@@ -259,7 +259,12 @@ int dcnv4_forward_host(const void* x_host, const void* offset_mask_host, void* o
     rc = host_pipe(&pipe);
     if (rc) return rc;
     cudaStream_t user = static_cast<cudaStream_t>(stream);
-    cudaEvent_t ev_start = nullptr, ev_done[2] = {nullptr, nullptr};
+    // chunks of whole images on NS streams, so that copies in the two directions and the kernels overlap;
+    // DCNV4_HOST_CHUNKS / DCNV4_HOST_STREAMS override the defaults for tuning runs
+    int max_chunks = 16, NS = 3;
+    if (const char* c = std::getenv("DCNV4_HOST_CHUNKS")) max_chunks = std::max(1, std::atoi(c));
+    if (const char* c = std::getenv("DCNV4_HOST_STREAMS")) NS = std::min(3, std::max(1, std::atoi(c)));
+    cudaEvent_t ev_start = nullptr, ev_done[3] = {nullptr, nullptr, nullptr};
     auto fail = [&](int code) {
         if (ev_start) cudaEventDestroy(ev_start);
         for (auto& ev : ev_done)
@@ -270,11 +275,10 @@ int dcnv4_forward_host(const void* x_host, const void* offset_mask_host, void* o
     for (auto& ev : ev_done)
         if (cudaEventCreateWithFlags(&ev, cudaEventDisableTiming) != cudaSuccess) return fail(DCNV4_ERR_CUDA);
     if (cudaEventRecord(ev_start, user) != cudaSuccess) return fail(DCNV4_ERR_CUDA);
-    for (int i = 0; i < 2; ++i)
+    for (int i = 0; i < NS; ++i)
         if (cudaStreamWaitEvent(pipe->s[i], ev_start, 0) != cudaSuccess) return fail(DCNV4_ERR_CUDA);
 
-    // chunks of whole images: enough of them for the two copy directions to overlap
-    const int chunks = N < 8 ? N : 8;
+    const int chunks = N < max_chunks ? N : max_chunks;
     const char* xh = static_cast<const char*>(x_host);
     const char* omh = static_cast<const char*>(offset_mask_host);
     char* oh = static_cast<char*>(out_host);
@@ -286,7 +290,7 @@ int dcnv4_forward_host(const void* x_host, const void* offset_mask_host, void* o
         const int n1 = static_cast<int>((static_cast<long long>(N) * (c + 1)) / chunks);
         const int nc = n1 - n0;
         if (nc == 0) continue;
-        cudaStream_t s = pipe->s[c & 1];
+        cudaStream_t s = pipe->s[c % NS];
         if (cudaMemcpyAsync(xd + n0 * x_img, xh + n0 * x_img, nc * x_img, cudaMemcpyHostToDevice, s) != cudaSuccess ||
             cudaMemcpyAsync(omd + n0 * om_img, omh + n0 * om_img, nc * om_img, cudaMemcpyHostToDevice, s) != cudaSuccess)
             return fail(DCNV4_ERR_CUDA);
@@ -297,7 +301,7 @@ int dcnv4_forward_host(const void* x_host, const void* offset_mask_host, void* o
             return fail(DCNV4_ERR_CUDA);
         n0 = n1;
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < NS; ++i) {
         if (cudaEventRecord(ev_done[i], pipe->s[i]) != cudaSuccess || cudaStreamWaitEvent(user, ev_done[i], 0) != cudaSuccess)
             return fail(DCNV4_ERR_CUDA);
     }

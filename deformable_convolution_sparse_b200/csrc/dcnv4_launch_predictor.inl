@@ -87,21 +87,10 @@ int launch_predictor(const void* y, const void* w, const float* bias, void* rec,
             }
         }
     }
-    // 8 warps per block, 4 pixels per warp; the pixels' inputs staged as fp32 in shared memory
-    const size_t psmem = static_cast<size_t>(32) * p.C * sizeof(float);
-    if (psmem > kTileSmemLimit) return DCNV4_ERR_SHAPE;
-    if (psmem > 48 * 1024) {
-        static std::once_flag once;
-        static cudaError_t attr = cudaSuccess;
-        std::call_once(once, [&] {
-            attr = cudaFuncSetAttribute(dcnv4::predictor_plain_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        static_cast<int>(kTileSmemLimit));
-        });
-        if (attr != cudaSuccess) return DCNV4_ERR_LAUNCH;
-    }
+    // 8 warps per block, 4 pixels per warp
     const long long wblocks = (static_cast<long long>(p.M) + 31) / 32;
     const unsigned blocks = static_cast<unsigned>(std::min<long long>(wblocks, 148LL * 8));
-    dcnv4::predictor_plain_kernel<T><<<blocks, 256, psmem, stream>>>(
+    dcnv4::predictor_plain_kernel<T><<<blocks, 256, 0, stream>>>(
         static_cast<const T*>(y), static_cast<const T*>(w), bias, static_cast<T*>(rec), p);
     return launch_status();
 }

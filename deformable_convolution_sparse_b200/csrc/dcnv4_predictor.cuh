@@ -374,43 +374,37 @@ predictor_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_const
 
 // CUDA-core kernel for the shapes and types the tensor-core kernel does not
 // take: one warp per 4 pixels; for every output channel the lanes read the
-// weight row (coalesced, it stays in L1/L2) against the pixels' inputs staged
-// in shared memory as fp32, and a warp reduction gives the 4 sums.
+// weight row and the 4 input rows (coalesced; both stay in L1/L2) and a warp
+// reduction gives the 4 sums.
 template <typename T>
 __global__ void __launch_bounds__(256)
 predictor_plain_kernel(const T* __restrict__ y, const T* __restrict__ w, const float* __restrict__ bias,
                        T* __restrict__ rec, PredParams p) {
-    extern __shared__ float ybuf[];  // [8 warps][4 pixels][C]
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    float* yw = ybuf + static_cast<size_t>(warp) * 4 * p.C;
     for (long long m0 = (static_cast<long long>(blockIdx.x) * 8 + warp) * 4; m0 < p.M;
          m0 += static_cast<long long>(gridDim.x) * 32) {
         const int np = static_cast<int>(min(4LL, p.M - m0));
-        for (int i = lane; i < 4 * p.C; i += 32) {
-            const int q = i / p.C;
-            yw[i] = q < np ? ElemTraits<T>::to_float(y[(m0 + q) * p.C + (i - q * p.C)]) : 0.f;
-        }
-        __syncwarp();
+        const T* yr = y + m0 * p.C;
         for (int o = 0; o < p.NO; ++o) {
             const T* wr = w + static_cast<size_t>(o) * p.C;
             float a[4] = {0.f, 0.f, 0.f, 0.f};
             for (int c = lane; c < p.C; c += 32) {
                 const float wv = ElemTraits<T>::to_float(__ldg(wr + c));
 #pragma unroll
-                for (int q = 0; q < 4; ++q) a[q] = fmaf(wv, yw[q * p.C + c], a[q]);
+                for (int q = 0; q < 4; ++q)
+                    if (q < np) a[q] = fmaf(wv, ElemTraits<T>::to_float(__ldg(yr + static_cast<size_t>(q) * p.C + c)), a[q]);
             }
 #pragma unroll
             for (int q = 0; q < 4; ++q)
                 for (int off = 16; off > 0; off >>= 1) a[q] += __shfl_xor_sync(0xffffffffu, a[q], off);
             if (lane < np) {
-                float acc = (lane == 0 ? a[0] : lane == 1 ? a[1] : lane == 2 ? a[2] : a[3]) + (bias ? bias[o] : 0.f);
+                const float acc = (lane == 0 ? a[0] : lane == 1 ? a[1] : lane == 2 ? a[2] : a[3]) + (bias ? bias[o] : 0.f);
                 T r;
                 if constexpr (sizeof(T) == 4) r = acc;
                 else r = from_float<T>(acc);
                 rec[static_cast<size_t>(m0 + lane) * p.NO + pred_dest(o, p.G, p.P)] = r;
             }
         }
-        __syncwarp();
     }
 }
 

@@ -61,6 +61,7 @@ CASES = [
     (500, 48, 2, 3, False, True),       # C not a multiple of 64: CUDA-core kernel
     (333, 64, 16, 3, False, True),      # 432 channels: CUDA-core kernel
     (1, 64, 4, 3, False, True),         # one pixel
+    (40, 2048, 1, 1, False, True),      # 32 k-blocks do not fit shared memory: CUDA-core kernel
 ]
 
 
