@@ -16,20 +16,24 @@ int launch_predictor(const void* y, const void* w, const float* bias, void* rec,
             p.NP = (p.NO + 15) / 16 * 16;
             p.kblocks = p.C / 64;
             p.tiles = (p.M + 127) / 128;
+            // two accumulator buffers: the MMA runs one tile ahead of the epilogue (a third measured slower)
             unsigned cols = 32;
             while (cols < 2u * static_cast<unsigned>(p.NP)) cols <<= 1;
             p.tmem_cols = cols;
             p.a_fmt = std::is_same<T, __half>::value ? 0 : 1;
             const size_t b_bytes = static_cast<size_t>(p.kblocks) * p.NP * 128;
             const size_t a_stage = static_cast<size_t>(p.kblocks) * 128 * 128;
-            const size_t meta = static_cast<size_t>(p.NO) * 8 + 8 + 8 * 16 + 16;
+            constexpr int kMaxStages = 8;
+            const size_t meta = static_cast<size_t>(p.NO) * 8 + 8 + 8 * (2 * kMaxStages + 1 + 2 * 2) + 16;
             // two output staging buffers (store of tile i overlaps the epilogue of tile i+1) when they fit
             size_t o_bytes = 0, fixed = 0;
             int stages = 0;
             for (int ob = 2; ob >= 1 && stages < 2; --ob) {
                 o_bytes = (static_cast<size_t>(ob) * 128 * p.NO * E + 15) / 16 * 16;
                 fixed = 1024 + b_bytes + o_bytes + meta;
+                // 4 activation stages (6 and 8 measured no faster); DCNV4_PRED_STAGES overrides, up to 8
                 stages = 4;
+                if (const char* e = std::getenv("DCNV4_PRED_STAGES")) stages = std::min(kMaxStages, std::max(2, std::atoi(e)));
                 while (stages >= 2 && fixed + stages * a_stage > kTileSmemLimit) --stages;
                 p.out_bufs = ob;
             }

@@ -17,17 +17,20 @@ TOL = {"f32": 1e-5, "f16": 4e-3, "bf16": 4e-3}
 TD = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}
 
 
-@pytest.fixture(params=["auto", "epi8", "plain"])
+@pytest.fixture(params=["auto", "epi8", "stages8", "plain"])
 def pred_variant(request, monkeypatch):
     """The default choice (tensor cores where the shape allows, 16 epilogue
-    warps), the tensor-core kernel with 8 epilogue warps (DCNV4_PRED_EPI=8), and
-    the CUDA-core kernel forced with DCNV4_PRED_VARIANT=plain."""
-    monkeypatch.delenv("DCNV4_PRED_VARIANT", raising=False)
-    monkeypatch.delenv("DCNV4_PRED_EPI", raising=False)
+    warps, 4 stages), the tensor-core kernel with 8 epilogue warps, with an
+    8-deep activation ring, and the CUDA-core kernel forced with
+    DCNV4_PRED_VARIANT=plain."""
+    for v in ("DCNV4_PRED_VARIANT", "DCNV4_PRED_EPI", "DCNV4_PRED_STAGES"):
+        monkeypatch.delenv(v, raising=False)
     if request.param == "plain":
         monkeypatch.setenv("DCNV4_PRED_VARIANT", "plain")
     elif request.param == "epi8":
         monkeypatch.setenv("DCNV4_PRED_EPI", "8")
+    elif request.param == "stages8":   # an 8-deep activation ring where it fits
+        monkeypatch.setenv("DCNV4_PRED_STAGES", "8")
     return request.param
 
 
