@@ -59,6 +59,8 @@ def _load():
         lib.oracle_dcnv4_backward.restype = i
         lib.oracle_dcnv4_forward_variants.argtypes = [p] * 4 + [i] * 9 + [f, i, i, i]
         lib.oracle_dcnv4_forward_variants.restype = i
+        lib.oracle_dcnv4_backward_variants.argtypes = [p] * 7 + [i] * 9 + [f, i, i, i]
+        lib.oracle_dcnv4_backward_variants.restype = i
         lib.oracle_dcnv4_predictor.argtypes = [p] * 4 + [i] * 4
         lib.oracle_dcnv4_predictor.restype = i
         _lib = lib
@@ -139,6 +141,33 @@ def dcnv4_forward_variants(x, offset_mask, G: int, K: int, stride: int = 1, pad:
     if rc != 0:
         raise ValueError("oracle rejected the arguments")
     return out
+
+
+def dcnv4_backward_variants(x, offset_mask, grad_out, G: int, K: int, stride: int = 1, pad: int = 0,
+                            dilation: int = 1, offset_scale: float = 1.0, softmax: bool = False,
+                            remove_center: bool = False, center_logit=None):
+    """fp64 backward of ``dcnv4_forward_variants``: returns (grad_x, grad_offset_mask, grad_center_logit),
+    the last None without centre scaling."""
+    x = _f64(x)
+    om = _f64(offset_mask)
+    go = _f64(grad_out)
+    N, H, W, C = x.shape
+    Hout, Wout = output_size(H, K, stride, pad, dilation), output_size(W, K, stride, pad, dilation)
+    P = K * K - (1 if remove_center else 0)
+    if om.shape != (N, Hout, Wout, G, 3 * P) or go.shape != (N, Hout, Wout, C):
+        raise ValueError("offset_mask / grad_out shapes do not match x")
+    z = None if center_logit is None else _f64(center_logit)
+    gx = np.zeros_like(x)
+    gom = np.zeros_like(om)
+    gz = None if z is None else np.zeros_like(z)
+    if N:
+        rc = _load().oracle_dcnv4_backward_variants(_ptr(x), _ptr(om), None if z is None else _ptr(z), _ptr(go),
+                                                    _ptr(gx), _ptr(gom), None if gz is None else _ptr(gz),
+                                                    N, H, W, C, G, K, stride, pad, dilation, float(offset_scale),
+                                                    int(bool(softmax)), int(bool(remove_center)), int(z is not None))
+        if rc != 0:
+            raise ValueError("oracle rejected the arguments")
+    return gx, gom, gz
 
 
 def dcnv4_predictor(y, weight, bias, G: int, P: int) -> np.ndarray:

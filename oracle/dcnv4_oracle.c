@@ -396,3 +396,109 @@ int oracle_dcnv4_backward(const double *x, const double *om, const double *grad_
                 }
     return 0;
 }
+
+/* ------------------------------------------------------------------------
+ * Backward of oracle_dcnv4_forward_variants (same readings). With
+ * m' the (optionally softmax-normalised) masks, s = sigmoid(z) the centre
+ * gate (s = 0 without centre scaling) and g = dL/dout:
+ *   the aggregation sees g' = (1 - s) g, so grad_x, the offset gradients and
+ *   dL/dm'_j = (1 - s) u_j with u_j = sum_c g[c] S_j[c] are those of the plain
+ *   backward with masks m' and upstream g';
+ *   softmax: dL/dm_j = m'_j (dL/dm'_j - sum_i m'_i dL/dm'_i);
+ *   centre scaling: grad_x[centre] += s g and
+ *   dL/dz = s (1 - s) (sum_c g[c] x_c[c] - sum_j m'_j u_j).
+ * grad_z: [N,Hout,Wout,G] (written only with center_scale).
+ * ------------------------------------------------------------------------ */
+int oracle_dcnv4_backward_variants(const double *x, const double *om, const double *center_logit,
+                                   const double *grad_out, double *grad_x, double *grad_om, double *grad_z,
+                                   int N, int H, int W, int C, int G, int K,
+                                   int stride, int pad, int dilation, float offset_scale,
+                                   int softmax, int remove_center, int center_scale)
+{
+    if (N < 0 || H <= 0 || W <= 0 || C <= 0 || G <= 0 || K <= 0 || K > 16 || C % G) return -1;
+    if (remove_center && (K % 2 == 0 || K < 3)) return -1;
+    if (center_scale && (!center_logit || !grad_z)) return -1;
+    const int Hout = oracle_output_size(H, K, stride, pad, dilation);
+    const int Wout = oracle_output_size(W, K, stride, pad, dilation);
+    if (Hout <= 0 || Wout <= 0) return -1;
+    const int Cg = C / G, KK = K * K;
+    const int centre = (KK - 1) / 2;
+    const int P = remove_center ? KK - 1 : KK;
+    double mk[256], u[256];
+    for (size_t i = 0; i < (size_t)N * H * W * C; ++i) grad_x[i] = 0.0;
+    for (int n = 0; n < N; ++n)
+        for (int ho = 0; ho < Hout; ++ho)
+            for (int wo = 0; wo < Wout; ++wo)
+                for (int g = 0; g < G; ++g) {
+                    const size_t unit = (((size_t)n * Hout + ho) * Wout + wo) * G + g;
+                    const double *r = om + unit * (size_t)(3 * P);
+                    double *gr = grad_om + unit * (size_t)(3 * P);
+                    const double *go = grad_out + (((size_t)n * Hout + ho) * Wout + wo) * (size_t)C + (size_t)g * Cg;
+                    if (softmax) {
+                        double mx = r[2 * P];
+                        for (int j = 1; j < P; ++j)
+                            if (r[2 * P + j] > mx) mx = r[2 * P + j];
+                        double sum = 0.0;
+                        for (int j = 0; j < P; ++j) sum += exp(r[2 * P + j] - mx);
+                        for (int j = 0; j < P; ++j) mk[j] = exp(r[2 * P + j] - mx) / sum;
+                    } else {
+                        for (int j = 0; j < P; ++j) mk[j] = r[2 * P + j];
+                    }
+                    const double sg = center_scale ? 1.0 / (1.0 + exp(-center_logit[unit])) : 0.0;
+                    for (int j = 0; j < P; ++j) {
+                        const int k = (remove_center && j >= centre) ? j + 1 : j;
+                        const int ky = k / K, kx = k % K;
+                        const int p0y = ho * stride - pad + ky * dilation;
+                        const int p0x = wo * stride - pad + kx * dilation;
+                        const double dx = scaled_offset(offset_scale, r[j]);
+                        const double dy = scaled_offset(offset_scale, r[P + j]);
+                        double uj = 0.0, g_fx = 0.0, g_fy = 0.0;
+                        if (isfinite(dx) && isfinite(dy)) {
+                            const double fy0 = floor(dy), fx0 = floor(dx);
+                            const double ly = dy - fy0, lx = dx - fx0;
+                            const double y0 = (double)p0y + fy0, x0 = (double)p0x + fx0;
+                            for (int a = 0; a <= 1; ++a)
+                                for (int b = 0; b <= 1; ++b) {
+                                    const double yy = y0 + a, xx = x0 + b;
+                                    if (!(yy >= 0.0 && yy <= (double)(H - 1) && xx >= 0.0 && xx <= (double)(W - 1)))
+                                        continue;
+                                    const double wy = a ? ly : 1.0 - ly, wx = b ? lx : 1.0 - lx;
+                                    const double dwy = a ? 1.0 : -1.0, dwx = b ? 1.0 : -1.0;
+                                    const size_t pix = (((size_t)n * H + (size_t)yy) * W + (size_t)xx) * C + (size_t)g * Cg;
+                                    for (int c = 0; c < Cg; ++c) {
+                                        const double xv = x[pix + c];
+                                        uj += go[c] * wy * wx * xv;
+                                        g_fy += go[c] * dwy * wx * xv;
+                                        g_fx += go[c] * wy * dwx * xv;
+                                        grad_x[pix + c] += mk[j] * wy * wx * (1.0 - sg) * go[c];
+                                    }
+                                }
+                        }
+                        u[j] = uj;
+                        gr[j] = mk[j] * (double)offset_scale * (1.0 - sg) * g_fx;
+                        gr[P + j] = mk[j] * (double)offset_scale * (1.0 - sg) * g_fy;
+                        gr[2 * P + j] = (1.0 - sg) * uj;      /* dL/dm'_j */
+                    }
+                    if (softmax) {
+                        double dot = 0.0;
+                        for (int j = 0; j < P; ++j) dot += mk[j] * gr[2 * P + j];
+                        for (int j = 0; j < P; ++j) gr[2 * P + j] = mk[j] * (gr[2 * P + j] - dot);
+                    }
+                    if (center_scale) {
+                        const int cy = ho * stride - pad + (K / 2) * dilation;
+                        const int cx = wo * stride - pad + (K / 2) * dilation;
+                        double gxc = 0.0;
+                        if (cy >= 0 && cy < H && cx >= 0 && cx < W) {
+                            const size_t pix = (((size_t)n * H + (size_t)cy) * W + (size_t)cx) * C + (size_t)g * Cg;
+                            for (int c = 0; c < Cg; ++c) {
+                                gxc += go[c] * x[pix + c];
+                                grad_x[pix + c] += sg * go[c];
+                            }
+                        }
+                        double mu = 0.0;
+                        for (int j = 0; j < P; ++j) mu += mk[j] * u[j];
+                        grad_z[unit] = sg * (1.0 - sg) * (gxc - mu);
+                    }
+                }
+    return 0;
+}
