@@ -269,29 +269,43 @@ def run_backward(args, w, dev, world, rank, barrier, max_over_ranks):
     import deformable_convolution_sparse_b200 as dcn
     from deformable_convolution_sparse_b200.workloads import workload_grad_out, workload_inputs
 
+    from deformable_convolution_sparse_b200.workloads import make_center_logit, make_inputs
+
+    flags = VARIANT_FLAGS.get(args.variant, 0)
+    P = w.K * w.K - (1 if flags & 2 else 0)
     wr = w.with_(seed=w.seed + 1000 * rank)
-    x, om = workload_inputs(wr)
+    x, om = make_inputs(w.N, w.H, w.W, w.C, w.G, w.K, w.Hout, w.Wout, w.dtype, w.offsets, w.masks, seed=wr.seed,
+                        points=P)
     go = workload_grad_out(wr)
+    z = make_center_logit(w.N, w.Hout, w.Wout, w.G, w.dtype, seed=wr.seed)
     lib = dcn.load_library()
     dtype_code = dcn.binding.TORCH_DTYPE[x.dtype]
     e = x.element_size()
-    nx, nom, nout = x.numel(), om.numel(), go.numel()
-    # algorithmic bytes: x, offset_mask and grad_out read once; grad_x and grad_offset_mask (fp32) written once
-    foot = (nx + nom + nout) * e + (nx + nom) * 4
+    nx, nom, nout, nz = x.numel(), om.numel(), go.numel(), (z.numel() if flags & 4 else 0)
+    # algorithmic bytes: x, offset_mask, grad_out (and the gate logits) read once; grad_x, grad_offset_mask
+    # (and the gate gradient) written once in fp32
+    foot = (nx + nom + nout + nz) * e + (nx + nom + nz) * 4
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     copies = max(3, math.ceil(3 * l2 / foot))
     sets = [(x.to(dev), om.to(dev), go.to(dev), torch.empty(x.shape, dtype=torch.float32, device=dev),
              torch.empty(om.shape, dtype=torch.float32, device=dev)) for _ in range(copies)]
+    zd = z.to(dev)
+    gzd = torch.empty(z.shape, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
     sh = stream.cuda_stream
     launches = [0]
 
     def call(xd, omd, god, gxd, gomd):
-        rc = lib.dcnv4_backward(xd.data_ptr(), omd.data_ptr(), god.data_ptr(), gxd.data_ptr(), gomd.data_ptr(),
-                                w.N, w.H, w.W, w.C, w.G, w.K, w.stride, w.pad, w.dilation, w.offset_scale,
-                                dtype_code, sh)
+        if flags:
+            rc = lib.dcnv4_backward_ex(xd.data_ptr(), omd.data_ptr(), zd.data_ptr(), god.data_ptr(), gxd.data_ptr(),
+                                       gomd.data_ptr(), gzd.data_ptr(), w.N, w.H, w.W, w.C, w.G, w.K, w.stride,
+                                       w.pad, w.dilation, w.offset_scale, dtype_code, flags, sh)
+        else:
+            rc = lib.dcnv4_backward(xd.data_ptr(), omd.data_ptr(), god.data_ptr(), gxd.data_ptr(), gomd.data_ptr(),
+                                    w.N, w.H, w.W, w.C, w.G, w.K, w.stride, w.pad, w.dilation, w.offset_scale,
+                                    dtype_code, sh)
         if rc != 0:
-            raise dcn.DCNv4Error(rc, "dcnv4_backward")
+            raise dcn.DCNv4Error(rc, "dcnv4_backward_ex" if flags else "dcnv4_backward")
 
     def step(i):
         call(*sets[i % copies])
@@ -299,7 +313,8 @@ def run_backward(args, w, dev, world, rank, barrier, max_over_ranks):
 
     ms, sampler, timed_launches = time_steps(step, launches, args, dev, stream, barrier, max_over_ranks)
     ms_step = ms / args.steps
-    value = w.points * world * args.steps / (ms / 1e3) / 1e9
+    points = w.N * w.Hout * w.Wout * w.G * P
+    value = points * world * args.steps / (ms / 1e3) / 1e9
     peak, peak_kind = measured_peaks()
     achieved = foot / (ms_step / 1e3) / 1e9
     traffic, traffic_src = profiled_traffic(w.name, "backward")
@@ -331,23 +346,24 @@ def run_backward(args, w, dev, world, rank, barrier, max_over_ranks):
     torch.cuda.synchronize(dev)
     barrier()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1))
-    e2e_value = w.points * world * args.e2e_steps / (e2e_ms / 1e3) / 1e9
+    e2e_value = points * world * args.e2e_steps / (e2e_ms / 1e3) / 1e9
     if not torch.equal(gomh, gomd.cpu()):
         raise SystemExit("end-to-end gradient record differs from the device-resident one")
 
     base = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not flags:
         base = cpu_baseline_backward(w, x, om, go)
     if rank == 0:
         line = {
             "metric": METRIC_BWD, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f32", "data": "synthetic", "pass": "backward",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic", "pass": "backward", "variant": args.variant,
             "config": {
-                "workload": f"{w.name} backward: N={w.N} per GPU, H=W={w.H}, C={w.C}, G={w.G} (C/G={w.Cg}), "
-                            f"K={w.K}, stride={w.stride}, pad={w.pad}, dilation={w.dilation}; fp32 gradients",
+                "workload": f"{w.name} backward, variant {args.variant}: N={w.N} per GPU, H=W={w.H}, C={w.C}, "
+                            f"G={w.G} (C/G={w.Cg}), K={w.K}, {P} points per unit, stride={w.stride}, pad={w.pad}, "
+                            f"dilation={w.dilation}; fp32 gradients",
                 "storage_dtype": w.dtype, "accumulate": "f32", "global_batch": w.N * world,
-                "points_per_step_per_gpu": w.points, "parallelism": f"dp{world} (independent batches)",
+                "points_per_step_per_gpu": points, "parallelism": f"dp{world} (independent batches)",
                 "l2": f"steps rotate over {copies} resident sets, {copies * foot / 1e6:.0f} MB in total vs "
                       f"{l2 / 1e6:.0f} MB L2",
                 "inputs": "seeded synthetic: x~N(0,1), offsets and masks as the forward, grad_out~N(0,1)",

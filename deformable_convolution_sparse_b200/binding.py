@@ -31,7 +31,7 @@ TORCH_DTYPE = {torch.float32: DCNV4_F32, torch.float16: DCNV4_F16, torch.bfloat1
 
 # every symbol include/dcnv4.h declares
 EXPORTS = ("dcnv4_output_shape", "dcnv4_validate", "dcnv4_validate_ex", "dcnv4_forward", "dcnv4_forward_ex",
-           "dcnv4_backward", "dcnv4_predictor", "dcnv4_sampling_index",
+           "dcnv4_backward", "dcnv4_backward_ex", "dcnv4_predictor", "dcnv4_sampling_index",
            "dcnv4_forward_host", "dcnv4_forward_host_noalloc", "dcnv4_device_status", "dcnv4_selftest_wait_timeout", "dcnv4_strerror",
            "dcnv4_abi_version")
 DEVSTATUS_COPY_TIMEOUT, DEVSTATUS_SELFTEST_TIMEOUT = 1, 2
@@ -70,6 +70,8 @@ def load_library():
     lib.dcnv4_predictor.argtypes = [p] * 4 + [i] * 4 + [ctypes.c_uint, i, p]
     lib.dcnv4_predictor.restype = i
     lib.dcnv4_backward.argtypes = [p] * 5 + [i] * 9 + [f, i, p]
+    lib.dcnv4_backward_ex.argtypes = [p] * 7 + [i] * 9 + [f, i, ctypes.c_uint, p]
+    lib.dcnv4_backward_ex.restype = i
     lib.dcnv4_backward.restype = i
     lib.dcnv4_sampling_index.argtypes = [p, p, p] + [i] * 8 + [f, i, p]
     lib.dcnv4_sampling_index.restype = i
@@ -205,13 +207,15 @@ def forward(x: torch.Tensor, offset_mask: torch.Tensor, G: int, K: int, stride: 
 
 def backward(x: torch.Tensor, offset_mask: torch.Tensor, grad_out: torch.Tensor, G: int, K: int, stride: int = 1,
              pad: int = 0, dilation: int = 1, offset_scale: float = 1.0, grad_x: torch.Tensor | None = None,
-             grad_offset_mask: torch.Tensor | None = None, stream=None):
-    """DCNv4 backward on the GPU through ``dcnv4_backward``.
+             grad_offset_mask: torch.Tensor | None = None, stream=None, softmax: bool = False,
+             remove_center: bool = False, center_logit: torch.Tensor | None = None):
+    """DCNv4 backward on the GPU through ``dcnv4_backward`` / ``dcnv4_backward_ex``.
 
-    x: [N,H,W,C]; offset_mask: [N,Hout,Wout,G,3*K*K]; grad_out: [N,Hout,Wout,C],
-    all of one dtype. Returns (grad_x [N,H,W,C], grad_offset_mask
-    [N,Hout,Wout,G,3*K*K]), both fp32; the record layout of grad_offset_mask
-    is that of offset_mask. Asynchronous on ``stream`` (default: current).
+    x: [N,H,W,C]; offset_mask: [N,Hout,Wout,G,3*P]; grad_out: [N,Hout,Wout,C],
+    all of one dtype; the variant switches as in ``forward``. Returns
+    (grad_x [N,H,W,C], grad_offset_mask [N,Hout,Wout,G,3*P]), both fp32, plus
+    grad_center_logit [N,Hout,Wout,G] (fp32) as a third element when
+    ``center_logit`` is given. Asynchronous on ``stream`` (default: current).
     """
     for t, name in ((x, "x"), (offset_mask, "offset_mask"), (grad_out, "grad_out")):
         _check_tensor(t, name)
@@ -222,10 +226,20 @@ def backward(x: torch.Tensor, offset_mask: torch.Tensor, grad_out: torch.Tensor,
         raise ValueError("offset_mask and grad_out must match x in dtype and device")
     N, H, W, C = x.shape
     Hout, Wout = output_shape(H, W, K, stride, pad, dilation)
-    if tuple(offset_mask.shape) != (N, Hout, Wout, G, 3 * K * K):
-        raise ValueError(f"offset_mask shape {tuple(offset_mask.shape)} != {(N, Hout, Wout, G, 3 * K * K)}")
+    P = K * K - (1 if remove_center else 0)
+    if tuple(offset_mask.shape) != (N, Hout, Wout, G, 3 * P):
+        raise ValueError(f"offset_mask shape {tuple(offset_mask.shape)} != {(N, Hout, Wout, G, 3 * P)}")
     if tuple(grad_out.shape) != (N, Hout, Wout, C):
         raise ValueError(f"grad_out shape {tuple(grad_out.shape)} != {(N, Hout, Wout, C)}")
+    flags = (FLAG_SOFTMAX if softmax else 0) | (FLAG_REMOVE_CENTER if remove_center else 0)
+    gz = None
+    if center_logit is not None:
+        _check_tensor(center_logit, "center_logit")
+        if tuple(center_logit.shape) != (N, Hout, Wout, G) or center_logit.dtype != x.dtype or \
+                center_logit.device != x.device:
+            raise ValueError(f"center_logit must be [N,Hout,Wout,G] = {(N, Hout, Wout, G)} in x's dtype and device")
+        flags |= FLAG_CENTER_SCALE
+        gz = torch.empty((N, Hout, Wout, G), dtype=torch.float32, device=x.device)
     outs = []
     for t, shape, name in ((grad_x, x.shape, "grad_x"), (grad_offset_mask, offset_mask.shape, "grad_offset_mask")):
         if t is None:
@@ -237,12 +251,20 @@ def backward(x: torch.Tensor, offset_mask: torch.Tensor, grad_out: torch.Tensor,
         outs.append(t)
     gx, gom = outs
     with torch.cuda.device(x.device):
-        rc = load_library().dcnv4_backward(x.data_ptr(), offset_mask.data_ptr(), grad_out.data_ptr(), gx.data_ptr(),
-                                           gom.data_ptr(), N, H, W, C, G, K, stride, pad, dilation,
-                                           float(offset_scale), TORCH_DTYPE[x.dtype], _stream_handle(stream))
+        lib = load_library()
+        if flags:
+            rc = lib.dcnv4_backward_ex(x.data_ptr(), offset_mask.data_ptr(),
+                                       0 if center_logit is None else center_logit.data_ptr(), grad_out.data_ptr(),
+                                       gx.data_ptr(), gom.data_ptr(), 0 if gz is None else gz.data_ptr(),
+                                       N, H, W, C, G, K, stride, pad, dilation, float(offset_scale),
+                                       TORCH_DTYPE[x.dtype], flags, _stream_handle(stream))
+        else:
+            rc = lib.dcnv4_backward(x.data_ptr(), offset_mask.data_ptr(), grad_out.data_ptr(), gx.data_ptr(),
+                                    gom.data_ptr(), N, H, W, C, G, K, stride, pad, dilation, float(offset_scale),
+                                    TORCH_DTYPE[x.dtype], _stream_handle(stream))
     if rc != DCNV4_OK:
-        raise DCNv4Error(rc, "dcnv4_backward")
-    return gx, gom
+        raise DCNv4Error(rc, "dcnv4_backward_ex" if flags else "dcnv4_backward")
+    return (gx, gom) if gz is None else (gx, gom, gz)
 
 
 def predictor(y: torch.Tensor, weight: torch.Tensor, bias: torch.Tensor | None, G: int, K: int,

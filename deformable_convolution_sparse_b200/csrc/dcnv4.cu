@@ -176,35 +176,57 @@ int dcnv4_forward(const void* x, const void* offset_mask, void* out,
                             dtype, 0u, stream);
 }
 
+int dcnv4_backward_ex(const void* x, const void* offset_mask, const void* center_logit, const void* grad_out,
+                      float* grad_x, float* grad_offset_mask, float* grad_center_logit,
+                      int N, int H, int W, int C, int G, int K,
+                      int stride, int pad, int dilation, float offset_scale, int dtype, unsigned flags,
+                      void* stream) {
+    long long nx = 0, nout = 0, nom = 0;
+    int rc = check_sizes(N, H, W, C, G, K, stride, pad, dilation, offset_scale, dtype, &nx, &nout, &nom);
+    if (rc) return rc;
+    if (flags & ~static_cast<unsigned>(DCNV4_FLAG_SOFTMAX | DCNV4_FLAG_REMOVE_CENTER | DCNV4_FLAG_CENTER_SCALE))
+        return DCNV4_ERR_FLAGS;
+    if ((flags & DCNV4_FLAG_REMOVE_CENTER) && (K % 2 == 0 || K < 3)) return DCNV4_ERR_SHAPE;
+    nom = nom / (3LL * K * K) * 3LL * points_per_unit(K, flags);
+    const long long ngate = nout / C * G;
+    const bool cs = (flags & DCNV4_FLAG_CENTER_SCALE) != 0u;
+    if (N == 0) return DCNV4_OK;
+    if (!x || !offset_mask || !grad_out || !grad_x || !grad_offset_mask) return DCNV4_ERR_NULL;
+    if (cs && (!center_logit || !grad_center_logit)) return DCNV4_ERR_NULL;
+    const int e = elem_size(dtype);
+    if (!aligned(x, e) || !aligned(offset_mask, e) || !aligned(grad_out, e) || !aligned(grad_x, 4) ||
+        !aligned(grad_offset_mask, 4) || (cs && (!aligned(center_logit, e) || !aligned(grad_center_logit, 4))))
+        return DCNV4_ERR_ALIGN;
+    const void* inputs[4] = {x, offset_mask, grad_out, cs ? center_logit : nullptr};
+    const long long in_bytes[4] = {nx * e, nom * e, nout * e, cs ? ngate * e : 0};
+    for (int i = 0; i < 4; ++i)
+        if (overlap(grad_x, nx * 4, inputs[i], in_bytes[i]) || overlap(grad_offset_mask, nom * 4, inputs[i], in_bytes[i]) ||
+            (cs && overlap(grad_center_logit, ngate * 4, inputs[i], in_bytes[i])))
+            return DCNV4_ERR_ALIAS;
+    if (overlap(grad_x, nx * 4, grad_offset_mask, nom * 4) ||
+        (cs && (overlap(grad_center_logit, ngate * 4, grad_x, nx * 4) ||
+                overlap(grad_center_logit, ngate * 4, grad_offset_mask, nom * 4))))
+        return DCNV4_ERR_ALIAS;
+    int Hout = 0, Wout = 0;
+    dcnv4_output_shape(H, W, K, stride, pad, dilation, &Hout, &Wout);
+    const FwdParams p = make_params(N, H, W, C, G, K, stride, pad, dilation, offset_scale, Hout, Wout, flags,
+                                    cs ? center_logit : nullptr);
+    float* gz = cs ? grad_center_logit : nullptr;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    switch (dtype) {
+        case DCNV4_F32: return launch_backward<float>(x, offset_mask, grad_out, grad_x, grad_offset_mask, gz, p, s);
+        case DCNV4_F16: return launch_backward<__half>(x, offset_mask, grad_out, grad_x, grad_offset_mask, gz, p, s);
+        default: return launch_backward<__nv_bfloat16>(x, offset_mask, grad_out, grad_x, grad_offset_mask, gz, p, s);
+    }
+}
+
 int dcnv4_backward(const void* x, const void* offset_mask, const void* grad_out,
                    float* grad_x, float* grad_offset_mask,
                    int N, int H, int W, int C, int G, int K,
                    int stride, int pad, int dilation, float offset_scale, int dtype,
                    void* stream) {
-    long long nx = 0, nout = 0, nom = 0;
-    int rc = check_sizes(N, H, W, C, G, K, stride, pad, dilation, offset_scale, dtype, &nx, &nout, &nom);
-    if (rc) return rc;
-    if (N == 0) return DCNV4_OK;
-    if (!x || !offset_mask || !grad_out || !grad_x || !grad_offset_mask) return DCNV4_ERR_NULL;
-    const int e = elem_size(dtype);
-    if (!aligned(x, e) || !aligned(offset_mask, e) || !aligned(grad_out, e) || !aligned(grad_x, 4) ||
-        !aligned(grad_offset_mask, 4))
-        return DCNV4_ERR_ALIGN;
-    const void* inputs[3] = {x, offset_mask, grad_out};
-    const long long in_bytes[3] = {nx * e, nom * e, nout * e};
-    for (int i = 0; i < 3; ++i)
-        if (overlap(grad_x, nx * 4, inputs[i], in_bytes[i]) || overlap(grad_offset_mask, nom * 4, inputs[i], in_bytes[i]))
-            return DCNV4_ERR_ALIAS;
-    if (overlap(grad_x, nx * 4, grad_offset_mask, nom * 4)) return DCNV4_ERR_ALIAS;
-    int Hout = 0, Wout = 0;
-    dcnv4_output_shape(H, W, K, stride, pad, dilation, &Hout, &Wout);
-    const FwdParams p = make_params(N, H, W, C, G, K, stride, pad, dilation, offset_scale, Hout, Wout);
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    switch (dtype) {
-        case DCNV4_F32: return launch_backward<float>(x, offset_mask, grad_out, grad_x, grad_offset_mask, p, s);
-        case DCNV4_F16: return launch_backward<__half>(x, offset_mask, grad_out, grad_x, grad_offset_mask, p, s);
-        default: return launch_backward<__nv_bfloat16>(x, offset_mask, grad_out, grad_x, grad_offset_mask, p, s);
-    }
+    return dcnv4_backward_ex(x, offset_mask, nullptr, grad_out, grad_x, grad_offset_mask, nullptr, N, H, W, C, G, K,
+                             stride, pad, dilation, offset_scale, dtype, 0u, stream);
 }
 
 int dcnv4_predictor(const void* y, const void* weight, const float* bias, void* offset_mask,

@@ -82,14 +82,24 @@ __device__ __forceinline__ void scatter_add(float* dst, float a, const float (&v
 // grad_om is overwritten. Shared memory: the block's records (T, staged at
 // their 16-byte phase plus 16 bytes) followed, 16-byte aligned, by the block's
 // fp32 gradient records.
-template <typename T, int CPL, int KS>
+//
+// VF: the variant flags of p may be set (softmax over the masks, centre point
+// removed, centre feature scaling); false compiles them out. With them, the
+// aggregation part is the plain backward with masks m' (softmax-normalised or
+// raw) and upstream (1 - s) dL/dout, s the centre gate; then the softmax's
+// Jacobian maps dL/dm' to dL/dm, and centre scaling adds s dL/dout at the
+// centre pixel of grad_x and writes dL/dz = s (1 - s) (sum_c g x_c -
+// sum_j m'_j u_j), u_j = sum_c g S_j, to grad_z.
+template <typename T, int CPL, int KS, bool VF>
 __global__ void __launch_bounds__(256)
 bwd_kernel(const T* __restrict__ x, const T* __restrict__ om, const T* __restrict__ go,
-           float* __restrict__ grad_x, float* __restrict__ grad_om, FwdParams p) {
+           float* __restrict__ grad_x, float* __restrict__ grad_om, float* __restrict__ grad_z, FwdParams p) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const int K = KS > 0 ? KS : p.K;
     const int KK = K * K;
-    const int R = 3 * KK;
+    const int NP = VF ? p.npts : KK;   // points per unit
+    const int kcs = VF ? p.kc : KK;    // grid index left out (none: KK)
+    const int R = 3 * NP;
 
     const int unit0 = blockIdx.x * p.units_per_block;
     const int nunits = min(p.units_per_block, p.units - unit0);
@@ -109,15 +119,23 @@ bwd_kernel(const T* __restrict__ x, const T* __restrict__ om, const T* __restric
     const T* ximg = x + static_cast<size_t>(n) * p.H * rowC;
     float* gimg = grad_x + static_cast<size_t>(n) * p.H * rowC;
     const T* gop = go + (static_cast<size_t>((n * p.Hout + ho) * p.Wout + wo)) * p.C + g * p.Cg;
+    const size_t unit = static_cast<size_t>(unit0 + (active ? lu : 0));
+    const MaskNorm mn = VF ? mask_norm(rec + 2 * NP, NP, p.flags) : MaskNorm{0.f, 1.f, false};
+    const bool cs = VF && (p.flags & kFlagCenterScale);
+    const float sg = cs ? center_gate<T>(p, unit) : 0.f;   // centre gate s
+    const float keep = 1.f - sg;                            // the aggregation's share of dL/dout
+    float mu = 0.f;                                         // sum_j m'_j u_j (centre scaling)
 
 #pragma unroll (KS > 0 ? KS * KS : 1)
     for (int k = 0; k < KK; ++k) {
+        if (k == kcs) continue;
+        const int jp = k - (k > kcs ? 1 : 0);  // point index in the record
         const int ky = k / K, kx = k - (k / K) * K;
         const int p0y = ho * p.stride - p.pad + ky * p.dilation;
         const int p0x = wo * p.stride - p.pad + kx * p.dilation;
-        const float rx = ElemTraits<T>::to_float(rec[k]);
-        const float ry = ElemTraits<T>::to_float(rec[KK + k]);
-        const float m = ElemTraits<T>::to_float(rec[2 * KK + k]);
+        const float rx = ElemTraits<T>::to_float(rec[jp]);
+        const float ry = ElemTraits<T>::to_float(rec[NP + jp]);
+        const float m = mask_value(ElemTraits<T>::to_float(rec[2 * NP + jp]), mn);
         Sample s = locate(p0y, p0x, ry, rx, p.offset_scale, p.H, p.W);
         if (!active) s.bits = 0u;
 
@@ -125,7 +143,8 @@ bwd_kernel(const T* __restrict__ x, const T* __restrict__ om, const T* __restric
         if (s.bits) {
             const float ly = s.ly, lx = s.lx;
             // mask times the corner weights, for the scatter into grad_x
-            const float a1 = m * ly, a0 = m - a1;
+            const float ms = VF ? m * keep : m;
+            const float a1 = ms * ly, a0 = ms - a1;
             const float w01 = a0 * lx, w00 = a0 - w01, w11 = a1 * lx, w10 = a1 - w11;
             const float wc[4] = {w00, w01, w10, w11};
             const size_t c00 = static_cast<size_t>(s.y0 * p.W + s.x0) * p.C;
@@ -168,10 +187,42 @@ bwd_kernel(const T* __restrict__ x, const T* __restrict__ om, const T* __restric
             gfy += __shfl_xor_sync(0xffffffffu, gfy, o);
         }
         if (active && part == 0) {
-            const float ms = m * p.offset_scale;
-            gbuf[lu * R + k] = ms * gfx;
-            gbuf[lu * R + KK + k] = ms * gfy;
-            gbuf[lu * R + 2 * KK + k] = gm;
+            const float ms = (VF ? m * keep : m) * p.offset_scale;
+            gbuf[lu * R + jp] = ms * gfx;
+            gbuf[lu * R + NP + jp] = ms * gfy;
+            gbuf[lu * R + 2 * NP + jp] = VF ? keep * gm : gm;   // dL/dm'
+            if (VF) mu = fmaf(m, gm, mu);
+        }
+    }
+    if constexpr (VF) {
+        if (active && part == 0 && mn.on) {
+            // softmax: dL/dm_j = m'_j (dL/dm'_j - sum_i m'_i dL/dm'_i)
+            float* gmrow = gbuf + lu * R + 2 * NP;
+            float dot = 0.f;
+            for (int j = 0; j < NP; ++j) dot = fmaf(mask_value(ElemTraits<T>::to_float(rec[2 * NP + j]), mn), gmrow[j], dot);
+            for (int j = 0; j < NP; ++j)
+                gmrow[j] = mask_value(ElemTraits<T>::to_float(rec[2 * NP + j]), mn) * (gmrow[j] - dot);
+        }
+        if (cs) {
+            // centre feature: grad_x[centre] += s g, and sum_c g x_c for the gate gradient
+            const int cy = ho * p.stride - p.pad + (K / 2) * p.dilation;
+            const int cx = wo * p.stride - p.pad + (K / 2) * p.dilation;
+            const bool inside = active && cy >= 0 && cy < p.H && cx >= 0 && cx < p.W;
+            float gxc = 0.f;
+            if (inside) {
+                const size_t cpix = static_cast<size_t>(cy * p.W + cx) * p.C;
+                for (int ch = part; ch < p.chunks; ch += p.lanes) {
+                    const int c0 = g * p.Cg + ch * CPL;
+                    float gv[CPL], xv[CPL];
+                    load_channels<T, CPL>(gop + ch * CPL, gv);
+                    load_channels<T, CPL>(ximg + cpix + c0, xv);
+#pragma unroll
+                    for (int q = 0; q < CPL; ++q) gxc = fmaf(gv[q], xv[q], gxc);
+                    scatter_add<CPL>(gimg + cpix + c0, sg, gv);
+                }
+            }
+            for (int o = p.lanes >> 1; o > 0; o >>= 1) gxc += __shfl_xor_sync(0xffffffffu, gxc, o);
+            if (active && part == 0) grad_z[unit] = sg * (1.f - sg) * (gxc - mu);
         }
     }
     __syncthreads();

@@ -4,7 +4,7 @@
 // gradient. Vector path (4 channels per thread, float4 reductions) when the
 // pointers and channel counts allow it, element path otherwise.
 template <typename T>
-int launch_backward(const void* x, const void* om, const void* go, float* gx, float* gom, FwdParams p,
+int launch_backward(const void* x, const void* om, const void* go, float* gx, float* gom, float* gz, FwdParams p,
                     cudaStream_t stream) {
     constexpr int E = sizeof(T);
     const bool vec = aligned(x, 4 * E) && aligned(go, 4 * E) && aligned(gx, 16) && p.C % 4 == 0 && p.Cg % 4 == 0;
@@ -14,7 +14,7 @@ int launch_backward(const void* x, const void* om, const void* go, float* gx, fl
     while (lanes < p.chunks && lanes < 32) lanes <<= 1;
     p.lanes = lanes;
     // units per block: full warps, records and fp32 gradient records in shared memory
-    const size_t R = static_cast<size_t>(3) * p.KK;
+    const size_t R = static_cast<size_t>(3) * p.npts;
     const int step = lanes < 32 ? 32 / lanes : 1;
     auto smem_for = [&](int upb) {
         return ((upb * R * E + 16 + 15) & ~static_cast<size_t>(15)) + upb * R * sizeof(float);
@@ -37,10 +37,14 @@ int launch_backward(const void* x, const void* om, const void* go, float* gx, fl
             cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
                 cudaSuccess)
             return DCNV4_ERR_LAUNCH;
-        kernel<<<static_cast<unsigned>(blocks), threads, smem, stream>>>(xt, omt, got, gx, gom, p);
+        kernel<<<static_cast<unsigned>(blocks), threads, smem, stream>>>(xt, omt, got, gx, gom, gz, p);
         return launch_status();
     };
     const bool k3 = p.K == 3;
-    if (vec) return k3 ? run(dcnv4::bwd_kernel<T, 4, 3>) : run(dcnv4::bwd_kernel<T, 4, 0>);
-    return k3 ? run(dcnv4::bwd_kernel<T, 1, 3>) : run(dcnv4::bwd_kernel<T, 1, 0>);
+    if (p.flags != 0) {  // the variants: their own instantiations, so that the plain backward carries none of it
+        if (vec) return k3 ? run(dcnv4::bwd_kernel<T, 4, 3, true>) : run(dcnv4::bwd_kernel<T, 4, 0, true>);
+        return k3 ? run(dcnv4::bwd_kernel<T, 1, 3, true>) : run(dcnv4::bwd_kernel<T, 1, 0, true>);
+    }
+    if (vec) return k3 ? run(dcnv4::bwd_kernel<T, 4, 3, false>) : run(dcnv4::bwd_kernel<T, 4, 0, false>);
+    return k3 ? run(dcnv4::bwd_kernel<T, 1, 3, false>) : run(dcnv4::bwd_kernel<T, 1, 0, false>);
 }

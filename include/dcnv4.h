@@ -228,6 +228,27 @@ DCNV4_API int dcnv4_backward(const void *x, const void *offset_mask, const void 
 DCNV4_API int dcnv4_predictor(const void *y, const void *weight, const float *bias, void *offset_mask,
                     int M, int C, int G, int K, unsigned int flags, int dtype, void *stream);
 
+/* dcnv4_backward for the variant flags of dcnv4_forward_ex (flags == 0 is
+ * dcnv4_backward). With m' the masks the aggregation used (softmax-normalised
+ * with DCNV4_FLAG_SOFTMAX) and s = sigmoid(center_logit) (0 without centre
+ * scaling), the aggregation's gradients are those of dcnv4_backward with
+ * masks m' and upstream (1 - s) * grad_out; the mask block of
+ * grad_offset_mask holds dL/dm, i.e. with the softmax's Jacobian applied:
+ * m'_j (dL/dm'_j - sum_i m'_i dL/dm'_i). With DCNV4_FLAG_CENTER_SCALE,
+ * grad_x additionally receives s * grad_out at the centre grid position
+ * (when inside the image) and grad_center_logit[n,ho,wo,g] (device fp32
+ * [N,Hout,Wout,G], fully overwritten) = s (1 - s) (sum_c grad_out * x_c -
+ * sum_j m'_j u_j), u_j = sum_c grad_out * S_j. Without the centre point the
+ * records have 3*(K*K-1) entries per group, as in dcnv4_forward_ex.
+ * center_logit and grad_center_logit are needed (non-NULL, aligned, not
+ * overlapping any other buffer) only with DCNV4_FLAG_CENTER_SCALE. Other
+ * checks, conventions and launch behaviour as dcnv4_backward. */
+DCNV4_API int dcnv4_backward_ex(const void *x, const void *offset_mask, const void *center_logit,
+                      const void *grad_out, float *grad_x, float *grad_offset_mask,
+                      float *grad_center_logit, int N, int H, int W, int C, int G, int K,
+                      int stride, int pad, int dilation, float offset_scale, int dtype,
+                      unsigned int flags, void *stream);
+
 /* The integer half of the forward, exposed so that it can be compared bit for
  * bit: for every sampling point (n, ho, wo, g, k) it writes the top-left
  * corner (y0, x0) into corner[2*p], corner[2*p+1] and a 4-bit mask of the

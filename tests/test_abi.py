@@ -221,3 +221,29 @@ def test_predictor_reports_each_error_class_before_any_cuda_call(kw, status):
 
 def test_predictor_empty_batch_touches_nothing():
     assert _pred(y=0, w=0, rec=0, M=0) == B.DCNV4_OK
+
+
+def _bwx(x=X, om=OM, z=0x60000000, go=OUT, gx=GX, gom=GOM, gz=0x70000000, flags=0, **kw):
+    a = dict(GOOD)
+    a.update(kw)
+    return B.load_library().dcnv4_backward_ex(x, om, z, go, gx, gom, gz, a["N"], a["H"], a["W"], a["C"], a["G"],
+                                              a["K"], a["stride"], a["pad"], a["dilation"], a["offset_scale"],
+                                              a["dtype"], flags, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(flags=8), "DCNV4_ERR_FLAGS"), (dict(flags=B.FLAG_REMOVE_CENTER, K=4, pad=1), "DCNV4_ERR_SHAPE"),
+    (dict(flags=B.FLAG_CENTER_SCALE, z=0), "DCNV4_ERR_NULL"), (dict(flags=B.FLAG_CENTER_SCALE, gz=0), "DCNV4_ERR_NULL"),
+    (dict(flags=B.FLAG_CENTER_SCALE, gz=0x70000002), "DCNV4_ERR_ALIGN"),
+    (dict(flags=B.FLAG_CENTER_SCALE, z=0x60000001), "DCNV4_ERR_ALIGN"),
+    (dict(flags=B.FLAG_CENTER_SCALE, gz=GX + 64), "DCNV4_ERR_ALIAS"),
+    (dict(flags=B.FLAG_CENTER_SCALE, gz=X), "DCNV4_ERR_ALIAS"),
+    (dict(flags=B.FLAG_CENTER_SCALE, gx=0x60000000), "DCNV4_ERR_ALIAS"),
+    (dict(gx=0), "DCNV4_ERR_NULL"), (dict(go=OUT + 1), "DCNV4_ERR_ALIGN"),
+])
+def test_backward_ex_reports_each_error_class_before_any_cuda_call(kw, status):
+    assert _bwx(**kw) == B.STATUS[status]
+
+
+def test_backward_ex_empty_batch_touches_nothing():
+    assert _bwx(x=0, om=0, z=0, go=0, gx=0, gom=0, gz=0, N=0, flags=7) == B.DCNV4_OK
