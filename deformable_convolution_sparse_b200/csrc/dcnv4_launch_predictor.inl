@@ -40,6 +40,9 @@ int launch_predictor(const void* y, const void* w, const float* bias, void* rec,
             tc = stages >= 2;
             if (tc) {
                 p.stages = stages;
+                // raw W in the staging area when it fits (DCNV4_PRED_WSTAGE=0 keeps it in the ring)
+                p.w_in_staging = b_bytes <= o_bytes ? 1 : 0;
+                if (const char* e = std::getenv("DCNV4_PRED_WSTAGE"); e && *e == '0') p.w_in_staging = 0;
                 p.smem_b = 0;
                 p.smem_a = static_cast<unsigned>(b_bytes);
                 p.smem_o = static_cast<unsigned>(b_bytes + stages * a_stage);

@@ -51,6 +51,7 @@ struct PredParams {
     unsigned tmem_cols;  // tensor-memory columns allocated (power of two >= 2*NP)
     int a_fmt;      // 0: fp16, 1: bf16 (instruction-descriptor format code)
     int out_bufs;   // output staging buffers (2, or 1 when two do not fit)
+    int w_in_staging;  // raw W fits the (still idle) output staging area: the activation loads start at once
     unsigned smem_b, smem_a, smem_o, smem_meta;  // byte offsets of the shared-memory regions
 };
 
@@ -209,15 +210,26 @@ predictor_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_const
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
-    // W, once per CTA: TMA into the (still unused) activation ring, then its rows
-    // copied into record order in bsm, so that accumulator column d is record
-    // slot d. Rows past NO are the TMA's zero fill. A 16-byte chunk j of row r
-    // sits at chunk j ^ (r mod 8) of the row (128-byte swizzle, 1024-byte atoms).
-    // Each "full" barrier completes on one arrival plus the bytes of its loads.
+    // W, once per CTA: TMA into an idle area (the output staging tiles when it
+    // fits there, else the activation ring), then its rows copied into record
+    // order in bsm, so that accumulator column d is record slot d. Rows past NO
+    // are the TMA's zero fill. A 16-byte chunk j of row r sits at chunk
+    // j ^ (r mod 8) of the row (128-byte swizzle, 1024-byte atoms). Each "full"
+    // barrier completes on one arrival plus the bytes of its loads. With W in
+    // the staging area the first activation tiles are requested at once too.
+    unsigned char* wraw = p.w_in_staging ? reinterpret_cast<unsigned char*>(osm) : asm_;
+    const int preissued = (p.w_in_staging && ntiles > 0) ? min(p.stages, ntiles) : 0;
     if (tid == 0 && ntiles > 0) {
         mbar_expect_tx(b_full, static_cast<unsigned>(p.kblocks) * b_kblock_bytes);
-        for (int kb = 0; kb < p.kblocks; ++kb) tma_load_2d(asm_ + kb * b_kblock_bytes, &bmap, kb * 64, 0, b_full);
+        for (int kb = 0; kb < p.kblocks; ++kb) tma_load_2d(wraw + kb * b_kblock_bytes, &bmap, kb * 64, 0, b_full);
         mbar_arrive(b_full);
+        for (int it = 0; it < preissued; ++it) {
+            const int tile = static_cast<int>(blockIdx.x) + it * static_cast<int>(gridDim.x);
+            mbar_expect_tx(&a_full[it], a_stage_bytes);
+            for (int kb = 0; kb < p.kblocks; ++kb)
+                tma_load_2d(asm_ + it * a_stage_bytes + kb * 16384u, &amap, kb * 64, tile * 128, &a_full[it]);
+            mbar_arrive(&a_full[it]);
+        }
     }
     const bool b_ok = __syncthreads_and(ntiles == 0 || mbar_wait_bounded(b_full, 0u, kCopyWaitLimitNs)) != 0;
     if (b_ok && ntiles > 0) {
@@ -225,7 +237,7 @@ predictor_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_const
         for (int i = tid; i < items; i += blockDim.x) {
             const int kb = i / (p.NP * 8), r = (i >> 3) % p.NP, j = i & 7;
             const int o = r < p.NO ? src[r] : r;
-            const unsigned char* from = asm_ + kb * b_kblock_bytes + (o >> 3) * 1024 + (o & 7) * 128 + ((j ^ (o & 7)) << 4);
+            const unsigned char* from = wraw + kb * b_kblock_bytes + (o >> 3) * 1024 + (o & 7) * 128 + ((j ^ (o & 7)) << 4);
             unsigned char* to = bsm + kb * b_kblock_bytes + (r >> 3) * 1024 + (r & 7) * 128 + ((j ^ (r & 7)) << 4);
             *reinterpret_cast<uint4*>(to) = *reinterpret_cast<const uint4*>(from);
         }
@@ -239,7 +251,7 @@ predictor_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_const
     } else if (warp == 0) {
         if (lane == 0 && ntiles > 0) {
             // -------------------------------------------------------- loads
-            for (int it = 0; it < ntiles; ++it) {
+            for (int it = preissued; it < ntiles; ++it) {
                 const int s = it % p.stages;
                 if (it >= p.stages &&
                     !mbar_wait_bounded(&a_empty[s], static_cast<unsigned>((it / p.stages) - 1) & 1u, kCopyWaitLimitNs)) {

@@ -17,18 +17,21 @@ TOL = {"f32": 1e-5, "f16": 4e-3, "bf16": 4e-3}
 TD = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}
 
 
-@pytest.fixture(params=["auto", "epi8", "stages8", "plain"])
+@pytest.fixture(params=["auto", "wring", "epi8", "stages8", "plain"])
 def pred_variant(request, monkeypatch):
     """The default choice (tensor cores where the shape allows, 16 epilogue
-    warps, 4 stages), the tensor-core kernel with 8 epilogue warps, with an
-    8-deep activation ring, and the CUDA-core kernel forced with
-    DCNV4_PRED_VARIANT=plain."""
-    for v in ("DCNV4_PRED_VARIANT", "DCNV4_PRED_EPI", "DCNV4_PRED_STAGES"):
+    warps, 4 stages, weights staged through the idle output area), the same
+    with the weights staged through the activation ring, with 8 epilogue
+    warps, with an 8-deep activation ring, and the CUDA-core kernel forced
+    with DCNV4_PRED_VARIANT=plain."""
+    for v in ("DCNV4_PRED_VARIANT", "DCNV4_PRED_EPI", "DCNV4_PRED_STAGES", "DCNV4_PRED_WSTAGE"):
         monkeypatch.delenv(v, raising=False)
     if request.param == "plain":
         monkeypatch.setenv("DCNV4_PRED_VARIANT", "plain")
     elif request.param == "epi8":
         monkeypatch.setenv("DCNV4_PRED_EPI", "8")
+    elif request.param == "wring":   # the weights staged through the activation ring
+        monkeypatch.setenv("DCNV4_PRED_WSTAGE", "0")
     elif request.param == "stages8":   # an 8-deep activation ring where it fits
         monkeypatch.setenv("DCNV4_PRED_STAGES", "8")
     return request.param
