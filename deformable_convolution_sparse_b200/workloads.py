@@ -159,3 +159,24 @@ def make_center_logit(N: int, Hout: int, Wout: int, G: int, dtype: str = "f32", 
     gen = torch.Generator(device="cpu")
     gen.manual_seed(2000 + int(seed))
     return _draw(gen, (N, Hout, Wout, G), dist).to(DTYPES[dtype]).contiguous()
+
+
+def make_inputs_on(device, N: int, H: int, W: int, C: int, G: int, K: int, Hout: int, Wout: int,
+                   dtype: str = "f16", offsets=("normal", 0.0, 1.0), masks=("normal", 0.0, 1.0), seed: int = 0):
+    """``make_inputs`` drawn directly on ``device`` (a seeded generator of that device) for batches too large
+    to draw on the host; the same draw order (x, offsets, masks), a different random stream."""
+    gen = torch.Generator(device=device)
+    gen.manual_seed(int(seed))
+
+    def draw(shape, dist):
+        kind, a, b = dist
+        if kind == "normal":
+            return torch.randn(shape, generator=gen, device=device) * float(b) + float(a)
+        return torch.rand(shape, generator=gen, device=device) * float(b - a) + float(a)
+
+    t = DTYPES[dtype]
+    x = draw((N, H, W, C), ("normal", 0.0, 1.0)).to(t)
+    om = torch.empty((N, Hout, Wout, G, 3 * K * K), dtype=t, device=device)
+    om[..., :2 * K * K] = draw((N, Hout, Wout, G, 2 * K * K), offsets).to(t)
+    om[..., 2 * K * K:] = draw((N, Hout, Wout, G, K * K), masks).to(t)
+    return x, om
