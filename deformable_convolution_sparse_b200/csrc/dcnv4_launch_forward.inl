@@ -15,7 +15,12 @@ Variant variant_from_env() {
     return Variant::Auto;
 }
 
-constexpr int kTileUnitsMax = 512;  // consumer threads (16 warps) per CTA, plus one producer warp
+// consumer threads (15 warps) per CTA, plus one producer warp: 16 warps, 4 per SM
+// sub-partition, whose 16 K registers then hold 4 warps at the kernel's 112-register cap
+// (a 17th warp would put 5 on one sub-partition: 17,920 registers, and the CTA would not launch)
+constexpr int kTileUnitsMax = 480;
+static_assert(((kTileUnitsMax / 32 + 1 + 3) / 4) * 112 * 32 <= 16384,
+              "the tile kernel's register cap must fit the warps of one SM sub-partition");
 
 struct TilePlan {
     dcnv4::TileParams p;
@@ -172,14 +177,35 @@ int launch_tile_q(const T* x, const T* om, T* out, const TilePlan& plan, cudaStr
     std::call_once(once, [&] {
         attr = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kTileSmemLimit));
     });
-    if (attr != cudaSuccess) return DCNV4_ERR_LAUNCH;
-    int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, plan.threads, plan.smem) != cudaSuccess || per_sm < 1)
+    const bool dbg = std::getenv("DCNV4_DEBUG") != nullptr;
+    if (attr != cudaSuccess) {
+        if (dbg) std::fprintf(stderr, "dcnv4 tile launch: shared-memory attribute: %s\n", cudaGetErrorString(attr));
         return DCNV4_ERR_LAUNCH;
+    }
+    int per_sm = 0;
+    const cudaError_t occ = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, plan.threads, plan.smem);
+    if (occ != cudaSuccess || per_sm < 1) {
+        if (dbg) std::fprintf(stderr, "dcnv4 tile launch: occupancy %d (%s) for %d threads, %zu bytes\n", per_sm,
+                              cudaGetErrorString(occ), plan.threads, plan.smem);
+        return DCNV4_ERR_LAUNCH;
+    }
     const long long slots = static_cast<long long>(sm_count()) * per_sm;
     const unsigned grid = static_cast<unsigned>(std::min<long long>(plan.p.tiles, slots));
-    kern<<<grid, plan.threads, plan.smem, stream>>>(plan.map, x, om, out, plan.p);
-    return launch_status();
+    // the last partial wave (tiles mod grid) is split by consumer warps over up to grid / L
+    // CTAs when at least two can share each tile (DCNV4_TAIL_SPLIT=0 turns it off)
+    dcnv4::TileParams p = plan.p;
+    const int L = static_cast<int>(p.tiles % static_cast<int>(grid));
+    const int consumer_warps = plan.threads / 32 - 1;
+    int split = 1;
+    if (L > 0 && static_cast<int>(grid) >= 2 * L) split = std::min(static_cast<int>(grid) / L, consumer_warps);
+    if (const char* e = std::getenv("DCNV4_TAIL_SPLIT"); e && *e == '0') split = 1;
+    p.tail_split = split;
+    p.main_tiles = split > 1 ? p.tiles - L : p.tiles;
+    p.items = p.main_tiles + (split > 1 ? L * split : 0);
+    kern<<<grid, plan.threads, plan.smem, stream>>>(plan.map, x, om, out, p);
+    const cudaError_t le = cudaGetLastError();
+    if (le != cudaSuccess && dbg) std::fprintf(stderr, "dcnv4 tile launch: %s\n", cudaGetErrorString(le));
+    return le == cudaSuccess ? DCNV4_OK : DCNV4_ERR_LAUNCH;
 }
 
 template <typename T, int Q, bool HW, bool VF>

@@ -72,6 +72,9 @@ struct TileParams {
     int PB;                 // bytes per window pixel: GS * Cg * sizeof(T)
     int cblk;               // channel blocks of the tensor map per group subset
     int tiles;              // N * tiles_y * tiles_x * nsub
+    int items;              // work items of the persistent loop: main_tiles + (tiles - main_tiles) * tail_split
+    int main_tiles;         // tiles processed whole; the rest (the last partial wave) are split by warps
+    int tail_split;         // CTAs sharing one tail tile (its consumer warps divided among them); 1: no split
     int units;              // TH * TW * GS
     int run_slot;           // shared bytes per record run
     int rec_bytes;          // one record buffer (multiple of 128)
@@ -245,6 +248,20 @@ __device__ __forceinline__ TileCoord tile_coord(const TileParams& p, unsigned t)
     return c;
 }
 
+// Tile of work item w of the persistent loop, and which warp slice of it the
+// item covers (-1: the whole tile). The last partial wave of tiles is split
+// by consumer warps over tail_split CTAs, so that it takes a fraction of a
+// tile's time instead of a whole one while most SMs idle.
+__device__ __forceinline__ unsigned item_tile(const TileParams& p, int w, int* part) {
+    if (w < p.main_tiles) {
+        *part = -1;
+        return static_cast<unsigned>(w);
+    }
+    const int q = w - p.main_tiles;
+    *part = q % p.tail_split;
+    return static_cast<unsigned>(p.main_tiles + q / p.tail_split);
+}
+
 // Address and element count of record run r of a tile.
 template <typename T>
 __device__ __forceinline__ const unsigned char* run_src(const TileParams& p, const TileCoord& c, const T* om, int r,
@@ -367,8 +384,12 @@ __device__ __forceinline__ void fma_chunk_h(float2* acc, uint32_t w2, const uint
 // PBC: the window's pixel stride as a compile-time constant (0: p.PB).
 // VF: the variant flags of p.f may be set (softmax over the masks, centre
 // point removed, centre feature scaling); false compiles them out.
+// Registers: capped at 112 per thread; the compiler's own choice under a
+// launch bound was 96, and the extra registers keep more corner loads in
+// flight. The planner keeps CTAs at 16 warps or fewer, so that each SM
+// sub-partition (16 K registers) holds its share of 4 warps.
 template <typename T, int Q, int KS, bool HW, int PBC, bool VF>
-__global__ void __launch_bounds__(544, 1)
+__global__ void __maxnreg__(112)
 fwd_tile_kernel(const __grid_constant__ CUtensorMap xmap, const T* __restrict__ x, const T* __restrict__ om,
                 T* __restrict__ out, TileParams p) {
     extern __shared__ __align__(128) unsigned char smem[];
@@ -403,9 +424,9 @@ fwd_tile_kernel(const __grid_constant__ CUtensorMap xmap, const T* __restrict__ 
     }
     __syncthreads();
     const int first = static_cast<int>(blockIdx.x);
-    if (first >= p.tiles) return;
+    if (first >= p.items) return;
     const int stride_t = static_cast<int>(gridDim.x);
-    const int ntiles = (p.tiles - first + stride_t - 1) / stride_t;
+    const int ntiles = (p.items - first + stride_t - 1) / stride_t;  // work items of this CTA
 
     if (warp == nc) {
         // ---------------------------------------------------------------- producer
@@ -429,11 +450,12 @@ fwd_tile_kernel(const __grid_constant__ CUtensorMap xmap, const T* __restrict__ 
                 return;
             }
             fence_proxy_async();  // the consumers' reads of those buffers before the async writes
+            int part_unused;
             if (i < ntiles)
-                issue_records<T>(p, om, tile_coord(p, static_cast<unsigned>(first + i * stride_t)),
+                issue_records<T>(p, om, tile_coord(p, item_tile(p, first + i * stride_t, &part_unused)),
                                  recbuf + (i % nrec) * p.rec_bytes, &rec_full[i % nrec], lane);
             if (j >= 0 && j < ntiles)
-                issue_window(p, &xmap, tile_coord(p, static_cast<unsigned>(first + j * stride_t)),
+                issue_window(p, &xmap, tile_coord(p, item_tile(p, first + j * stride_t, &part_unused)),
                              winbuf + (j & 1) * p.win_bytes, &win_full[j & 1], lane);
         }
         return;
@@ -465,8 +487,11 @@ fwd_tile_kernel(const __grid_constant__ CUtensorMap xmap, const T* __restrict__ 
     const float fdil = static_cast<float>(f.dilation);
     const int within = row_runs ? (px * f.G + gl) : gl;  // unit index inside its record run
 
+    const int wslice = warp % p.tail_split;  // this warp's slice of a split tail tile
     for (int i = 0; i < ntiles; ++i) {
-        const unsigned t = static_cast<unsigned>(first + i * stride_t);
+        int part;
+        const unsigned t = item_tile(p, first + i * stride_t, &part);
+        const bool my_slice = part < 0 || part == wslice;
         const int rb = i % nrec, wb = i & 1;
         bool ok = mbar_wait_bounded(&rec_full[rb], (i / nrec) & 1, kCopyWaitLimitNs);
         ok = ok && mbar_wait_bounded(&win_full[wb], (i >> 1) & 1, kCopyWaitLimitNs);
@@ -475,7 +500,7 @@ fwd_tile_kernel(const __grid_constant__ CUtensorMap xmap, const T* __restrict__ 
             return;
         }
         const TileCoord c = tile_coord(p, t);
-        if (has_unit && py < c.nh && px < c.nw) {
+        if (has_unit && my_slice && py < c.nh && px < c.nw) {
             const unsigned char* win = winbuf + wb * p.win_bytes;
             const T* ximg = x + static_cast<size_t>(c.n) * f.H * rowC;
             const int ho = c.ho0 + py, wo = c.wo0 + px, g = c.gsub * p.GS + gl;
