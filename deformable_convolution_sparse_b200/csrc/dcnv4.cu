@@ -282,7 +282,7 @@ int dcnv4_forward_host(const void* x_host, const void* offset_mask_host, void* o
     if (rc) return rc;
     cudaStream_t user = static_cast<cudaStream_t>(stream);
     // chunks of whole images on NS streams, so that copies in the two directions and the kernels overlap;
-    // DCNV4_HOST_CHUNKS / DCNV4_HOST_STREAMS override the defaults for tuning runs
+    // DCNV4_HOST_CHUNKS (the most chunks) / DCNV4_HOST_STREAMS override the defaults for tuning runs
     int max_chunks = 16, NS = 3;
     if (const char* c = std::getenv("DCNV4_HOST_CHUNKS")) max_chunks = std::max(1, std::atoi(c));
     if (const char* c = std::getenv("DCNV4_HOST_STREAMS")) NS = std::min(3, std::max(1, std::atoi(c)));
@@ -300,7 +300,11 @@ int dcnv4_forward_host(const void* x_host, const void* offset_mask_host, void* o
     for (int i = 0; i < NS; ++i)
         if (cudaStreamWaitEvent(pipe->s[i], ev_start, 0) != cudaSuccess) return fail(DCNV4_ERR_CUDA);
 
-    const int chunks = N < max_chunks ? N : max_chunks;
+    // about 4 MiB of copies per chunk (smaller ones are dominated by per-copy overhead), 2..max_chunks
+    const size_t step_bytes = static_cast<size_t>(N) * (x_img + om_img + out_img);
+    int chunks = static_cast<int>(std::min<size_t>(static_cast<size_t>(max_chunks),
+                                                   std::max<size_t>(2, step_bytes >> 22)));
+    if (chunks > N) chunks = N;
     const char* xh = static_cast<const char*>(x_host);
     const char* omh = static_cast<const char*>(offset_mask_host);
     char* oh = static_cast<char*>(out_host);
