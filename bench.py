@@ -86,6 +86,31 @@ KERNEL_SOURCES = {
 }
 
 
+SHAPE_ORIGIN = {
+    "tiny": "tiny case",
+    "stage1": "FlashInternImage-T stage-1 shaped",
+    "stage3": "FlashInternImage-T stage-3 shaped",
+    "sd_latent": "SD-1.5 latent U-Net block shaped",
+    "highres": "high-resolution, dilated",
+}
+
+
+def shape_origin(w) -> str:
+    for key, text in SHAPE_ORIGIN.items():
+        if w.name.startswith(key):
+            return text
+    return "synthetic"
+
+
+def _dist(d) -> str:
+    kind, a, b = d
+    return f"N({a:g},{b:g}^2)" if kind == "normal" else f"U[{a:g},{b:g}]"
+
+
+def input_recipe(w) -> str:
+    return f"seeded synthetic (seed {w.seed}): x~N(0,1), offsets~{_dist(w.offsets)}, masks~{_dist(w.masks)}"
+
+
 def kernel_sources_sha(kind: str = "forward") -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "deformable_convolution_sparse_b200", "csrc")
@@ -366,7 +391,7 @@ def run_backward(args, w, dev, world, rank, barrier, max_over_ranks):
                 "points_per_step_per_gpu": points, "parallelism": f"dp{world} (independent batches)",
                 "l2": f"steps rotate over {copies} resident sets, {copies * foot / 1e6:.0f} MB in total vs "
                       f"{l2 / 1e6:.0f} MB L2",
-                "inputs": "seeded synthetic: x~N(0,1), offsets and masks as the forward, grad_out~N(0,1)",
+                "inputs": input_recipe(w) + f", grad_out~N(0,1) (seed {1000 + w.seed})",
             },
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak,
@@ -487,7 +512,7 @@ def run_variant(args, w, dev, world, rank, barrier, max_over_ranks):
                 "points_per_step_per_gpu": points, "parallelism": f"dp{world} (independent batches)",
                 "l2": f"steps rotate over {copies} resident sets, {copies * foot / 1e6:.0f} MB in total vs "
                       f"{l2 / 1e6:.0f} MB L2",
-                "inputs": "seeded synthetic as the plain forward; gate logits ~N(0,1.5^2)",
+                "inputs": input_recipe(w) + "; gate logits ~N(0,1.5^2)",
             },
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak,
@@ -739,14 +764,14 @@ def main():
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {
-                "workload": f"{w.name}: FlashInternImage-T stage-1 shaped DCNv4 forward, N={w.N} per GPU, "
+                "workload": f"{w.name}: {shape_origin(w)} DCNv4 forward, N={w.N} per GPU, "
                             f"H=W={w.H}, C={w.C}, G={w.G} (C/G={w.Cg}), K={w.K}, stride={w.stride}, pad={w.pad}, "
                             f"dilation={w.dilation}, offset_scale={w.offset_scale}",
                 "storage_dtype": w.dtype, "accumulate": "f32", "global_batch": w.N * world,
                 "points_per_step_per_gpu": w.points, "parallelism": f"dp{world} (independent batches)",
                 "l2": f"steps rotate over {copies} resident input/output sets, {copies * foot / 1e6:.0f} MB "
                       f"in total vs {l2 / 1e6:.0f} MB L2",
-                "inputs": "seeded synthetic: x~N(0,1), offsets~N(0,1.5^2), masks~N(0,0.5^2)",
+                "inputs": input_recipe(w),
             },
             "hbm_gbs": achieved,
             "hbm_pct_of_peak": 100.0 * achieved / peak,

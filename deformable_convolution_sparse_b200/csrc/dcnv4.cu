@@ -8,6 +8,7 @@
 #include <cstdint>
 #include <algorithm>
 #include <cmath>
+#include <map>
 #include <mutex>
 
 #include <cstdio>

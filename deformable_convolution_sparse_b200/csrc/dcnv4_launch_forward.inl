@@ -22,6 +22,53 @@ constexpr int kTileUnitsMax = 480;
 static_assert(((kTileUnitsMax / 32 + 1 + 3) / 4) * 112 * 32 <= 16384,
               "the tile kernel's register cap must fit the warps of one SM sub-partition");
 
+// Mean shared-memory wavefronts of one quarter-warp LDS.128 in the tile
+// kernel's gather, for window pixels of GS groups x Q chunks (PB = 16 GS Q
+// bytes). A quarter warp is 8 consecutive units: ceil(8 / GS) pixels at
+// independent window positions, each read at the lane's rotated chunk (the
+// kernel's `rot`). With PB a multiple of 128 a chunk's bank quad does not depend
+// on the pixel and the rotation makes it exactly 1; otherwise the pixels'
+// placements collide on bank quads and the mean is taken over 256 placements
+// drawn by a fixed linear congruential generator, so the plan stays
+// deterministic. Cached per (Q, GS).
+double gather_wavefronts(int Q, int GS) {
+    static std::mutex mu;
+    static std::map<std::pair<int, int>, double> cache;
+    std::lock_guard<std::mutex> lock(mu);
+    const auto key = std::make_pair(Q, GS);
+    if (auto it = cache.find(key); it != cache.end()) return it->second;
+    const int step = GS * Q;  // chunks per pixel
+    const int npx = GS < 8 ? (8 + GS - 1) / GS : 1;
+    int rot[8];
+    for (int l = 0; l < 8; ++l) rot[l] = Q == 2 ? (l >> 2) : Q == 4 ? (l >> 1) : Q == 8 ? l : 0;
+    unsigned s = 12345u;
+    double total = 0.0;
+    long n = 0;
+    for (int it = 0; it < 256; ++it) {
+        long long pos[8];
+        for (int p = 0; p < npx; ++p) {
+            s = (s * 1103515245u + 12345u) & 0x7fffffffu;
+            pos[p] = s >> 8;
+        }
+        for (int j = 0; j < Q; ++j) {
+            long long addr[8];
+            int cnt[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+            for (int l = 0; l < 8; ++l) {
+                const int gl = GS < 8 ? l % GS : l, p = GS < 8 ? l / GS : 0;
+                addr[l] = pos[p] * step + gl * Q + (rot[l] + j) % Q;
+                bool dup = false;
+                for (int m = 0; m < l; ++m) dup = dup || addr[m] == addr[l];
+                if (!dup) ++cnt[addr[l] % 8];
+            }
+            total += *std::max_element(cnt, cnt + 8);
+            ++n;
+        }
+    }
+    const double w = total / static_cast<double>(n);
+    cache.emplace(key, w);
+    return w;
+}
+
 struct TilePlan {
     dcnv4::TileParams p;
     CUtensorMap map;
@@ -64,8 +111,13 @@ bool plan_tile(const void* x, const void* om, const void* out, const FwdParams& 
             if (sub_ch % d == 0 && (d * E) % 16 == 0) { c2 = d; break; }
         if (c2 == 0 || sub_ch / c2 > 256) continue;
         // a pixel stride that is a multiple of 128 bytes keeps the gathers free of
-        // bank conflicts (see the kernel); other strides pay for some
-        const double banks = (PB % 128 == 0) ? 1.0 : 0.6;
+        // bank conflicts (see the kernel); other strides pay in extra wavefronts.
+        // The gather's shared-memory reads dominate a tile's cost there, and the
+        // squared factor matches the measured 1.21x between 80- and 160-byte
+        // pixels of the 40-channel groups (2.60 vs 2.13 wavefronts), against
+        // which the window-reuse and ring-depth terms would otherwise win.
+        const double w = gather_wavefronts(Q, GS);
+        const double banks = 1.0 / (w * w);
         const bool row_runs = GS == f.G;
         for (int TH : THs) {
             for (int TW : TWs) {
