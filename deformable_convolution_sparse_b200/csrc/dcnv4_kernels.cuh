@@ -239,8 +239,10 @@ __device__ __forceinline__ void unit_coords(int unit, const FwdParams& p, int& n
 
 // One thread covers LB bytes (LB / VB vectors of VB bytes) of one unit's
 // channels per pass; `p.lanes` threads share a unit and loop over
-// `p.chunks` chunks. KS > 0 fixes K at compile time (0: runtime K).
-template <typename T, int VB, int LB, int KS>
+// `p.chunks` chunks. KS > 0 fixes K at compile time (0: runtime K). VF: the
+// variant flags of p may be set (softmax over the masks, centre point
+// removed, centre feature scaling); false compiles them out.
+template <typename T, int VB, int LB, int KS, bool VF>
 __global__ void __launch_bounds__(256)
 fwd_vector_kernel(const T* __restrict__ x, const T* __restrict__ om, T* __restrict__ out, FwdParams p) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -250,7 +252,8 @@ fwd_vector_kernel(const T* __restrict__ x, const T* __restrict__ om, T* __restri
     constexpr int CPL = LB / E;         // channels per thread per pass
     const int K = KS > 0 ? KS : p.K;
     const int KK = K * K;
-    const int NP = p.npts;
+    const int NP = VF ? p.npts : KK;  // points per unit
+    const int kcs = VF ? p.kc : KK;   // grid index left out (none: KK)
     const int R = 3 * NP;
 
     const int unit0 = blockIdx.x * p.units_per_block;
@@ -269,7 +272,7 @@ fwd_vector_kernel(const T* __restrict__ x, const T* __restrict__ om, T* __restri
     const int rowC = p.W * p.C;
     const T* ximg = x + static_cast<size_t>(n) * p.H * rowC;
     T* o = out + (static_cast<size_t>((n * p.Hout + ho) * p.Wout + wo)) * p.C + g * p.Cg;
-    const MaskNorm mn = mask_norm(rec + 2 * NP, NP, p.flags);
+    const MaskNorm mn = VF ? mask_norm(rec + 2 * NP, NP, p.flags) : MaskNorm{0.f, 1.f, false};
 
     for (int ch = part; ch < p.chunks; ch += p.lanes) {
         const int c0 = g * p.Cg + ch * CPL;   // first channel of this thread's slice
@@ -279,8 +282,8 @@ fwd_vector_kernel(const T* __restrict__ x, const T* __restrict__ om, T* __restri
 
 #pragma unroll (KS > 0 ? KS * KS : 1)
         for (int k = 0; k < KK; ++k) {
-            if (k == p.kc) continue;
-            const int jp = k - (k > p.kc ? 1 : 0);  // point index in the record
+            if (k == kcs) continue;
+            const int jp = k - (k > kcs ? 1 : 0);  // point index in the record
             const int ky = k / K, kx = k - (k / K) * K;
             const int p0y = ho * p.stride - p.pad + ky * p.dilation;
             const int p0x = wo * p.stride - p.pad + kx * p.dilation;
@@ -331,7 +334,7 @@ fwd_vector_kernel(const T* __restrict__ x, const T* __restrict__ om, T* __restri
             }
         }
 
-        if (p.flags & kFlagCenterScale) {
+        if (VF && (p.flags & kFlagCenterScale)) {
             // out = (1 - s) * aggregate + s * x at the centre grid position (zero outside)
             const float sg = center_gate<T>(p, static_cast<size_t>(unit));
             const int cy = ho * p.stride - p.pad + (K / 2) * p.dilation;
@@ -381,13 +384,14 @@ fwd_vector_kernel(const T* __restrict__ x, const T* __restrict__ om, T* __restri
 
 // Element-wise fallback for any channel count and alignment: one thread per
 // (unit, channel) slot, looping over the unit's channels with stride p.lanes.
-template <typename T, int KS>
+template <typename T, int KS, bool VF>
 __global__ void __launch_bounds__(256)
 fwd_scalar_kernel(const T* __restrict__ x, const T* __restrict__ om, T* __restrict__ out, FwdParams p) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const int K = KS > 0 ? KS : p.K;
     const int KK = K * K;
-    const int NP = p.npts;
+    const int NP = VF ? p.npts : KK;  // points per unit
+    const int kcs = VF ? p.kc : KK;   // grid index left out (none: KK)
     const int R = 3 * NP;
     const int unit0 = blockIdx.x * p.units_per_block;
     const int nunits = min(p.units_per_block, p.units - unit0);
@@ -404,13 +408,13 @@ fwd_scalar_kernel(const T* __restrict__ x, const T* __restrict__ om, T* __restri
     const int rowC = p.W * p.C;
     const T* ximg = x + static_cast<size_t>(n) * p.H * rowC;
     T* o = out + (static_cast<size_t>((n * p.Hout + ho) * p.Wout + wo)) * p.C + g * p.Cg;
-    const MaskNorm mn = mask_norm(rec + 2 * NP, NP, p.flags);
+    const MaskNorm mn = VF ? mask_norm(rec + 2 * NP, NP, p.flags) : MaskNorm{0.f, 1.f, false};
 
     for (int c = part; c < p.Cg; c += p.lanes) {
         float acc = 0.f;
         for (int k = 0; k < KK; ++k) {
-            if (k == p.kc) continue;
-            const int jp = k - (k > p.kc ? 1 : 0);  // point index in the record
+            if (k == kcs) continue;
+            const int jp = k - (k > kcs ? 1 : 0);  // point index in the record
             const int ky = k / K, kx = k - (k / K) * K;
             const int p0y = ho * p.stride - p.pad + ky * p.dilation;
             const int p0x = wo * p.stride - p.pad + kx * p.dilation;
@@ -426,7 +430,7 @@ fwd_scalar_kernel(const T* __restrict__ x, const T* __restrict__ om, T* __restri
             if (s.bits & 4u) acc = fmaf(m * s.ly * wx0, ElemTraits<T>::to_float(c00[rowC]), acc);
             if (s.bits & 8u) acc = fmaf(m * s.ly * s.lx, ElemTraits<T>::to_float(c00[rowC + p.C]), acc);
         }
-        if (p.flags & kFlagCenterScale) {
+        if (VF && (p.flags & kFlagCenterScale)) {
             const float sg = center_gate<T>(p, static_cast<size_t>(unit));
             const int cy = ho * p.stride - p.pad + (K / 2) * p.dilation;
             const int cx = wo * p.stride - p.pad + (K / 2) * p.dilation;

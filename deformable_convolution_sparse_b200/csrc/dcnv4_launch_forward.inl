@@ -302,6 +302,28 @@ int launch_tile(const void* x, const void* om, void* out, const TilePlan& plan, 
     }
 }
 
+// The global-gather kernels for one thread-slice width (lane_bytes: 64, 32 or
+// 16 bytes per thread, 0 for the element-wise kernel).
+template <typename T, bool VF>
+int launch_gather(const T* xt, const T* omt, T* ot, const FwdParams& p, int lane_bytes, dim3 grid, int threads,
+                  size_t smem, cudaStream_t stream) {
+    const bool k3 = p.K == 3;
+    if (lane_bytes == 64) {
+        if (k3) dcnv4::fwd_vector_kernel<T, 32, 64, 3, VF><<<grid, threads, smem, stream>>>(xt, omt, ot, p);
+        else dcnv4::fwd_vector_kernel<T, 32, 64, 0, VF><<<grid, threads, smem, stream>>>(xt, omt, ot, p);
+    } else if (lane_bytes == 32) {
+        if (k3) dcnv4::fwd_vector_kernel<T, 32, 32, 3, VF><<<grid, threads, smem, stream>>>(xt, omt, ot, p);
+        else dcnv4::fwd_vector_kernel<T, 32, 32, 0, VF><<<grid, threads, smem, stream>>>(xt, omt, ot, p);
+    } else if (lane_bytes == 16) {
+        if (k3) dcnv4::fwd_vector_kernel<T, 16, 16, 3, VF><<<grid, threads, smem, stream>>>(xt, omt, ot, p);
+        else dcnv4::fwd_vector_kernel<T, 16, 16, 0, VF><<<grid, threads, smem, stream>>>(xt, omt, ot, p);
+    } else {
+        if (k3) dcnv4::fwd_scalar_kernel<T, 3, VF><<<grid, threads, smem, stream>>>(xt, omt, ot, p);
+        else dcnv4::fwd_scalar_kernel<T, 0, VF><<<grid, threads, smem, stream>>>(xt, omt, ot, p);
+    }
+    return launch_status();
+}
+
 template <typename T>
 int launch_forward(const void* x, const void* om, void* out, FwdParams p, cudaStream_t stream) {
     constexpr int E = sizeof(T);
@@ -344,19 +366,7 @@ int launch_forward(const void* x, const void* om, void* out, FwdParams p, cudaSt
     const T* xt = static_cast<const T*>(x);
     const T* omt = static_cast<const T*>(om);
     T* ot = static_cast<T*>(out);
-    const bool k3 = p.K == 3;
-    if (lane_bytes == 64) {
-        if (k3) dcnv4::fwd_vector_kernel<T, 32, 64, 3><<<grid, threads, smem, stream>>>(xt, omt, ot, p);
-        else dcnv4::fwd_vector_kernel<T, 32, 64, 0><<<grid, threads, smem, stream>>>(xt, omt, ot, p);
-    } else if (lane_bytes == 32) {
-        if (k3) dcnv4::fwd_vector_kernel<T, 32, 32, 3><<<grid, threads, smem, stream>>>(xt, omt, ot, p);
-        else dcnv4::fwd_vector_kernel<T, 32, 32, 0><<<grid, threads, smem, stream>>>(xt, omt, ot, p);
-    } else if (lane_bytes == 16) {
-        if (k3) dcnv4::fwd_vector_kernel<T, 16, 16, 3><<<grid, threads, smem, stream>>>(xt, omt, ot, p);
-        else dcnv4::fwd_vector_kernel<T, 16, 16, 0><<<grid, threads, smem, stream>>>(xt, omt, ot, p);
-    } else {
-        if (k3) dcnv4::fwd_scalar_kernel<T, 3><<<grid, threads, smem, stream>>>(xt, omt, ot, p);
-        else dcnv4::fwd_scalar_kernel<T, 0><<<grid, threads, smem, stream>>>(xt, omt, ot, p);
-    }
-    return launch_status();
+    // the variant flags get their own instantiations, as in the tile kernel
+    if (p.flags != 0) return launch_gather<T, true>(xt, omt, ot, p, lane_bytes, grid, threads, smem, stream);
+    return launch_gather<T, false>(xt, omt, ot, p, lane_bytes, grid, threads, smem, stream);
 }
