@@ -111,6 +111,25 @@ def input_recipe(w) -> str:
     return f"seeded synthetic (seed {w.seed}): x~N(0,1), offsets~{_dist(w.offsets)}, masks~{_dist(w.masks)}"
 
 
+def workload_text(w, which: str = "forward", variant: str = "none") -> str:
+    """config.workload of a line: the same text on both arms for the same pass and variant."""
+    P = w.K * w.K - (1 if VARIANT_FLAGS.get(variant, 0) & 2 else 0)
+    if which == "predictor":
+        M, NO = w.N * w.Hout * w.Wout, 3 * w.G * w.K * w.K
+        return (f"{w.name} predictor: y [{M}, {w.C}] x W [{NO}, {w.C}] + bias -> offset_mask "
+                f"[{M}, {w.G}, {3 * w.K * w.K}] (the records of the {w.name} aggregation)")
+    if which == "backward":
+        return (f"{w.name} backward, variant {variant}: N={w.N} per GPU, H=W={w.H}, C={w.C}, "
+                f"G={w.G} (C/G={w.Cg}), K={w.K}, {P} points per unit, stride={w.stride}, pad={w.pad}, "
+                f"dilation={w.dilation}; fp32 gradients")
+    if variant != "none":
+        return (f"{w.name} forward, variant {variant}: N={w.N} per GPU, H=W={w.H}, C={w.C}, "
+                f"G={w.G}, K={w.K}, {P} points per unit")
+    return (f"{w.name}: {shape_origin(w)} DCNv4 forward, N={w.N} per GPU, H=W={w.H}, C={w.C}, G={w.G} "
+            f"(C/G={w.Cg}), K={w.K}, stride={w.stride}, pad={w.pad}, dilation={w.dilation}, "
+            f"offset_scale={w.offset_scale}")
+
+
 def kernel_sources_sha(kind: str = "forward") -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "deformable_convolution_sparse_b200", "csrc")
@@ -214,43 +233,90 @@ def cpu_baseline_backward(w, x, om, go):
 
 
 def run_reference(args):
+    """The reference arm: the fp64 oracle as it stands, on the host cores, for the same pass, variant,
+    workload, metric and unit as this implementation's line; each step is a bounded sample of the workload."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    from deformable_convolution_sparse_b200.workloads import BENCH_WORKLOAD, WORKLOADS, workload_inputs
+    import torch
+    from deformable_convolution_sparse_b200.workloads import (BENCH_WORKLOAD, WORKLOADS, make_center_logit,
+                                                              make_inputs, workload_grad_out)
     import oracle
     w = WORKLOADS[args.workload or BENCH_WORKLOAD]
-    x, om = workload_inputs(w)
-    xd, omd = x.double().numpy(), om.double().numpy()
+    flags = VARIANT_FLAGS.get(args.variant, 0)
+    P = w.K * w.K - (1 if flags & 2 else 0)
+    kw = w.kwargs()
+    vkw = dict(softmax=bool(flags & 1), remove_center=bool(flags & 2))
     n_s = max(1, min(w.N, 8))  # images per step: a bounded sample (~0.1 s of CPU work each)
-    pts = w.points // w.N * n_s
-    if args.which == "backward":
-        from deformable_convolution_sparse_b200.workloads import workload_grad_out
-        god = workload_grad_out(w).double().numpy()
+    if args.which == "predictor":
+        M, NO = w.N * w.Hout * w.Wout, 3 * w.G * w.K * w.K
+        rows = n_s * w.Hout * w.Wout
+        # the same draws as this implementation's predictor line (rank 0)
+        td = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}[w.dtype]
+        gen = torch.Generator().manual_seed(w.seed)
+        y = torch.randn(M, w.C, generator=gen).to(td).double().numpy()
+        wt = (torch.randn(NO, w.C, generator=gen) * w.C ** -0.5).to(td).double().numpy()
+        b = torch.randn(NO, generator=gen).double().numpy()
+        metric, unit, per_step = METRIC_PRED, "Grecords/s", rows * w.G
 
-        def one(b):
-            oracle.dcnv4_backward(xd[b:b + n_s], omd[b:b + n_s], god[b:b + n_s], **w.kwargs())
+        def one(i):
+            r0 = (i * rows) % (M - rows + 1)
+            oracle.dcnv4_predictor(y[r0:r0 + rows], wt, b, G=w.G, P=w.K * w.K)
     else:
-        def one(b):
-            oracle.dcnv4_forward(xd, omd, **w.kwargs(), n_begin=b, n_end=b + n_s)
+        x, om = make_inputs(w.N, w.H, w.W, w.C, w.G, w.K, w.Hout, w.Wout, w.dtype, w.offsets, w.masks,
+                            seed=w.seed, points=P)
+        xd, omd = x.double().numpy(), om.double().numpy()
+        zd = make_center_logit(w.N, w.Hout, w.Wout, w.G, w.dtype, seed=w.seed).double().numpy()
+        per_step = w.N * w.Hout * w.Wout * w.G * P // w.N * n_s
+        unit = UNIT
+        if args.which == "backward":
+            metric = METRIC_BWD
+            god = workload_grad_out(w).double().numpy()
+
+            def one(i):
+                b0 = (i * n_s) % (w.N - n_s + 1)
+                sl = slice(b0, b0 + n_s)
+                if flags:
+                    oracle.dcnv4_backward_variants(xd[sl], omd[sl], god[sl], **kw, **vkw,
+                                                   center_logit=zd[sl] if flags & 4 else None)
+                else:
+                    oracle.dcnv4_backward(xd[sl], omd[sl], god[sl], **kw)
+        else:
+            metric = METRIC
+
+            def one(i):
+                b0 = (i * n_s) % (w.N - n_s + 1)
+                sl = slice(b0, b0 + n_s)
+                if flags:
+                    oracle.dcnv4_forward_variants(xd[sl], omd[sl], **kw, **vkw,
+                                                  center_logit=zd[sl] if flags & 4 else None)
+                else:
+                    oracle.dcnv4_forward(xd, omd, **kw, n_begin=b0, n_end=b0 + n_s)
     for _ in range(args.warmup):
         one(0)
     t0 = time.perf_counter()
     for i in range(args.steps):
-        one((i * n_s) % (w.N - n_s + 1))
+        one(i)
     dt = time.perf_counter() - t0
-    value = pts * args.steps / dt / 1e9
+    value = per_step * args.steps / dt / 1e9
+    what = f"{args.which}" + (f", variant {args.variant}" if args.variant != "none" else "")
+    sample = (f"{n_s * w.Hout * w.Wout} of {w.N * w.Hout * w.Wout} pixels ({n_s} images) per step"
+              if args.which == "predictor" else f"{n_s} of {w.N} images per step")
     line = {
-        "impl": "reference", "metric": METRIC_BWD if args.which == "backward" else METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "impl": "reference", "metric": metric, "value": value, "unit": unit, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": f"{w.name}: N={w.N} H=W={w.H} C={w.C} G={w.G} K={w.K} pad={w.pad} "
-                               f"dilation={w.dilation}, {w.dtype} storage", "sample_images_per_step": n_s},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
-                         "sample": f"{n_s} of {w.N} images per step, fp64 C oracle "
-                                   f"{args.which}, one thread"},
-        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "config": {"workload": workload_text(w, args.which, args.variant), "storage_dtype": w.dtype,
+                   "accumulate": "f64 (oracle)", "sample_per_step": sample},
+        "cpu_baseline": {"value": value, "unit": unit, "cores": 1, "kind": "oracle",
+                         "sample": f"{sample}, fp64 C oracle {what}, one thread"},
+        "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
+    # the same pass/variant keys as this implementation's line for that row
+    if args.which != "forward":
+        line["pass"] = args.which
+    if args.which == "backward" or (args.which == "forward" and args.variant != "none"):
+        line["variant"] = args.variant
     print(json.dumps(line), flush=True)
 
 
@@ -384,9 +450,7 @@ def run_backward(args, w, dev, world, rank, barrier, max_over_ranks):
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic", "pass": "backward", "variant": args.variant,
             "config": {
-                "workload": f"{w.name} backward, variant {args.variant}: N={w.N} per GPU, H=W={w.H}, C={w.C}, "
-                            f"G={w.G} (C/G={w.Cg}), K={w.K}, {P} points per unit, stride={w.stride}, pad={w.pad}, "
-                            f"dilation={w.dilation}; fp32 gradients",
+                "workload": workload_text(w, "backward", args.variant),
                 "storage_dtype": w.dtype, "accumulate": "f32", "global_batch": w.N * world,
                 "points_per_step_per_gpu": points, "parallelism": f"dp{world} (independent batches)",
                 "l2": f"steps rotate over {copies} resident sets, {copies * foot / 1e6:.0f} MB in total vs "
@@ -506,8 +570,7 @@ def run_variant(args, w, dev, world, rank, barrier, max_over_ranks):
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic", "variant": args.variant,
             "config": {
-                "workload": f"{w.name} forward, variant {args.variant}: N={w.N} per GPU, H=W={w.H}, C={w.C}, "
-                            f"G={w.G}, K={w.K}, {P} points per unit",
+                "workload": workload_text(w, "forward", args.variant),
                 "storage_dtype": w.dtype, "accumulate": "f32", "global_batch": w.N * world,
                 "points_per_step_per_gpu": points, "parallelism": f"dp{world} (independent batches)",
                 "l2": f"steps rotate over {copies} resident sets, {copies * foot / 1e6:.0f} MB in total vs "
@@ -618,8 +681,7 @@ def run_predictor(args, w, dev, world, rank, barrier, max_over_ranks):
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": w.dtype, "data": "synthetic", "pass": "predictor",
             "config": {
-                "workload": f"{w.name} predictor: y [{M}, {w.C}] x W [{NO}, {w.C}] + bias -> offset_mask "
-                            f"[{M}, {w.G}, {3 * P}] (the records of the {w.name} aggregation)",
+                "workload": workload_text(w, "predictor"),
                 "storage_dtype": w.dtype, "accumulate": "f32 (tensor memory)", "global_batch": w.N * world,
                 "parallelism": f"dp{world} (independent batches)",
                 "l2": f"steps rotate over {copies} resident sets, {copies * foot / 1e6:.0f} MB in total vs "
@@ -764,9 +826,7 @@ def main():
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {
-                "workload": f"{w.name}: {shape_origin(w)} DCNv4 forward, N={w.N} per GPU, "
-                            f"H=W={w.H}, C={w.C}, G={w.G} (C/G={w.Cg}), K={w.K}, stride={w.stride}, pad={w.pad}, "
-                            f"dilation={w.dilation}, offset_scale={w.offset_scale}",
+                "workload": workload_text(w),
                 "storage_dtype": w.dtype, "accumulate": "f32", "global_batch": w.N * world,
                 "points_per_step_per_gpu": w.points, "parallelism": f"dp{world} (independent batches)",
                 "l2": f"steps rotate over {copies} resident input/output sets, {copies * foot / 1e6:.0f} MB "
