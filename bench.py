@@ -206,6 +206,24 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+def host_cpu() -> str:
+    """Model name of the host CPU (from /proc/cpuinfo) and the cores this process may run on."""
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    try:
+        avail = len(os.sched_getaffinity(0))
+    except (AttributeError, OSError):
+        avail = os.cpu_count() or 0
+    return f"{model}; {avail} cores available, 1 used"
+
+
 def cpu_baseline(w, x, om):
     """The fp64 oracle, as it stands, on the whole batch (single thread)."""
     import oracle
@@ -214,7 +232,7 @@ def cpu_baseline(w, x, om):
     t0 = time.perf_counter()
     oracle.dcnv4_forward(xd, omd, **w.kwargs())
     dt = time.perf_counter() - t0
-    return {"value": w.points / dt / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
+    return {"value": w.points / dt / 1e9, "unit": UNIT, "cores": 1, "cpu": host_cpu(), "kind": "oracle",
             "seconds": dt, "sample": f"the whole {w.name} batch ({w.N} images, {w.points} points), "
                                     "fp64 C oracle, one thread"}
 
@@ -227,7 +245,7 @@ def cpu_baseline_backward(w, x, om, go):
     t0 = time.perf_counter()
     oracle.dcnv4_backward(xd, omd, god, **w.kwargs())
     dt = time.perf_counter() - t0
-    return {"value": w.points / dt / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
+    return {"value": w.points / dt / 1e9, "unit": UNIT, "cores": 1, "cpu": host_cpu(), "kind": "oracle",
             "seconds": dt, "sample": f"the whole {w.name} batch ({w.N} images, {w.points} points), "
                                     "fp64 C oracle backward, one thread"}
 
@@ -308,7 +326,7 @@ def run_reference(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": workload_text(w, args.which, args.variant), "storage_dtype": w.dtype,
                    "accumulate": "f64 (oracle)", "sample_per_step": sample},
-        "cpu_baseline": {"value": value, "unit": unit, "cores": 1, "kind": "oracle",
+        "cpu_baseline": {"value": value, "unit": unit, "cores": 1, "cpu": host_cpu(), "kind": "oracle",
                          "sample": f"{sample}, fp64 C oracle {what}, one thread"},
         "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -562,7 +580,7 @@ def run_variant(args, w, dev, world, rank, barrier, max_over_ranks):
         t0 = time.perf_counter()
         oracle.dcnv4_forward_variants(xs64, oms64, **kw)
         dt = time.perf_counter() - t0
-        base = {"value": points // w.N * n_s / dt / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
+        base = {"value": points // w.N * n_s / dt / 1e9, "unit": UNIT, "cores": 1, "cpu": host_cpu(), "kind": "oracle",
                 "seconds": dt, "sample": f"{n_s} of {w.N} images, fp64 C oracle ({args.variant}), one thread"}
     if rank == 0:
         line = {
@@ -673,7 +691,7 @@ def run_predictor(args, w, dev, world, rank, barrier, max_over_ranks):
         t0 = time.perf_counter()
         oracle.dcnv4_predictor(ys, ws, bs, G=w.G, P=P)
         dt = time.perf_counter() - t0
-        base = {"value": n_s * w.G / dt / 1e9, "unit": "Grecords/s", "cores": 1, "kind": "oracle", "seconds": dt,
+        base = {"value": n_s * w.G / dt / 1e9, "unit": "Grecords/s", "cores": 1, "cpu": host_cpu(), "kind": "oracle", "seconds": dt,
                 "sample": f"{n_s} of {M} pixels (8 images), fp64 C oracle predictor, one thread"}
     if rank == 0:
         line = {
