@@ -80,3 +80,42 @@ def test_gloo_world2_shard_and_gather(N):
         assert own_n == hi - lo
         np.testing.assert_array_equal(full, ref)
         assert slowest == 2.0
+
+
+def _failing_worker(rank, world, port, q):
+    """Rank 1's compute raises before the all-gather; rank 0 must get an error, not wait for good."""
+    import datetime
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=20))
+    x, om = make_inputs(4, 9, 10, 16, 2, 3, 9, 10, "f32", ("normal", 0, 1.5), seed=22)
+
+    def compute(xs, oms, **kw):
+        if rank == 1:
+            raise RuntimeError("injected failure")
+        return _oracle_compute([])(xs, oms, **kw)
+
+    try:
+        forward_sharded(x, om, G=2, K=3, pad=1, compute=compute)
+        q.put((rank, "finished"))
+    except RuntimeError as e:
+        q.put((rank, "injected" if "injected failure" in str(e) else "peer error"))
+    # rank 1 leaves without taking part in the collective; rank 0 leaves after its error
+    q.close()
+    q.join_thread()
+    os._exit(0)
+
+
+def test_gloo_failed_rank_ends_the_collective_with_an_error():
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_failing_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    got = dict(q.get(timeout=120) for _ in range(world))
+    for p in procs:
+        p.join(timeout=60)
+        if p.is_alive():
+            p.kill()
+    assert got == {0: "peer error", 1: "injected"}
