@@ -1,13 +1,17 @@
 #!/usr/bin/env python
 """Throughput benchmark of the DCNv4 forward spatial aggregation on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
     torchrun --nproc-per-node N bench.py --gpus N ...     (one rank per GPU)
 
-A step is one dcnv4_forward call over one batch of the FlashInternImage-T
-stage-1 shaped workload (N=64, 56x56, C=64, G=4, K=3, fp16 storage, fp32
-arithmetic; seeded synthetic inputs). With N GPUs every rank processes its own
-batch of 64 images (weak scaling, no collective on the data path).
+A step is one dcnv4_forward call over one batch of a named workload (seeded
+synthetic inputs in the workload's shape and value distributions). Without
+--workload the run prints one JSON line per named workload, in the order
+stage1_f32, stage1_f16, stage3_f16, sd_latent_f16, highres_bf16: the last
+line, the high-resolution bf16 batch (the largest workload by sampling points,
+9.29 M per step), is the headline. tiny_f32 is a parity case, not a line.
+With N GPUs every rank processes its own batch of the workload (weak
+scaling, no collective on the data path).
 
 Timing: W untimed warm-up steps, a ~1 s untimed soak (clocks settle and are
 sampled), then exactly K steps between CUDA events on the launching stream,
@@ -16,13 +20,14 @@ ranks. The steps rotate over several resident copies of the inputs whose total
 exceeds the L2 cache, so no step starts with its inputs in L2.
 
 --impl reference times the fp64 CPU oracle (the reference arm of this
-repository: there is no other implementation to install) on the host cores.
+repository: there is no other implementation to install) on the host cores,
+for the same workloads, metric and unit.
 
 Secondary lines (not the headline): --pass backward times dcnv4_backward on
-the same workload; --pass predictor times dcnv4_predictor (the tcgen05
-projection that produces the workload's offset_mask records); --variant
-softmax|remove_center|center_scale|all times dcnv4_forward_ex with those
-variant flags.
+the stage-1 fp16 batch (or --workload); --pass predictor times
+dcnv4_predictor (the tcgen05 projection that produces the workload's
+offset_mask records); --variant softmax|remove_center|center_scale|all times
+dcnv4_forward_ex with those variant flags.
 """
 from __future__ import annotations
 
@@ -54,7 +59,8 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default=None, help="named workload (default: the stage-1 fp16 batch)")
+    ap.add_argument("--workload", default=None, help="one named workload (default: every forward line; the "
+                                                     "stage-1 fp16 batch for the other passes)")
     ap.add_argument("--soak-s", type=float, default=1.0)
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -79,9 +85,10 @@ def measured_peaks():
 
 # the source files that define each profiled kernel and its launch configuration
 KERNEL_SOURCES = {
-    "forward": ("dcnv4_kernels.cuh", "dcnv4_window.cuh", "dcnv4_host_common.inl", "dcnv4_launch_forward.inl"),
+    "forward": ("dcnv4_kernels.cuh", "dcnv4_async.cuh", "dcnv4_window.cuh", "dcnv4_host_common.inl",
+                "dcnv4_launch_forward.inl"),
     "backward": ("dcnv4_kernels.cuh", "dcnv4_backward.cuh", "dcnv4_host_common.inl", "dcnv4_launch_backward.inl"),
-    "predictor": ("dcnv4_kernels.cuh", "dcnv4_window.cuh", "dcnv4_predictor.cuh", "dcnv4_host_common.inl",
+    "predictor": ("dcnv4_kernels.cuh", "dcnv4_async.cuh", "dcnv4_predictor.cuh", "dcnv4_host_common.inl",
                   "dcnv4_launch_predictor.inl"),
 }
 
@@ -206,7 +213,7 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
-def host_cpu() -> str:
+def host_cpu(used: int = 1) -> str:
     """Model name of the host CPU (from /proc/cpuinfo) and the cores this process may run on."""
     model = "unknown"
     try:
@@ -217,24 +224,33 @@ def host_cpu() -> str:
                     break
     except OSError:
         pass
+    return f"{model}; {host_cores()} cores available, {used} used"
+
+
+def host_cores() -> int:
     try:
-        avail = len(os.sched_getaffinity(0))
+        return len(os.sched_getaffinity(0))
     except (AttributeError, OSError):
-        avail = os.cpu_count() or 0
-    return f"{model}; {avail} cores available, 1 used"
+        return os.cpu_count() or 1
 
 
 def cpu_baseline(w, x, om):
-    """The fp64 oracle, as it stands, on the whole batch (single thread)."""
+    """The fp64 oracle, as it stands, on the whole batch: on every host core this process may use
+    (OpenMP over output rows; the same per-element code, so the same bits) and on one thread."""
     import oracle
     xd, omd = x.double().numpy(), om.double().numpy()
-    oracle.dcnv4_forward(xd, omd, **w.kwargs(), n_begin=0, n_end=1)  # load + warm
+    cores = host_cores()
+    oracle.dcnv4_forward(xd, omd, **w.kwargs(), n_begin=0, n_end=1, threads=cores)  # load + warm
+    t0 = time.perf_counter()
+    oracle.dcnv4_forward(xd, omd, **w.kwargs(), threads=cores)
+    dt = time.perf_counter() - t0
     t0 = time.perf_counter()
     oracle.dcnv4_forward(xd, omd, **w.kwargs())
-    dt = time.perf_counter() - t0
-    return {"value": w.points / dt / 1e9, "unit": UNIT, "cores": 1, "cpu": host_cpu(), "kind": "oracle",
-            "seconds": dt, "sample": f"the whole {w.name} batch ({w.N} images, {w.points} points), "
-                                    "fp64 C oracle, one thread"}
+    dt1 = time.perf_counter() - t0
+    return {"value": w.points / dt / 1e9, "unit": UNIT, "cores": cores, "cpu": host_cpu(cores), "kind": "oracle",
+            "seconds": dt, "sample": f"the whole {w.name} batch ({w.N} images, {w.points} points), fp64 C oracle, "
+                                    f"output rows shared out among {cores} OpenMP threads",
+            "single_thread": {"value": w.points / dt1 / 1e9, "unit": UNIT, "cores": 1, "seconds": dt1}}
 
 
 def cpu_baseline_backward(w, x, om, go):
@@ -256,14 +272,21 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
+    from deformable_convolution_sparse_b200.workloads import WORKLOADS
+    for name in workloads_to_run(args):
+        reference_line(args, WORKLOADS[name])
+
+
+def reference_line(args, w):
     import torch
-    from deformable_convolution_sparse_b200.workloads import (BENCH_WORKLOAD, WORKLOADS, make_center_logit,
-                                                              make_inputs, workload_grad_out)
+    from deformable_convolution_sparse_b200.workloads import make_center_logit, make_inputs, workload_grad_out
     import oracle
-    w = WORKLOADS[args.workload or BENCH_WORKLOAD]
     flags = VARIANT_FLAGS.get(args.variant, 0)
     P = w.K * w.K - (1 if flags & 2 else 0)
     kw = w.kwargs()
+    # the plain forward runs on every host core (OpenMP over output rows, the same bits as one thread);
+    # the other passes time the oracle's single-thread code
+    cores = host_cores() if (args.which == "forward" and not flags) else 1
     vkw = dict(softmax=bool(flags & 1), remove_center=bool(flags & 2))
     n_s = max(1, min(w.N, 8))  # images per step: a bounded sample (~0.1 s of CPU work each)
     if args.which == "predictor":
@@ -309,7 +332,7 @@ def run_reference(args):
                     oracle.dcnv4_forward_variants(xd[sl], omd[sl], **kw, **vkw,
                                                   center_logit=zd[sl] if flags & 4 else None)
                 else:
-                    oracle.dcnv4_forward(xd, omd, **kw, n_begin=b0, n_end=b0 + n_s)
+                    oracle.dcnv4_forward(xd, omd, **kw, n_begin=b0, n_end=b0 + n_s, threads=cores)
     for _ in range(args.warmup):
         one(0)
     t0 = time.perf_counter()
@@ -326,8 +349,9 @@ def run_reference(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": workload_text(w, args.which, args.variant), "storage_dtype": w.dtype,
                    "accumulate": "f64 (oracle)", "sample_per_step": sample},
-        "cpu_baseline": {"value": value, "unit": unit, "cores": 1, "cpu": host_cpu(), "kind": "oracle",
-                         "sample": f"{sample}, fp64 C oracle {what}, one thread"},
+        "cpu_baseline": {"value": value, "unit": unit, "cores": cores, "cpu": host_cpu(cores), "kind": "oracle",
+                         "sample": f"{sample}, fp64 C oracle {what}, "
+                                   + (f"{cores} OpenMP threads" if cores > 1 else "one thread")},
         "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     # the same pass/variant keys as this implementation's line for that row
@@ -336,6 +360,25 @@ def run_reference(args):
     if args.which == "backward" or (args.which == "forward" and args.variant != "none"):
         line["variant"] = args.variant
     print(json.dumps(line), flush=True)
+
+
+# the forward lines of the default run, in print order: the last one (the largest
+# workload by sampling points) is the headline
+FORWARD_LINES = ("stage1_f32", "stage1_f16", "stage3_f16", "sd_latent_f16", "highres_bf16")
+
+# the arithmetic each storage type's forward computes in (the line's "dtype")
+ARITH = {"f32": "f32", "bf16": "f32",
+         "f16": "f32 accumulate, fp16-rounded corner weights (fp16 x fp16 products exact in f32)"}
+
+
+def workloads_to_run(args):
+    """--workload names one line; without it the forward prints every named workload's line (the
+    tiny parity case excepted), the largest last, and the other passes use the stage-1 fp16 batch."""
+    if args.workload:
+        return [args.workload]
+    if args.which == "forward" and args.variant == "none":
+        return list(FORWARD_LINES)
+    return [BENCH_WORKLOAD]
 
 
 def time_steps(step, launches, args, dev, stream, barrier, max_over_ranks):
@@ -586,7 +629,7 @@ def run_variant(args, w, dev, world, rank, barrier, max_over_ranks):
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f32", "data": "synthetic", "variant": args.variant,
+            "vs_baseline": None, "dtype": ARITH[w.dtype], "data": "synthetic", "variant": args.variant,
             "config": {
                 "workload": workload_text(w, "forward", args.variant),
                 "storage_dtype": w.dtype, "accumulate": "f32", "global_batch": w.N * world,
@@ -758,8 +801,8 @@ def main():
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         return float(t.item())
 
-    w = WORKLOADS[args.workload or BENCH_WORKLOAD]
     if args.which != "forward" or args.variant != "none":
+        w = WORKLOADS[args.workload or BENCH_WORKLOAD]
         if args.which == "backward":
             run_backward(args, w, dev, world, rank, barrier, max_over_ranks)
         elif args.which == "predictor":
@@ -769,6 +812,19 @@ def main():
         if world > 1:
             dist.destroy_process_group()
         return
+    for name in workloads_to_run(args):
+        run_forward(args, WORKLOADS[name], dev, world, rank, barrier, max_over_ranks)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def run_forward(args, w, dev, world, rank, barrier, max_over_ranks):
+    """One forward line: dcnv4_forward over the workload's batch per step (per GPU), inputs rotating over
+    resident sets larger than L2; the end-to-end path through dcnv4_forward_host; the CPU oracle."""
+    import torch
+    import deformable_convolution_sparse_b200 as dcn
+    from deformable_convolution_sparse_b200.workloads import workload_inputs
+
     # weak scaling: rank r owns images [64 r, 64 (r+1)) of the global batch, drawn from seed + r
     wr = w.with_(seed=w.seed + 1000 * rank)
     x, om = workload_inputs(wr)
@@ -842,7 +898,7 @@ def main():
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "vs_baseline": None, "dtype": ARITH[w.dtype], "data": "synthetic",
             "config": {
                 "workload": workload_text(w),
                 "storage_dtype": w.dtype, "accumulate": "f32", "global_batch": w.N * world,
@@ -864,14 +920,12 @@ def main():
                     "steps": args.e2e_steps,
                     "h2d_bytes_per_step": (x.numel() + om.numel()) * x.element_size(),
                     "d2h_bytes_per_step": oh.numel() * oh.element_size(),
-                    "path": "dcnv4_forward_host: pinned host buffers, chunked H2D/kernel/D2H on two streams"},
+                    "path": "dcnv4_forward_host: pinned host buffers, chunked H2D/kernel/D2H on three streams"},
             "gpu_launches": timed_launches,
             "clocks": clocks,
             "cpu_baseline": base,
         }
         print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.destroy_process_group()
 
 
 if __name__ == "__main__":

@@ -31,9 +31,10 @@ TORCH_DTYPE = {torch.float32: DCNV4_F32, torch.float16: DCNV4_F16, torch.bfloat1
 
 # every symbol include/dcnv4.h declares
 EXPORTS = ("dcnv4_output_shape", "dcnv4_validate", "dcnv4_validate_ex", "dcnv4_forward", "dcnv4_forward_ex",
+           "dcnv4_forward_trace",
            "dcnv4_backward", "dcnv4_backward_ex", "dcnv4_predictor", "dcnv4_sampling_index",
-           "dcnv4_forward_host", "dcnv4_forward_host_noalloc", "dcnv4_device_status", "dcnv4_selftest_wait_timeout", "dcnv4_strerror",
-           "dcnv4_abi_version")
+           "dcnv4_forward_host", "dcnv4_forward_host_noalloc", "dcnv4_device_status", "dcnv4_selftest_wait_timeout",
+           "dcnv4_probe_smem_gather", "dcnv4_strerror", "dcnv4_abi_version")
 DEVSTATUS_COPY_TIMEOUT, DEVSTATUS_SELFTEST_TIMEOUT = 1, 2
 
 _lib = None
@@ -63,6 +64,8 @@ def load_library():
     lib.dcnv4_validate.restype = i
     lib.dcnv4_forward.argtypes = [p, p, p] + [i] * 9 + [f, i, p]
     lib.dcnv4_forward.restype = i
+    lib.dcnv4_forward_trace.argtypes = [p] * 4 + [i] * 9 + [f, i, p]
+    lib.dcnv4_forward_trace.restype = i
     lib.dcnv4_validate_ex.argtypes = [p] * 4 + [i] * 9 + [f, i, ctypes.c_uint]
     lib.dcnv4_validate_ex.restype = i
     lib.dcnv4_forward_ex.argtypes = [p] * 4 + [i] * 9 + [f, i, ctypes.c_uint, p]
@@ -83,6 +86,8 @@ def load_library():
     lib.dcnv4_device_status.restype = i
     lib.dcnv4_selftest_wait_timeout.argtypes = [ctypes.c_ulonglong, p]
     lib.dcnv4_selftest_wait_timeout.restype = i
+    lib.dcnv4_probe_smem_gather.argtypes = [i, ctypes.POINTER(ctypes.c_double)]
+    lib.dcnv4_probe_smem_gather.restype = i
     lib.dcnv4_strerror.argtypes = [i]
     lib.dcnv4_strerror.restype = ctypes.c_char_p
     lib.dcnv4_abi_version.argtypes = []
@@ -113,6 +118,15 @@ def selftest_wait_timeout(limit_ns: int = 1_000_000, stream=None) -> None:
     rc = load_library().dcnv4_selftest_wait_timeout(int(limit_ns), _stream_handle(stream))
     if rc != DCNV4_OK:
         raise DCNv4Error(rc, "dcnv4_selftest_wait_timeout")
+
+
+def probe_smem_gather(pattern: int = 0) -> float:
+    """Shared-memory gather bytes per SM clock per SM (dcnv4_probe_smem_gather; synchronous)."""
+    v = ctypes.c_double(0.0)
+    rc = load_library().dcnv4_probe_smem_gather(int(pattern), ctypes.byref(v))
+    if rc != DCNV4_OK:
+        raise DCNv4Error(rc, "dcnv4_probe_smem_gather")
+    return v.value
 
 
 def output_shape(H: int, W: int, K: int, stride: int = 1, pad: int = 0, dilation: int = 1):
@@ -408,3 +422,35 @@ def sampling_index(offset_mask: torch.Tensor, H: int, W: int, G: int, K: int, st
     if rc != DCNV4_OK:
         raise DCNv4Error(rc, "dcnv4_sampling_index")
     return corner, valid
+
+# path codes of forward_trace
+TRACE_WINDOW, TRACE_GLOBAL_PASS, TRACE_GATHER_KERNEL = 0, 1, 2
+
+
+def forward_trace(x: torch.Tensor, offset_mask: torch.Tensor, G: int, K: int, stride: int = 1, pad: int = 0,
+                  dilation: int = 1, offset_scale: float = 1.0, stream=None):
+    """The forward through ``dcnv4_forward_trace``: returns (out, trace).
+
+    out is what ``forward`` returns, bit for bit; trace [N,Hout,Wout,G,K*K,4]
+    int32 holds, per sampling point, the top-left corner (y0, x0) and the
+    validity bits that the gather used, and the path it took (0: the ring
+    kernel's shared-memory window, 1: its global-memory pass, 2: the
+    global-gather kernel).
+    """
+    _check_tensor(x, "x")
+    _check_tensor(offset_mask, "offset_mask")
+    if offset_mask.dtype != x.dtype or offset_mask.device != x.device:
+        raise ValueError("offset_mask must match x in dtype and device")
+    N, H, W, C = x.shape
+    Hout, Wout = output_shape(H, W, K, stride, pad, dilation)
+    if tuple(offset_mask.shape) != (N, Hout, Wout, G, 3 * K * K):
+        raise ValueError("offset_mask shape does not match H, W, G, K")
+    out = torch.empty((N, Hout, Wout, C), dtype=x.dtype, device=x.device)
+    trace = torch.empty((N, Hout, Wout, G, K * K, 4), dtype=torch.int32, device=x.device)
+    with torch.cuda.device(x.device):
+        rc = load_library().dcnv4_forward_trace(x.data_ptr(), offset_mask.data_ptr(), out.data_ptr(),
+                                                trace.data_ptr(), N, H, W, C, G, K, stride, pad, dilation,
+                                                float(offset_scale), TORCH_DTYPE[x.dtype], _stream_handle(stream))
+    if rc != DCNV4_OK:
+        raise DCNv4Error(rc, "dcnv4_forward_trace")
+    return out, trace

@@ -17,7 +17,9 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libdcnv4.so")
-SOURCES = [os.path.join(CSRC, "dcnv4.cu")]
+# the C ABI, and the forward of each storage type in a unit of its own (its kernel
+# specialisations compile in parallel with the others)
+SOURCES = [os.path.join(CSRC, f) for f in ("dcnv4.cu", "dcnv4_fwd_f32.cu", "dcnv4_fwd_f16.cu", "dcnv4_fwd_bf16.cu")]
 DEPS = SOURCES + [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".cuh", ".h", ".inl"))] + \
     [os.path.join(INCLUDE, "dcnv4.h")]
 
@@ -47,14 +49,33 @@ def stale() -> bool:
 def build(force: bool = False, verbose: bool = False) -> str:
     if not force and not stale():
         return LIB
-    tmp = LIB + ".tmp.%d" % os.getpid()
-    cmd = [nvcc(), *NVCC_FLAGS, "-shared", "-I", INCLUDE, "-I", CSRC, "-o", tmp, *SOURCES]
+    tmpdir = os.path.join(PKG, "_build")
+    os.makedirs(tmpdir, exist_ok=True)
+    tag = "%d" % os.getpid()
+    objs, procs = [], []
+    for src in SOURCES:
+        obj = os.path.join(tmpdir, os.path.basename(src) + "." + tag + ".o")
+        cmd = [nvcc(), *NVCC_FLAGS, "-c", "-I", INCLUDE, "-I", CSRC, "-o", obj, src]
+        procs.append((src, subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.PIPE, text=True)))
+        objs.append(obj)
+    failed = False
+    for src, proc in procs:
+        out, err = proc.communicate()
+        if proc.returncode != 0:
+            sys.stderr.write(out + err)
+            failed = True
+        elif verbose:
+            sys.stderr.write(err)
+    if failed:
+        raise RuntimeError("nvcc failed building libdcnv4.so")
+    tmp = LIB + ".tmp." + tag
+    cmd = [nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-o", tmp, *objs]
     res = subprocess.run(cmd, capture_output=True, text=True)
+    for o in objs:
+        os.remove(o)
     if res.returncode != 0:
         sys.stderr.write(res.stdout + res.stderr)
-        raise RuntimeError("nvcc failed building libdcnv4.so")
-    if verbose:
-        sys.stderr.write(res.stderr)
+        raise RuntimeError("nvcc failed linking libdcnv4.so")
     os.replace(tmp, LIB)
     return LIB
 

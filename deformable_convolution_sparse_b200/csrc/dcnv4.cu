@@ -16,10 +16,88 @@
 #include <cstring>
 
 #include "dcnv4.h"
+#include "dcnv4_async.cuh"
+#include "dcnv4_internal.h"
 #include "dcnv4_kernels.cuh"
-#include "dcnv4_window.cuh"
 #include "dcnv4_backward.cuh"
 #include "dcnv4_predictor.cuh"
+
+namespace dcnv4 {
+
+// Device-side status word (kStatus* bits), read and cleared from the host
+// through dcnv4_device_status(). The kernels of every translation unit get its
+// device address as a parameter.
+__device__ unsigned int g_device_status;
+
+// Self-test of the bounded wait: arms an mbarrier for 16 bytes that never
+// arrive (no copy is issued), waits `limit_ns`, records the timeout in
+// *status and returns. Nothing is in flight, so nothing faults or hangs.
+__global__ void selftest_wait_timeout_kernel(unsigned long long limit_ns, unsigned* status) {
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_barrier_init();
+        mbar_expect_tx(&bar, 16);
+        mbar_arrive(&bar);
+        if (!mbar_wait_bounded(&bar, 0, limit_ns)) atomicOr(status, kStatusSelftestTimeout);
+    }
+}
+
+// Shared-memory gather probe (dcnv4_probe_smem_gather): per CTA cycle counts.
+constexpr int kProbeMaxCtas = 1024;
+__device__ unsigned long long g_probe_cycles[kProbeMaxCtas];
+
+// Every thread reads 16-byte chunks of 128-byte shared-memory rows picked by a
+// per-thread linear congruential sequence (a power-of-two row count, so the
+// pick is a mask), each lane of a quarter warp at a different 16-byte bank
+// position: one 128-byte wavefront per quarter warp and load, whatever the
+// rows. pattern 0: one chunk per pick; pattern 1: the forward's gather, 2x2
+// corners x 2 chunks of a 128-byte pixel in a 26-pixel-wide window with the
+// chunk rotation of the ring kernel (8 loads per pick).
+__global__ void __launch_bounds__(512)
+probe_smem_gather_kernel(int pattern, int iters) {
+    extern __shared__ __align__(128) unsigned char psm[];
+    constexpr int kRows = 512;  // 64 KB
+    for (int i = threadIdx.x; i < kRows * 32; i += blockDim.x) reinterpret_cast<unsigned*>(psm)[i] = i * 2654435761u;
+    __syncthreads();
+    const int lane = threadIdx.x & 31;
+    unsigned s = 12345u + 977u * (blockIdx.x * blockDim.x + threadIdx.x);
+    unsigned acc = 0;
+    const unsigned long long t0 = clock64();
+    if (pattern == 0) {
+        for (int it = 0; it < iters; ++it) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                s = s * 1664525u + 1013904223u;
+                const unsigned off = ((s >> 9) & (kRows - 1)) * 128u + (((lane & 7) + j) & 7) * 16u;
+                const uint4 v = *reinterpret_cast<const uint4*>(psm + off);
+                acc ^= v.x ^ v.y ^ v.z ^ v.w;
+            }
+        }
+    } else {
+        // window of 19 x 26 pixels of 128 bytes; corners of a pixel at (r, c): +128, +26*128
+        const int gl = lane & 3, rot = (lane & 7) >> 2;
+        for (int it = 0; it < iters; ++it) {
+            s = s * 1664525u + 1013904223u;
+            const unsigned r = (s >> 10) % 18u, c = (s >> 20) % 25u;
+            const unsigned base = (r * 26u + c) * 128u + gl * 32u;
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const unsigned pc = base + ((rot + j) & 1) * 16u;
+                const uint4 a = *reinterpret_cast<const uint4*>(psm + pc);
+                const uint4 b = *reinterpret_cast<const uint4*>(psm + pc + 128u);
+                const uint4 c2 = *reinterpret_cast<const uint4*>(psm + pc + 26u * 128u);
+                const uint4 d = *reinterpret_cast<const uint4*>(psm + pc + 27u * 128u);
+                acc ^= a.x ^ b.y ^ c2.z ^ d.w ^ a.w ^ b.x ^ c2.y ^ d.z;
+            }
+        }
+    }
+    const unsigned long long t1 = clock64();
+    if (acc == 0x9e3779b9u) reinterpret_cast<unsigned*>(psm)[0] = acc;  // keeps the loads
+    if (threadIdx.x == 0) g_probe_cycles[blockIdx.x] = t1 - t0;
+}
+
+}  // namespace dcnv4
 
 namespace {
 
@@ -27,15 +105,30 @@ using dcnv4::FwdParams;
 
 #include "dcnv4_host_common.inl"
 
-#include "dcnv4_launch_forward.inl"
-
 #include "dcnv4_launch_backward.inl"
 
 #include "dcnv4_launch_predictor.inl"
 
-// Two non-blocking streams per device for the host-memory entry point,
-// created on first use and kept for the life of the process.
 constexpr int kMaxDevices = 64;
+
+// Device address of the status word on the current device, looked up once per
+// device (cudaGetSymbolAddress with that device current); NULL on failure.
+unsigned* status_word() {
+    static unsigned* addr[kMaxDevices];
+    static std::mutex mu;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, dcnv4::g_device_status) != cudaSuccess) return nullptr;
+        addr[dev] = static_cast<unsigned*>(p);
+    }
+    return addr[dev];
+}
+
+// Three non-blocking streams per device for the host-memory entry points,
+// created on first use and kept for the life of the process.
 struct HostPipe {
     cudaStream_t s[3] = {nullptr, nullptr, nullptr};
     bool ready = false;
@@ -72,6 +165,18 @@ FwdParams make_params(int N, int H, int W, int C, int G, int K, int stride, int 
     p.kc = rc ? (p.KK - 1) / 2 : p.KK;
     p.center_logit = center_logit;
     return p;
+}
+
+// The forward of one storage type through its translation unit.
+int run_forward(const void* x, const void* om, void* out, const FwdParams& p, int dtype, int4* trace,
+                cudaStream_t s) {
+    unsigned* status = status_word();
+    if (!status) return DCNV4_ERR_CUDA;
+    switch (dtype) {
+        case DCNV4_F32: return dcnv4_host::forward_f32(x, om, out, p, status, trace, s);
+        case DCNV4_F16: return dcnv4_host::forward_f16(x, om, out, p, status, trace, s);
+        default: return dcnv4_host::forward_bf16(x, om, out, p, status, trace, s);
+    }
 }
 
 // Points per unit for a flag set (K*K, or K*K - 1 without the centre).
@@ -161,12 +266,7 @@ int dcnv4_forward_ex(const void* x, const void* offset_mask, const void* center_
     dcnv4_output_shape(H, W, K, stride, pad, dilation, &Hout, &Wout);
     const FwdParams p = make_params(N, H, W, C, G, K, stride, pad, dilation, offset_scale, Hout, Wout, flags,
                                     (flags & DCNV4_FLAG_CENTER_SCALE) ? center_logit : nullptr);
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    switch (dtype) {
-        case DCNV4_F32: return launch_forward<float>(x, offset_mask, out, p, s);
-        case DCNV4_F16: return launch_forward<__half>(x, offset_mask, out, p, s);
-        default: return launch_forward<__nv_bfloat16>(x, offset_mask, out, p, s);
-    }
+    return run_forward(x, offset_mask, out, p, dtype, nullptr, static_cast<cudaStream_t>(stream));
 }
 
 int dcnv4_forward(const void* x, const void* offset_mask, void* out,
@@ -175,6 +275,47 @@ int dcnv4_forward(const void* x, const void* offset_mask, void* out,
                   void* stream) {
     return dcnv4_forward_ex(x, offset_mask, nullptr, out, N, H, W, C, G, K, stride, pad, dilation, offset_scale,
                             dtype, 0u, stream);
+}
+
+int dcnv4_forward_trace(const void* x, const void* offset_mask, void* out, int32_t* trace,
+                        int N, int H, int W, int C, int G, int K,
+                        int stride, int pad, int dilation, float offset_scale, int dtype,
+                        void* stream) {
+    const int rc = dcnv4_validate(x, offset_mask, out, N, H, W, C, G, K, stride, pad, dilation, offset_scale, dtype);
+    if (rc) return rc;
+    if (N == 0) return DCNV4_OK;
+    if (!trace) return DCNV4_ERR_NULL;
+    if (!aligned(trace, 16)) return DCNV4_ERR_ALIGN;
+    int Hout = 0, Wout = 0;
+    dcnv4_output_shape(H, W, K, stride, pad, dilation, &Hout, &Wout);
+    const int e = elem_size(dtype);
+    const long long npts = static_cast<long long>(N) * Hout * Wout * G * K * K;
+    if (4 * npts >= kLimit) return DCNV4_ERR_TOO_LARGE;
+    const long long nx = static_cast<long long>(N) * H * W * C, nout = static_cast<long long>(N) * Hout * Wout * C;
+    if (overlap(trace, 16 * npts, x, nx * e) || overlap(trace, 16 * npts, offset_mask, 3 * npts * e) ||
+        overlap(trace, 16 * npts, out, nout * e))
+        return DCNV4_ERR_ALIAS;
+    const FwdParams p = make_params(N, H, W, C, G, K, stride, pad, dilation, offset_scale, Hout, Wout);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int4* tr = reinterpret_cast<int4*>(trace);
+    const int frc = run_forward(x, offset_mask, out, p, dtype, tr, s);
+    if (frc != DCNV4_NOT_TRACED) return frc;
+    // the global-gather kernel ran: trace its sampling with the code it shares
+    const long long want = (npts + 255) / 256;
+    const unsigned blocks = static_cast<unsigned>(want < 148 * 32 ? want : 148 * 32);
+    switch (dtype) {
+        case DCNV4_F32:
+            dcnv4::trace_index_kernel<float><<<blocks, 256, 0, s>>>(static_cast<const float*>(offset_mask), tr, p);
+            break;
+        case DCNV4_F16:
+            dcnv4::trace_index_kernel<__half><<<blocks, 256, 0, s>>>(static_cast<const __half*>(offset_mask), tr, p);
+            break;
+        default:
+            dcnv4::trace_index_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(
+                static_cast<const __nv_bfloat16*>(offset_mask), tr, p);
+            break;
+    }
+    return launch_status();
 }
 
 int dcnv4_backward_ex(const void* x, const void* offset_mask, const void* center_logit, const void* grad_out,
@@ -250,6 +391,8 @@ int dcnv4_predictor(const void* y, const void* weight, const float* bias, void* 
         return DCNV4_ERR_ALIAS;
     dcnv4::PredParams p{};
     p.M = M; p.C = C; p.G = G; p.P = static_cast<int>(P); p.NO = static_cast<int>(NO);
+    p.status = status_word();
+    if (!p.status) return DCNV4_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     switch (dtype) {
         case DCNV4_F32: return launch_predictor<float>(y, weight, bias, offset_mask, p, s);
@@ -288,7 +431,19 @@ int dcnv4_forward_host(const void* x_host, const void* offset_mask_host, void* o
     if (const char* c = std::getenv("DCNV4_HOST_CHUNKS")) max_chunks = std::max(1, std::atoi(c));
     if (const char* c = std::getenv("DCNV4_HOST_STREAMS")) NS = std::min(3, std::max(1, std::atoi(c)));
     cudaEvent_t ev_start = nullptr, ev_done[3] = {nullptr, nullptr, nullptr};
+    bool queued = false;  // copies or kernels are on the library's streams
+    // Ends the call: once anything is queued the caller's stream waits for all
+    // of it, on success and after an error alike, so that no copy into out_host
+    // is still pending when the caller's stream moves on.
     auto fail = [&](int code) {
+        if (queued) {
+            for (int i = 0; i < NS; ++i) {
+                const bool ok = ev_done[i] && cudaEventRecord(ev_done[i], pipe->s[i]) == cudaSuccess &&
+                                cudaStreamWaitEvent(user, ev_done[i], 0) == cudaSuccess;
+                if (!ok && code == DCNV4_OK) code = DCNV4_ERR_CUDA;
+            }
+        }
+        // events may be destroyed while pending: the waits already queued keep their meaning
         if (ev_start) cudaEventDestroy(ev_start);
         for (auto& ev : ev_done)
             if (ev) cudaEventDestroy(ev);
@@ -318,6 +473,7 @@ int dcnv4_forward_host(const void* x_host, const void* offset_mask_host, void* o
         const int nc = n1 - n0;
         if (nc == 0) continue;
         cudaStream_t s = pipe->s[c % NS];
+        queued = true;
         if (cudaMemcpyAsync(xd + n0 * x_img, xh + n0 * x_img, nc * x_img, cudaMemcpyHostToDevice, s) != cudaSuccess ||
             cudaMemcpyAsync(omd + n0 * om_img, omh + n0 * om_img, nc * om_img, cudaMemcpyHostToDevice, s) != cudaSuccess)
             return fail(DCNV4_ERR_CUDA);
@@ -328,13 +484,7 @@ int dcnv4_forward_host(const void* x_host, const void* offset_mask_host, void* o
             return fail(DCNV4_ERR_CUDA);
         n0 = n1;
     }
-    for (int i = 0; i < NS; ++i) {
-        if (cudaEventRecord(ev_done[i], pipe->s[i]) != cudaSuccess || cudaStreamWaitEvent(user, ev_done[i], 0) != cudaSuccess)
-            return fail(DCNV4_ERR_CUDA);
-    }
-    // events may be destroyed while pending: the waits already queued keep their meaning
-    fail(DCNV4_OK);
-    return DCNV4_OK;
+    return fail(DCNV4_OK);
 }
 
 int dcnv4_device_status(unsigned int* status, int clear) {
@@ -351,8 +501,35 @@ int dcnv4_device_status(unsigned int* status, int clear) {
 
 int dcnv4_selftest_wait_timeout(unsigned long long limit_ns, void* stream) {
     if (limit_ns == 0 || limit_ns > 2000000000ull) return DCNV4_ERR_SHAPE;
-    dcnv4::selftest_wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns);
+    unsigned* status = status_word();
+    if (!status) return DCNV4_ERR_CUDA;
+    dcnv4::selftest_wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns, status);
     return launch_status();
+}
+
+int dcnv4_probe_smem_gather(int pattern, double* bytes_per_clock_per_sm) {
+    if (!bytes_per_clock_per_sm) return DCNV4_ERR_NULL;
+    if (pattern != 0 && pattern != 1) return DCNV4_ERR_SHAPE;
+    const int nsm = sm_count();
+    if (nsm <= 0 || nsm > dcnv4::kProbeMaxCtas) return DCNV4_ERR_CUDA;
+    constexpr int threads = 512, iters = 2048;
+    const size_t smem = 512 * 128;
+    if (cudaFuncSetAttribute(dcnv4::probe_smem_gather_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+        return DCNV4_ERR_CUDA;
+    unsigned long long cyc[dcnv4::kProbeMaxCtas];
+    for (int rep = 0; rep < 2; ++rep) {  // the first launch warms up
+        dcnv4::probe_smem_gather_kernel<<<nsm, threads, smem>>>(pattern, iters);
+        if (cudaGetLastError() != cudaSuccess) return DCNV4_ERR_LAUNCH;
+        if (cudaDeviceSynchronize() != cudaSuccess) return DCNV4_ERR_CUDA;
+    }
+    if (cudaMemcpyFromSymbol(cyc, dcnv4::g_probe_cycles, sizeof(unsigned long long) * nsm) != cudaSuccess)
+        return DCNV4_ERR_CUDA;
+    unsigned long long mx = 1;
+    for (int i = 0; i < nsm; ++i) mx = std::max(mx, cyc[i]);
+    const double loads = static_cast<double>(threads) * iters * 8.0;  // 16-byte loads per CTA
+    *bytes_per_clock_per_sm = loads * 16.0 / static_cast<double>(mx);
+    return DCNV4_OK;
 }
 
 int dcnv4_sampling_index(const void* offset_mask, int32_t* corner, uint8_t* valid,
@@ -457,7 +634,17 @@ extern "C" int dcnv4_forward_host_noalloc(const void* x_host, const void* offset
     if (rc) return rc;
     cudaStream_t user = static_cast<cudaStream_t>(stream);
     cudaEvent_t ev_start = nullptr, ev_done[2] = {nullptr, nullptr};
+    bool queued = false;  // copies or kernels are on the library's streams
+    // Ends the call: once anything is queued the caller's stream waits for all
+    // of it, on success and after an error alike (see dcnv4_forward_host).
     auto release = [&](int code) {
+        if (queued) {
+            for (int i = 0; i < 2; ++i) {
+                const bool ok = ev_done[i] && cudaEventRecord(ev_done[i], pipe->s[i]) == cudaSuccess &&
+                                cudaStreamWaitEvent(user, ev_done[i], 0) == cudaSuccess;
+                if (!ok && code == DCNV4_OK) code = DCNV4_ERR_CUDA;
+            }
+        }
         if (ev_start) cudaEventDestroy(ev_start);
         for (auto& ev : ev_done)
             if (ev) cudaEventDestroy(ev);
@@ -482,16 +669,13 @@ extern "C" int dcnv4_forward_host_noalloc(const void* x_host, const void* offset
         unsigned char* omd = xd + round256(nc * x_img);
         unsigned char* od = omd + round256(nc * om_img);
         cudaStream_t s = pipe->s[c & 1];
+        queued = true;
         if (cudaMemcpyAsync(xd, xh + n0 * x_img, nc * x_img, cudaMemcpyHostToDevice, s) != cudaSuccess ||
             cudaMemcpyAsync(omd, omh + n0 * om_img, nc * om_img, cudaMemcpyHostToDevice, s) != cudaSuccess)
             return release(DCNV4_ERR_CUDA);
         rc = dcnv4_forward(xd, omd, od, nc, H, W, C, G, K, stride, pad, dilation, offset_scale, dtype, s);
         if (rc) return release(rc);
         if (cudaMemcpyAsync(oh + n0 * out_img, od, nc * out_img, cudaMemcpyDeviceToHost, s) != cudaSuccess)
-            return release(DCNV4_ERR_CUDA);
-    }
-    for (int i = 0; i < 2; ++i) {
-        if (cudaEventRecord(ev_done[i], pipe->s[i]) != cudaSuccess || cudaStreamWaitEvent(user, ev_done[i], 0) != cudaSuccess)
             return release(DCNV4_ERR_CUDA);
     }
     return release(DCNV4_OK);

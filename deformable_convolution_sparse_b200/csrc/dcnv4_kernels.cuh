@@ -472,4 +472,27 @@ sampling_index_kernel(const T* __restrict__ om, int32_t* __restrict__ corner, ui
     }
 }
 
+// Trace of the global-gather kernel's sampling (a shape the ring kernel does not
+// take): per sampling point (y0, x0, validity bits, path 2), computed by the
+// same `locate` that kernel uses.
+template <typename T>
+__global__ void __launch_bounds__(256)
+trace_index_kernel(const T* __restrict__ om, int4* __restrict__ trace, FwdParams p) {
+    const int KK = p.KK;
+    const long long total = static_cast<long long>(p.units) * KK;
+    for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
+         i += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const int unit = static_cast<int>(i / KK);
+        const int k = static_cast<int>(i - static_cast<long long>(unit) * KK);
+        int n, ho, wo, g;
+        unit_coords(unit, p, n, ho, wo, g);
+        const T* rec = om + static_cast<size_t>(unit) * 3 * KK;
+        const int ky = k / p.K, kx = k - (k / p.K) * p.K;
+        const Sample s = locate(ho * p.stride - p.pad + ky * p.dilation, wo * p.stride - p.pad + kx * p.dilation,
+                                ElemTraits<T>::to_float(rec[KK + k]), ElemTraits<T>::to_float(rec[k]),
+                                p.offset_scale, p.H, p.W);
+        trace[i] = make_int4(s.bits ? s.y0 : INT32_MIN, s.bits ? s.x0 : INT32_MIN, static_cast<int>(s.bits), 2);
+    }
+}
+
 }  // namespace dcnv4

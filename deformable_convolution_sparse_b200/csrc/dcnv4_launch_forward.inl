@@ -1,12 +1,14 @@
-// Launcher of the forward aggregation: kernel choice, the tile kernel's planner
-// (group subset, tile, halo, tensor map of x) and the dispatch over the
-// kernels' template specialisations. Included by dcnv4.cu inside its anonymous
+// Launcher of the forward aggregation: kernel choice, the ring kernel's planner
+// (group subset, band width, item height, halo, ring depth, tensor map of x)
+// and the dispatch over the kernels' template specialisations. Included by the
+// per-storage-type translation units (dcnv4_fwd_*.cu) inside their anonymous
 // namespace, after dcnv4_host_common.inl.
 
 // Kernel choice: DCNV4_VARIANT=gather forces the global-gather kernel (A/B
-// comparisons); unset or anything else selects the persistent shared-memory
-// tile kernel whenever the shape allows it. DCNV4_HALO overrides the window
-// halo (pixels) and DCNV4_TILE=<TH>x<TW> the output tile, for tuning runs.
+// comparisons); unset or anything else selects the ring kernel whenever the
+// shape allows it. Tuning overrides of the planner: DCNV4_HALO (pixels),
+// DCNV4_TILE=<TH>x<TW> (item rows x band columns), DCNV4_GS (groups per
+// strip), DCNV4_NREC (items in flight, 2..4), DCNV4_RING (ring rows).
 enum class Variant { Auto, Gather };
 
 Variant variant_from_env() {
@@ -15,14 +17,19 @@ Variant variant_from_env() {
     return Variant::Auto;
 }
 
+int env_int(const char* name, int dflt) {
+    const char* v = std::getenv(name);
+    return (v && *v) ? std::atoi(v) : dflt;
+}
+
 // consumer threads (15 warps) per CTA, plus one producer warp: 16 warps, 4 per SM
 // sub-partition, whose 16 K registers then hold 4 warps at the kernel's 112-register cap
 // (a 17th warp would put 5 on one sub-partition: 17,920 registers, and the CTA would not launch)
-constexpr int kTileUnitsMax = 480;
-static_assert(((kTileUnitsMax / 32 + 1 + 3) / 4) * 112 * 32 <= 16384,
-              "the tile kernel's register cap must fit the warps of one SM sub-partition");
+constexpr int kUnitsMax = 480;
+static_assert(((kUnitsMax / 32 + 1 + 3) / 4) * 112 * 32 <= 16384,
+              "the ring kernel's register cap must fit the warps of one SM sub-partition");
 
-// Mean shared-memory wavefronts of one quarter-warp LDS.128 in the tile
+// Mean shared-memory wavefronts of one quarter-warp LDS.128 in the ring
 // kernel's gather, for window pixels of GS groups x Q chunks (PB = 16 GS Q
 // bytes). A quarter warp is 8 consecutive units: ceil(8 / GS) pixels at
 // independent window positions, each read at the lane's rotated chunk (the
@@ -69,39 +76,63 @@ double gather_wavefronts(int Q, int GS) {
     return w;
 }
 
-struct TilePlan {
-    dcnv4::TileParams p;
+// Smallest odd multiple of 16 that holds `bytes`: consecutive record slots
+// then start on different 16-byte bank positions, so the record reads of a
+// warp's pixels do not all fall on the same banks.
+int odd16(int bytes) {
+    int s = (bytes + 15) / 16;
+    if ((s & 1) == 0) ++s;
+    return s * 16;
+}
+
+// The halo the planner aims for: samples whose corners stay within R pixels of
+// their unit's grid footprint are gathered from shared memory, so R bounds the
+// offsets served from the window. It grows with the dilation (the spacing of
+// the grid the offsets move around): 6 pixels at dilation 1, 9 at 2 and more.
+int default_halo(int dilation) { return std::min(9, 4 * dilation + 2); }
+
+struct RingPlan {
+    dcnv4::RingParams p;
     CUtensorMap map;
     size_t smem;
     int threads;
 };
 
-// Chooses group subset, tile and halo for the tile kernel and encodes the
-// tensor map of x; false when the shape or the alignment does not suit it.
+struct RingShape {  // one candidate of the planner
+    int GS, R, TW, TH, nrec, NR, units, threads, slot, rec, WW, UH, c2;
+    size_t smem;
+    double score;
+};
+
+// The best plan for halo R (score < 0: none fits). Everything but R leaves the
+// per-unit arithmetic unchanged; it is chosen for speed and may depend on N.
+// The score multiplies estimated efficiencies: filled columns and rows,
+// shared-memory wavefronts of the gather, active warps, the window width
+// against the band (L2 -> SM traffic), record-buffer depth, and the part of a
+// CTA's time spent waiting for windows:
+//  - the ring should hold the current window plus the next item's rows
+//    (NR >= nrows + TH*stride), else every item waits for its own rows;
+//  - a CTA whose row range crosses into a new strip loads a whole window
+//    there; with NR >= 2*nrows that load overlaps the last items of the
+//    previous strip, else the CTA waits for it (about 1500 cycles plus the
+//    window's bytes at 100 B per cycle from L2), against about
+//    (0.75*Q + 0.5) cycles of SM time per sampling point.
 template <typename T>
-bool plan_tile(const void* x, const void* om, const void* out, const FwdParams& f, TilePlan* plan) {
+RingShape best_ring_shape(const FwdParams& f, int R, int nsm) {
     constexpr int E = sizeof(T);
     const int row_bytes = f.Cg * E;
-    if (!aligned(x, 16) || !aligned(out, 16) || (f.C * E) % 16 || row_bytes % 16) return false;
     const int Q = row_bytes / 16;
-    if (!(Q == 1 || Q == 2 || Q == 4 || Q == 5 || Q == 8)) return false;
-    if (f.KK > 64) return false;  // the per-unit mask of points outside the window has 64 bits
-    int R = 5;
-    if (const char* h = std::getenv("DCNV4_HALO")) R = std::atoi(h) > 0 ? std::atoi(h) : R;
-    int forceTH = 0, forceTW = 0, forceGS = 0, forceNrec = 0;
-    if (const char* n = std::getenv("DCNV4_NREC")) forceNrec = (std::atoi(n) == 2 || std::atoi(n) == 3) ? std::atoi(n) : 0;
-    if (const char* t = std::getenv("DCNV4_TILE")) std::sscanf(t, "%dx%d", &forceTH, &forceTW);
-    if (const char* g = std::getenv("DCNV4_GS")) forceGS = std::atoi(g);
     const int R3 = 3 * f.npts;
-    const int nsm = sm_count();
-    if (nsm <= 0) return false;
-
-    static const int THs[] = {1, 2, 4, 7, 8, 14, 16, 28, 32};
-    static const int TWs[] = {1, 2, 4, 7, 8, 14, 16, 28, 32};
-    double best = -1.0;
-    dcnv4::TileParams bp{};
-    int best_threads = 0, best_c2 = 0;
-    size_t best_smem = 0;
+    int forceTH = 0, forceTW = 0;
+    if (const char* t = std::getenv("DCNV4_TILE")) std::sscanf(t, "%dx%d", &forceTH, &forceTW);
+    const int forceGS = env_int("DCNV4_GS", 0);
+    const int forceNrec = env_int("DCNV4_NREC", 0);
+    const int forceNR = env_int("DCNV4_RING", 0);
+    const int s = f.stride;
+    const int UH = (f.K - 1) * f.dilation + 2 * R + 1;
+    RingShape best{};
+    best.score = -1.0;
+    static const int TWs[] = {1, 2, 4, 7, 8, 14, 16, 28, 32, 56, 64};
     for (int GS = 1; GS <= f.G; ++GS) {
         if (f.G % GS || (forceGS && GS != forceGS)) continue;
         const int PB = GS * row_bytes;
@@ -112,105 +143,157 @@ bool plan_tile(const void* x, const void* om, const void* out, const FwdParams& 
         if (c2 == 0 || sub_ch / c2 > 256) continue;
         // a pixel stride that is a multiple of 128 bytes keeps the gathers free of
         // bank conflicts (see the kernel); other strides pay in extra wavefronts.
-        // The gather's shared-memory reads dominate a tile's cost there, and the
-        // squared factor matches the measured 1.21x between 80- and 160-byte
-        // pixels of the 40-channel groups (2.60 vs 2.13 wavefronts), against
-        // which the window-reuse and ring-depth terms would otherwise win.
+        // The squared factor matches the measured 1.21x between 80- and 160-byte
+        // pixels of the 40-channel groups (2.60 vs 2.13 wavefronts).
         const double w = gather_wavefronts(Q, GS);
         const double banks = 1.0 / (w * w);
         const bool row_runs = GS == f.G;
-        for (int TH : THs) {
-            for (int TW : TWs) {
-                if (forceTH && (TH != forceTH || TW != forceTW)) continue;
+        for (int TW : TWs) {
+            if (forceTW && TW != forceTW) continue;
+            if (TW > f.Wout && TW != TWs[0]) {
+                // one band wider than the image only if no narrower TW covers it
+                bool smaller = false;
+                for (int t2 : TWs) smaller = smaller || (t2 < TW && t2 >= f.Wout);
+                if (smaller) continue;
+            }
+            const int WW = (TW - 1) * s + UH;
+            if (WW > 256) continue;
+            const int rowB = (WW * PB + 127) / 128 * 128;  // ring row pitch: every TMA destination 128-byte aligned
+            const int bands = (f.Wout + TW - 1) / TW;
+            const double fill_w = static_cast<double>(f.Wout) / (static_cast<double>(bands) * TW);
+            for (int TH = 1; TH <= 16; ++TH) {
+                if (forceTH && TH != forceTH) continue;
+                if (TH > f.Hout) break;
                 const int units = TH * TW * GS;
-                if (units > kTileUnitsMax || units < 32) continue;
-                if (TH > f.Hout + 7 || TW > f.Wout + 7) continue;
-                const int WH = (TH - 1) * f.stride + (f.K - 1) * f.dilation + 2 * R + 1;
-                const int WW = (TW - 1) * f.stride + (f.K - 1) * f.dilation + 2 * R + 1;
-                if (WH > 256 || WW > 256) continue;
-                const int nruns = row_runs ? TH : TH * TW;
-                const int count = (row_runs ? TW * f.G : GS) * R3;
-                const int slot = (count * E + 32 + 15) / 16 * 16;
-                const size_t rec = (static_cast<size_t>(nruns) * slot + 127) / 128 * 128;
-                const size_t win = (static_cast<size_t>(WH) * WW * PB + 127) / 128 * 128;
-                // records get a third buffer (a longer lead for their DRAM reads) when it fits
-                int nrec = (2 * win + 3 * rec <= kTileSmemLimit) ? 3 : 2;
-                if (forceNrec) nrec = forceNrec;
-                const size_t smem = 2 * win + nrec * rec;
-                if (smem > kTileSmemLimit) continue;
-                const int threads = (units + 31) / 32 * 32 + 32;  // consumers + the producer warp
-                const int tiles_y = (f.Hout + TH - 1) / TH, tiles_x = (f.Wout + TW - 1) / TW;
-                const long long tiles = static_cast<long long>(f.N) * tiles_y * tiles_x * (f.G / GS);
-                // the choice must not depend on N: an image's result (which samples take
-                // the window path) then never depends on the batch it comes in. The wave
-                // balance is judged for a nominal batch of 64 images.
-                const long long tiles_nominal = 64LL * tiles_y * tiles_x * (f.G / GS);
-                const int per_sm = std::max(1, static_cast<int>(std::min<size_t>(
-                                                   (kTileSmemLimit + 2048) / (smem + 1024), 2048 / threads)));
-                const double slots = static_cast<double>(nsm) * per_sm;
-                const double waves = static_cast<double>(tiles_nominal) / slots;
-                const double balance = waves / std::ceil(waves);
-                const double useful =
-                    static_cast<double>(f.Hout) * f.Wout / (static_cast<double>(tiles_y) * TH * tiles_x * TW);
-                const double reuse = static_cast<double>(TH * TW) / (static_cast<double>(WH) * WW);
-                const double fill = static_cast<double>(units) / (threads - 32);
-                const double occ = std::min(1.0, per_sm * (threads - 32) / 384.0);
-                const double depth = nrec == 3 ? 1.0 : 0.9;
-                // a ragged tile loses threads and still loads a full window: useful counts twice
-                const double score = useful * useful * balance * fill * occ * banks * depth * std::sqrt(reuse);
-                if (score > best) {
-                    best = score;
-                    bp.TH = TH; bp.TW = TW; bp.tiles_x = tiles_x; bp.tiles_y = tiles_y;
-                    bp.WH = WH; bp.WW = WW; bp.run_slot = slot; bp.rec_bytes = static_cast<int>(rec);
-                    bp.win_bytes = static_cast<int>(win);
-                    bp.nrec = nrec;
-                    bp.tiles = static_cast<int>(tiles); bp.units = units;
-                    bp.GS = GS; bp.PB = PB; bp.cblk = sub_ch / c2;
-                    best_threads = threads;
-                    best_smem = smem;
-                    best_c2 = c2;
+                if (units > kUnitsMax) break;
+                if (units < 32) continue;
+                const int nrows = (TH - 1) * s + UH;
+                const int slot = odd16((row_runs ? TW * f.G : GS) * R3 * E + 32);
+                const int rec = ((row_runs ? TH : TH * TW) * slot + 127) / 128 * 128;
+                for (int nrec = 2; nrec <= 4; ++nrec) {
+                    if (forceNrec ? nrec != forceNrec : nrec == 4) continue;
+                    const long long avail = static_cast<long long>(kTileSmemLimit) - static_cast<long long>(nrec) * rec;
+                    if (avail <= 0) continue;
+                    int NR = static_cast<int>(avail / rowB) - 1;  // one mirror row
+                    NR = std::min(NR, 2 * nrows);                 // deeper never helps
+                    if (forceNR) NR = std::min(NR, forceNR);
+                    if (NR < nrows) continue;
+                    const size_t smem = (static_cast<size_t>(NR + 1) * rowB + 127) / 128 * 128 +
+                                        static_cast<size_t>(nrec) * rec;
+                    if (smem > kTileSmemLimit) continue;
+                    const int threads = (units + 31) / 32 * 32 + 32;
+                    // a new strip's window loaded while the last one is still read
+                    // (NR >= 2 nrows), or at least the next item's rows (NR >= nrows + TH s)
+                    double prefetch = NR >= nrows + TH * s ? 1.0 : 0.5;
+                    if (NR < 2 * nrows) {
+                        const int bands_ = (f.Wout + TW - 1) / TW;
+                        const double rows_per_cta = static_cast<double>(f.N) * bands_ * (f.G / GS) * f.Hout / nsm;
+                        const double compute = rows_per_cta * TW * GS * f.npts * (0.75 * Q + 0.5);
+                        const double stall = rows_per_cta / f.Hout * (1500.0 + static_cast<double>(nrows) * rowB / 100.0);
+                        prefetch *= compute / (compute + stall);
+                    }
+                    const int tiles_h = (f.Hout + TH - 1) / TH;
+                    const double fill_h = static_cast<double>(f.Hout) / (static_cast<double>(tiles_h) * TH);
+                    const double occ = std::min(1.0, (threads - 32) / 384.0);
+                    const double l2 = std::sqrt(std::sqrt(static_cast<double>(TW * s) / WW));
+                    (void)nsm;
+                    const double depth = nrec >= 3 ? 1.0 : 0.97;
+                    const double score = fill_w * fill_w * fill_h * banks * prefetch * occ * l2 * depth;
+                    if (score > best.score) {
+                        best = RingShape{GS, R, TW, TH, nrec, NR, units, threads, slot, rec, WW, UH, c2, smem, score};
+                    }
                 }
             }
         }
     }
-    if (best < 0) return false;
-    const int GS = bp.GS, PB = bp.PB, c2 = best_c2;
+    return best;
+}
+
+// Chooses the halo, group subset, band, item height and ring depth for the
+// ring kernel and encodes the tensor map of x; false when the shape or the
+// alignment does not suit it. The halo (the only choice that changes which
+// samples take the window path) depends on the geometry alone, so an image's
+// result never depends on the batch it comes in.
+template <typename T>
+bool plan_ring(const void* x, const void* om, const void* out, const FwdParams& f, unsigned* status, int4* trace,
+               RingPlan* plan) {
+    constexpr int E = sizeof(T);
+    const int row_bytes = f.Cg * E;
+    if (!aligned(x, 16) || !aligned(out, 16) || (f.C * E) % 16 || row_bytes % 16) return false;
+    const int Q = row_bytes / 16;
+    if (!(Q == 1 || Q == 2 || Q == 4 || Q == 5 || Q == 8)) return false;
+    if (f.KK > 64) return false;  // the per-unit mask of points outside the window has 64 bits
+    const int nsm = sm_count();
+    if (nsm <= 0) return false;
+    int Rhi = default_halo(f.dilation), Rlo = 1;
+    if (const int h = env_int("DCNV4_HALO", 0); h > 0) Rhi = Rlo = h;
+    // the largest halo whose best plan keeps at least 8 consumer warps busy (or
+    // covers a whole item of a small image), judged for a nominal batch of 64
+    // images and 148 SMs so that the halo does not depend on N
+    int R = -1;
+    FwdParams nominal = f;
+    nominal.N = 64;
+    for (int r = Rhi; r >= Rlo && R < 0; --r) {
+        const RingShape c = best_ring_shape<T>(nominal, r, 148);
+        if (c.score >= 0.0 && (c.units >= 256 || r == Rlo || c.units >= f.Hout * f.Wout * f.G)) R = r;
+    }
+    if (R < 0) return false;
+    const RingShape sh = best_ring_shape<T>(f, R, nsm);
+    if (sh.score < 0.0) return false;
+
+    dcnv4::RingParams bp{};
     bp.f = f;
-    bp.nsub = f.G / GS;
-    bp.R = R;
-    const size_t om_bytes = static_cast<size_t>(f.N) * f.Hout * f.Wout * f.G * R3 * E;
+    bp.TH = sh.TH; bp.TW = sh.TW; bp.GS = sh.GS; bp.nsub = f.G / sh.GS; bp.R = sh.R;
+    bp.UH = sh.UH; bp.UW = sh.UH; bp.WW = sh.WW; bp.NR = sh.NR;
+    bp.PB = sh.GS * row_bytes;
+    bp.rowB = (sh.WW * bp.PB + 127) / 128 * 128;
+    bp.cblk = sh.GS * f.Cg / sh.c2;
+    bp.bands = (f.Wout + sh.TW - 1) / sh.TW;
+    const long long rows_total = static_cast<long long>(f.N) * bp.bands * bp.nsub * f.Hout;
+    if (rows_total >= (1LL << 31)) return false;
+    bp.rows_total = static_cast<int>(rows_total);
+    bp.units = sh.units;
+    bp.run_slot = sh.slot;
+    bp.rec_bytes = sh.rec;
+    bp.ring_bytes = static_cast<int>((static_cast<size_t>(sh.NR + 1) * bp.rowB + 127) / 128 * 128);
+    bp.nrec = sh.nrec;
+    const size_t om_bytes = static_cast<size_t>(f.N) * f.Hout * f.Wout * f.G * 3 * f.npts * E;
     bp.om_lo = reinterpret_cast<unsigned long long>(om);
     bp.om_hi = bp.om_lo + om_bytes;
-    bp.div_tw_gs = dcnv4::make_fastdiv(bp.TW * GS);
-    bp.div_gs = dcnv4::make_fastdiv(GS);
+    bp.div_tw_gs = dcnv4::make_fastdiv(sh.TW * sh.GS);
+    bp.div_gs = dcnv4::make_fastdiv(sh.GS);
     bp.div_nsub = dcnv4::make_fastdiv(bp.nsub);
-    bp.div_tx = dcnv4::make_fastdiv(bp.tiles_x);
-    bp.div_ty = dcnv4::make_fastdiv(bp.tiles_y);
+    bp.div_bands = dcnv4::make_fastdiv(bp.bands);
+    bp.div_hout = dcnv4::make_fastdiv(f.Hout);
+    bp.status = status;
+    bp.trace = trace;
 
     auto encode = tensor_map_encoder();
     if (!encode) return false;
+    const int c2 = sh.c2;
     const cuuint64_t dims[5] = {static_cast<cuuint64_t>(c2), static_cast<cuuint64_t>(f.C / c2),
                                 static_cast<cuuint64_t>(f.W), static_cast<cuuint64_t>(f.H),
                                 static_cast<cuuint64_t>(f.N)};
     const cuuint64_t strides[4] = {static_cast<cuuint64_t>(c2) * E, static_cast<cuuint64_t>(f.C) * E,
                                    static_cast<cuuint64_t>(f.W) * f.C * E,
                                    static_cast<cuuint64_t>(f.H) * f.W * f.C * E};
+    // one ring row per load: WW pixels of GS*Cg channels
     const cuuint32_t box[5] = {static_cast<cuuint32_t>(c2), static_cast<cuuint32_t>(bp.cblk),
-                               static_cast<cuuint32_t>(bp.WW), static_cast<cuuint32_t>(bp.WH), 1u};
+                               static_cast<cuuint32_t>(sh.WW), 1u, 1u};
     const cuuint32_t estr[5] = {1u, 1u, 1u, 1u, 1u};
     if (encode(&plan->map, tma_dtype<T>(), 5, const_cast<void*>(x), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return false;
     plan->p = bp;
-    plan->smem = best_smem;
-    plan->threads = best_threads;
+    plan->smem = sh.smem;
+    plan->threads = sh.threads;
     if (const char* d = std::getenv("DCNV4_DEBUG"); d && *d == '1')
         std::fprintf(stderr,
-                     "dcnv4 tile plan: tile %dx%d GS %d (nsub %d) R %d window %dx%d PB %d cblk %d tiles %d units %d "
-                     "threads %d nrec %d smem %zu\n",
-                     bp.TH, bp.TW, GS, bp.nsub, R, bp.WH, bp.WW, PB, bp.cblk, bp.tiles, bp.units, best_threads,
-                     bp.nrec, best_smem);
+                     "dcnv4 ring plan: item %dx%d GS %d (nsub %d) R %d unit window %d window width %d PB %d "
+                     "ring %d rows rows_total %d units %d threads %d nrec %d smem %zu score %.3f\n",
+                     bp.TH, bp.TW, bp.GS, bp.nsub, bp.R, bp.UH, bp.WW, bp.PB, bp.NR, bp.rows_total, bp.units,
+                     sh.threads, bp.nrec, sh.smem, sh.score);
     return true;
 }
 
@@ -221,9 +304,9 @@ bool f16_exact_from_env() {
     return v && *v == '1';
 }
 
-template <typename T, int Q, int KS, bool HW, int PBC, bool VF = false>
-int launch_tile_q(const T* x, const T* om, T* out, const TilePlan& plan, cudaStream_t stream) {
-    auto kern = dcnv4::fwd_tile_kernel<T, Q, KS, HW, PBC, VF>;
+template <typename T, int Q, int KS, bool HW, int PBC, bool VF, bool TRACE>
+int launch_ring_q(const T* x, const T* om, T* out, const RingPlan& plan, cudaStream_t stream) {
+    auto kern = dcnv4::fwd_ring_kernel<T, Q, KS, HW, PBC, VF, TRACE>;
     static std::once_flag once;
     static cudaError_t attr = cudaSuccess;
     std::call_once(once, [&] {
@@ -231,74 +314,67 @@ int launch_tile_q(const T* x, const T* om, T* out, const TilePlan& plan, cudaStr
     });
     const bool dbg = std::getenv("DCNV4_DEBUG") != nullptr;
     if (attr != cudaSuccess) {
-        if (dbg) std::fprintf(stderr, "dcnv4 tile launch: shared-memory attribute: %s\n", cudaGetErrorString(attr));
+        if (dbg) std::fprintf(stderr, "dcnv4 ring launch: shared-memory attribute: %s\n", cudaGetErrorString(attr));
         return DCNV4_ERR_LAUNCH;
     }
     int per_sm = 0;
     const cudaError_t occ = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, plan.threads, plan.smem);
     if (occ != cudaSuccess || per_sm < 1) {
-        if (dbg) std::fprintf(stderr, "dcnv4 tile launch: occupancy %d (%s) for %d threads, %zu bytes\n", per_sm,
+        if (dbg) std::fprintf(stderr, "dcnv4 ring launch: occupancy %d (%s) for %d threads, %zu bytes\n", per_sm,
                               cudaGetErrorString(occ), plan.threads, plan.smem);
         return DCNV4_ERR_LAUNCH;
     }
     const long long slots = static_cast<long long>(sm_count()) * per_sm;
-    const unsigned grid = static_cast<unsigned>(std::min<long long>(plan.p.tiles, slots));
-    // the last partial wave (tiles mod grid) is split by consumer warps over up to grid / L
-    // CTAs when at least two can share each tile (DCNV4_TAIL_SPLIT=0 turns it off)
-    dcnv4::TileParams p = plan.p;
-    const int L = static_cast<int>(p.tiles % static_cast<int>(grid));
-    const int consumer_warps = plan.threads / 32 - 1;
-    int split = 1;
-    if (L > 0 && static_cast<int>(grid) >= 2 * L) split = std::min(static_cast<int>(grid) / L, consumer_warps);
-    if (const char* e = std::getenv("DCNV4_TAIL_SPLIT"); e && *e == '0') split = 1;
-    p.tail_split = split;
-    p.main_tiles = split > 1 ? p.tiles - L : p.tiles;
-    p.items = p.main_tiles + (split > 1 ? L * split : 0);
-    kern<<<grid, plan.threads, plan.smem, stream>>>(plan.map, x, om, out, p);
+    const unsigned grid = static_cast<unsigned>(std::min<long long>(plan.p.rows_total, slots));
+    kern<<<grid, plan.threads, plan.smem, stream>>>(plan.map, x, om, out, plan.p);
     const cudaError_t le = cudaGetLastError();
-    if (le != cudaSuccess && dbg) std::fprintf(stderr, "dcnv4 tile launch: %s\n", cudaGetErrorString(le));
+    if (le != cudaSuccess && dbg) std::fprintf(stderr, "dcnv4 ring launch: %s\n", cudaGetErrorString(le));
     return le == cudaSuccess ? DCNV4_OK : DCNV4_ERR_LAUNCH;
 }
 
 template <typename T, int Q, bool HW, bool VF>
-int launch_tile_v(const T* x, const T* om, T* out, const TilePlan& plan, cudaStream_t s) {
-    // a 128-byte window pixel (the common case) as a compile-time stride
-    if constexpr (Q != 5) {
+int launch_ring_v(const T* x, const T* om, T* out, const RingPlan& plan, cudaStream_t s) {
+    // the plain forward with a 128-byte window pixel (the common case) takes the pitch as a constant
+    if constexpr (!VF && Q != 5) {
         if (plan.p.PB == 128) {
-            if (plan.p.f.K == 3) return launch_tile_q<T, Q, 3, HW, 128, VF>(x, om, out, plan, s);
-            return launch_tile_q<T, Q, 0, HW, 128, VF>(x, om, out, plan, s);
+            if (plan.p.f.K == 3) return launch_ring_q<T, Q, 3, HW, 128, false, false>(x, om, out, plan, s);
+            return launch_ring_q<T, Q, 0, HW, 128, false, false>(x, om, out, plan, s);
         }
     }
-    if (plan.p.f.K == 3) return launch_tile_q<T, Q, 3, HW, 0, VF>(x, om, out, plan, s);
-    return launch_tile_q<T, Q, 0, HW, 0, VF>(x, om, out, plan, s);
+    if (plan.p.f.K == 3) return launch_ring_q<T, Q, 3, HW, 0, VF, false>(x, om, out, plan, s);
+    return launch_ring_q<T, Q, 0, HW, 0, VF, false>(x, om, out, plan, s);
 }
 
 template <typename T, int Q, bool HW>
-int launch_tile_k(const T* x, const T* om, T* out, const TilePlan& plan, cudaStream_t s) {
-    // the variant flags get their own instantiations, so that the plain forward carries none of their code
-    if (plan.p.f.flags != 0) return launch_tile_v<T, Q, HW, true>(x, om, out, plan, s);
-    return launch_tile_v<T, Q, HW, false>(x, om, out, plan, s);
+int launch_ring_k(const T* x, const T* om, T* out, const RingPlan& plan, cudaStream_t s) {
+    // the variant flags and the trace get their own instantiations, so that the
+    // plain forward carries none of their code. The tracing build is the generic
+    // one (runtime K and pixel pitch): those template constants change neither the
+    // arithmetic nor its order, so its output is the forward's bit for bit.
+    if (plan.p.trace) return launch_ring_q<T, Q, 0, HW, 0, false, true>(x, om, out, plan, s);
+    if (plan.p.f.flags != 0) return launch_ring_v<T, Q, HW, true>(x, om, out, plan, s);
+    return launch_ring_v<T, Q, HW, false>(x, om, out, plan, s);
 }
 
 template <typename T, int Q>
-int launch_tile_k(const T* x, const T* om, T* out, const TilePlan& plan, cudaStream_t s) {
+int launch_ring_k(const T* x, const T* om, T* out, const RingPlan& plan, cudaStream_t s) {
     if constexpr (std::is_same<T, __half>::value) {
-        if (!f16_exact_from_env()) return launch_tile_k<T, Q, true>(x, om, out, plan, s);
+        if (!f16_exact_from_env()) return launch_ring_k<T, Q, true>(x, om, out, plan, s);
     }
-    return launch_tile_k<T, Q, false>(x, om, out, plan, s);
+    return launch_ring_k<T, Q, false>(x, om, out, plan, s);
 }
 
 template <typename T>
-int launch_tile(const void* x, const void* om, void* out, const TilePlan& plan, cudaStream_t s) {
+int launch_ring(const void* x, const void* om, void* out, const RingPlan& plan, cudaStream_t s) {
     const T* xt = static_cast<const T*>(x);
     const T* omt = static_cast<const T*>(om);
     T* ot = static_cast<T*>(out);
     switch (plan.p.f.Cg * static_cast<int>(sizeof(T)) / 16) {
-        case 1: return launch_tile_k<T, 1>(xt, omt, ot, plan, s);
-        case 2: return launch_tile_k<T, 2>(xt, omt, ot, plan, s);
-        case 4: return launch_tile_k<T, 4>(xt, omt, ot, plan, s);
-        case 5: return launch_tile_k<T, 5>(xt, omt, ot, plan, s);
-        default: return launch_tile_k<T, 8>(xt, omt, ot, plan, s);
+        case 1: return launch_ring_k<T, 1>(xt, omt, ot, plan, s);
+        case 2: return launch_ring_k<T, 2>(xt, omt, ot, plan, s);
+        case 4: return launch_ring_k<T, 4>(xt, omt, ot, plan, s);
+        case 5: return launch_ring_k<T, 5>(xt, omt, ot, plan, s);
+        default: return launch_ring_k<T, 8>(xt, omt, ot, plan, s);
     }
 }
 
@@ -324,27 +400,29 @@ int launch_gather(const T* xt, const T* omt, T* ot, const FwdParams& p, int lane
     return launch_status();
 }
 
+// The forward for one storage type. With `trace` non-NULL the ring kernel's
+// tracing build runs (the same arithmetic, plus one int4 per sampling point);
+// returns DCNV4_NOT_TRACED when the shape takes the global-gather kernel, which
+// has no tracing build.
 template <typename T>
-int launch_forward(const void* x, const void* om, void* out, FwdParams p, cudaStream_t stream) {
+int launch_forward(const void* x, const void* om, void* out, FwdParams p, unsigned* status, int4* trace,
+                   cudaStream_t stream) {
     constexpr int E = sizeof(T);
     if (variant_from_env() == Variant::Auto) {
-        TilePlan plan;
-        if (plan_tile<T>(x, om, out, p, &plan)) return launch_tile<T>(x, om, out, plan, stream);
+        RingPlan plan;
+        if (plan_ring<T>(x, om, out, p, status, trace, &plan)) return launch_ring<T>(x, om, out, plan, stream);
     }
     const int row_bytes = p.Cg * E;
     const bool a16 = aligned(x, 16) && aligned(out, 16) && (p.C * E) % 16 == 0;
     const bool a32 = aligned(x, 32) && aligned(out, 32) && (p.C * E) % 32 == 0;
     const size_t rec_bytes = static_cast<size_t>(3) * p.npts * E;
 
-    int lane_bytes = 0, vec_bytes = 0;
+    int lane_bytes = 0;
     if (a16 && row_bytes % 16 == 0) {
-        if (a32 && row_bytes % 32 == 0) {
-            vec_bytes = 32;
+        if (a32 && row_bytes % 32 == 0)
             lane_bytes = (E == 4 && row_bytes % 64 == 0) ? 64 : 32;
-        } else {
-            vec_bytes = 16;
+        else
             lane_bytes = 16;
-        }
     }
     if (lane_bytes) {
         p.chunks = row_bytes / lane_bytes;
@@ -366,7 +444,10 @@ int launch_forward(const void* x, const void* om, void* out, FwdParams p, cudaSt
     const T* xt = static_cast<const T*>(x);
     const T* omt = static_cast<const T*>(om);
     T* ot = static_cast<T*>(out);
-    // the variant flags get their own instantiations, as in the tile kernel
-    if (p.flags != 0) return launch_gather<T, true>(xt, omt, ot, p, lane_bytes, grid, threads, smem, stream);
-    return launch_gather<T, false>(xt, omt, ot, p, lane_bytes, grid, threads, smem, stream);
+    int rc;
+    // the variant flags get their own instantiations, as in the ring kernel
+    if (p.flags != 0) rc = launch_gather<T, true>(xt, omt, ot, p, lane_bytes, grid, threads, smem, stream);
+    else rc = launch_gather<T, false>(xt, omt, ot, p, lane_bytes, grid, threads, smem, stream);
+    if (rc == DCNV4_OK && trace) return DCNV4_NOT_TRACED;
+    return rc;
 }

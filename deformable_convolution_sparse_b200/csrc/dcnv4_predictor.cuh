@@ -35,7 +35,8 @@
 
 #include <cuda.h>
 
-#include "dcnv4_window.cuh"
+#include "dcnv4_async.cuh"
+#include "dcnv4_kernels.cuh"
 
 namespace dcnv4 {
 
@@ -53,6 +54,7 @@ struct PredParams {
     int out_bufs;   // output staging buffers (2, or 1 when two do not fit)
     int w_in_staging;  // raw W fits the (still idle) output staging area: the activation loads start at once
     unsigned smem_b, smem_a, smem_o, smem_meta;  // byte offsets of the shared-memory regions
+    unsigned* status;  // device status word (bit kStatusCopyTimeout)
 };
 
 // slot of projection channel o in its record: offsets (g, comp, j) -> g*3P + comp*P + j,
@@ -244,7 +246,7 @@ predictor_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_const
         fence_proxy_async();  // the generic writes of W, before the tensor cores read them
     }
     __syncthreads();
-    if (!b_ok && tid == 0) atomicOr(&g_device_status, kStatusCopyTimeout);
+    if (!b_ok && tid == 0) atomicOr(p.status, kStatusCopyTimeout);
 
     if (!b_ok) {
         // nothing was started: straight to the release of tensor memory
@@ -255,7 +257,7 @@ predictor_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_const
                 const int s = it % p.stages;
                 if (it >= p.stages &&
                     !mbar_wait_bounded(&a_empty[s], static_cast<unsigned>((it / p.stages) - 1) & 1u, kCopyWaitLimitNs)) {
-                    atomicOr(&g_device_status, kStatusCopyTimeout);
+                    atomicOr(p.status, kStatusCopyTimeout);
                     break;
                 }
                 const int tile = static_cast<int>(blockIdx.x) + it * static_cast<int>(gridDim.x);
@@ -289,7 +291,7 @@ predictor_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_const
                 umma_commit(&a_empty[s]);
                 umma_commit(&acc_full[b]);
             }
-            if (!ok) atomicOr(&g_device_status, kStatusCopyTimeout);
+            if (!ok) atomicOr(p.status, kStatusCopyTimeout);
         }
     } else {
         // ------------------------------------------------------------ epilogue
@@ -313,7 +315,7 @@ predictor_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_const
             const bool ok = mbar_wait_bounded(&acc_full[b], static_cast<unsigned>(it >> 1) & 1u, kCopyWaitLimitNs);
             // one decision for all epilogue threads, so that they leave together
             if (!named_bar_and(1, NE, ok)) {
-                if (et == 0) atomicOr(&g_device_status, kStatusCopyTimeout);
+                if (et == 0) atomicOr(p.status, kStatusCopyTimeout);
                 break;
             }
             tc_fence_after();

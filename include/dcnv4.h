@@ -70,7 +70,10 @@ extern "C" {
 #define DCNV4_API
 #endif
 
-/* Storage type of x, offset_mask and out. Arithmetic is fp32 in all cases. */
+/* Storage type of x, offset_mask and out. Sums are fp32 in every case; the
+ * corner weights are fp32 for DCNV4_F32 and DCNV4_BF16 and are rounded once to
+ * fp16 for DCNV4_F16 (fp16 x fp16 products, exact in fp32, accumulated in
+ * fp32), as stated with the formula above. */
 typedef enum {
     DCNV4_F32 = 0,
     DCNV4_F16 = 1,
@@ -264,6 +267,33 @@ DCNV4_API int dcnv4_sampling_index(const void *offset_mask, int32_t *corner, uin
                          int stride, int pad, int dilation, float offset_scale, int dtype,
                          void *stream);
 
+/* The forward of dcnv4_forward, traced: the same plan, kernel code and
+ * arithmetic (out receives the same bits as dcnv4_forward writes), and for
+ * every sampling point p = (((n*Hout+ho)*Wout+wo)*G+g)*K*K+k the integer
+ * corner and validity that the gather actually used, for bit-exact comparison
+ * with a reference ("不只是卷积的平替", jsqmd.com, section 1: the sample sits at
+ * the regular grid position plus the learned offset):
+ *   trace[4p+0], trace[4p+1] = top-left corner (y0, x0), or (INT32_MIN,
+ *                              INT32_MIN) when no corner is inside the image;
+ *   trace[4p+2]              = validity bits as in dcnv4_sampling_index;
+ *   trace[4p+3]              = path: 0 = read from the shared-memory window
+ *                              of the ring kernel (validity is then the image
+ *                              test that the window's zero fill implements),
+ *                              1 = the ring kernel's global-memory pass,
+ *                              2 = the global-gather kernel (shapes the ring
+ *                              kernel does not take; traced by the index code
+ *                              that kernel shares).
+ * trace: device int32 [N,Hout,Wout,G,K*K,4], 16-byte aligned, overlapping no
+ * other buffer (DCNV4_ERR_NULL / DCNV4_ERR_ALIGN / DCNV4_ERR_ALIAS); other
+ * checks as dcnv4_forward, plus DCNV4_ERR_TOO_LARGE when 4*N*Hout*Wout*G*K*K
+ * reaches 2^31. A debugging and testing entry point: the tracing kernel is a
+ * separate build of the forward kernel with the trace stores compiled in.
+ * Asynchronous on `stream`; nothing is launched when N == 0. */
+DCNV4_API int dcnv4_forward_trace(const void *x, const void *offset_mask, void *out, int32_t *trace,
+                                  int N, int H, int W, int C, int G, int K,
+                                  int stride, int pad, int dilation, float offset_scale, int dtype,
+                                  void *stream);
+
 /* The forward from and to HOST memory, for callers whose data lives on the
  * host. x_host, offset_mask_host: inputs in host memory (pinned memory lets
  * the copies run asynchronously and overlap; pageable memory works but the
@@ -280,7 +310,14 @@ DCNV4_API int dcnv4_sampling_index(const void *offset_mask, int32_t *corner, uin
  * out_host. Checks: those of dcnv4_forward on the device buffers, plus NULL
  * host pointers (DCNV4_ERR_NULL) and out_host overlapping x_host or
  * offset_mask_host (DCNV4_ERR_ALIAS). A failing CUDA copy, event or stream
- * call returns DCNV4_ERR_CUDA. */
+ * call returns DCNV4_ERR_CUDA. After any error return that came once copies
+ * were queued, `stream` still waits for everything the call queued, so
+ * out_host may have been written in part when `stream` reaches that point;
+ * synchronise `stream` before reusing or freeing the buffers. The library's
+ * streams and cached device addresses belong to the CUDA context current at
+ * the first call on each device: the library must not be used after
+ * cudaDeviceReset (or any other destruction of that context) in the same
+ * process. */
 DCNV4_API int dcnv4_forward_host(const void *x_host, const void *offset_mask_host, void *out_host,
                                  void *x_dev, void *offset_mask_dev, void *out_dev,
                                  int N, int H, int W, int C, int G, int K,
@@ -312,7 +349,11 @@ DCNV4_API int dcnv4_forward_host(const void *x_host, const void *offset_mask_hos
  *     GPU race on the array: queue them on one stream, or order them.
  *   - Ordering, streams and the other checks are those of dcnv4_forward_host
  *     (the host pointers are checked for NULL, alignment and overlap); the
- *     result is in out_host once `stream` reaches the end of the call's work. */
+ *     result is in out_host once `stream` reaches the end of the call's work. After an error return
+ *     that came once copies were queued, `stream` still waits for them (see
+ *     dcnv4_forward_host). As there, do not use the library after
+ *     cudaDeviceReset in the same process: the array's cached address and the
+ *     library's streams belong to the context that the first call saw. */
 #define DCNV4_NOALLOC_STAGING_BYTES (32u << 20)
 DCNV4_API int dcnv4_forward_host_noalloc(const void *x_host, const void *offset_mask_host, void *out_host,
                                          int N, int H, int W, int C, int G, int K,
@@ -336,6 +377,21 @@ DCNV4_API int dcnv4_device_status(unsigned int *status, int clear);
  * sets DCNV4_DEVSTATUS_SELFTEST_TIMEOUT and returns. Asynchronous on `stream`.
  * Returns DCNV4_OK, DCNV4_ERR_SHAPE (limit out of range) or DCNV4_ERR_LAUNCH. */
 DCNV4_API int dcnv4_selftest_wait_timeout(unsigned long long limit_ns, void *stream);
+
+/* Measures this GPU's shared-memory gather rate, the ceiling of the forward
+ * kernel's inner loop (each sampling point reads 4 corners x C/G channels from
+ * shared memory). The pages have no counterpart; it backs the roofline
+ * discussion of the measurements. One CTA per SM, 512 threads, 64 KB of shared
+ * memory; every 16-byte load of a quarter warp falls on a different bank
+ * position (one 128-byte wavefront per quarter warp and load). pattern 0:
+ * independent rows picked at random; pattern 1: the forward's own access
+ * pattern (2x2 corners x 2 chunks of 128-byte pixels at random window
+ * positions, chunk rotation as in the ring kernel). Writes the bytes moved per
+ * SM clock per SM (the slowest CTA's clock64 span). Synchronous: runs on the
+ * legacy default stream and waits for the device. Returns DCNV4_OK,
+ * DCNV4_ERR_NULL, DCNV4_ERR_SHAPE (unknown pattern), DCNV4_ERR_LAUNCH or
+ * DCNV4_ERR_CUDA. */
+DCNV4_API int dcnv4_probe_smem_gather(int pattern, double *bytes_per_clock_per_sm);
 
 /* Static description of an error code; never NULL. */
 DCNV4_API const char *dcnv4_strerror(int status);

@@ -36,7 +36,7 @@ def build(force: bool = False) -> str:
     """Compile ``dcnv4_oracle.c`` into ``liboracle.so`` (gcc, no fused multiply-add)."""
     if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
         tmp = _LIB + ".tmp.%d" % os.getpid()
-        subprocess.check_call(["gcc", "-O2", "-std=c99", "-ffp-contract=off", "-fno-fast-math",
+        subprocess.check_call(["gcc", "-O2", "-std=c99", "-ffp-contract=off", "-fno-fast-math", "-fopenmp",
                                "-shared", "-fPIC", "-o", tmp, _SRC, "-lm"])
         os.replace(tmp, _LIB)
     return _LIB
@@ -53,6 +53,10 @@ def _load():
         lib.oracle_dcnv4_forward.restype = i
         lib.oracle_dcnv4_forward_images.argtypes = [p, p, p] + [i] * 9 + [f, i, i]
         lib.oracle_dcnv4_forward_images.restype = i
+        lib.oracle_dcnv4_forward_images_mt.argtypes = [p, p, p] + [i] * 9 + [f, i, i, i]
+        lib.oracle_dcnv4_forward_images_mt.restype = i
+        lib.oracle_max_threads.argtypes = []
+        lib.oracle_max_threads.restype = i
         lib.oracle_dcnv4_sampling_index.argtypes = [p, p, p] + [i] * 8 + [f]
         lib.oracle_dcnv4_sampling_index.restype = i
         lib.oracle_dcnv4_backward.argtypes = [p] * 5 + [i] * 9 + [f]
@@ -80,13 +84,21 @@ def _ptr(a: np.ndarray):
     return a.ctypes.data_as(ctypes.c_void_p)
 
 
+def max_threads() -> int:
+    """Threads the oracle's parallel forward uses by default (OpenMP)."""
+    return _load().oracle_max_threads()
+
+
 def dcnv4_forward(x, offset_mask, G: int, K: int, stride: int = 1, pad: int = 0,
                   dilation: int = 1, offset_scale: float = 1.0,
-                  n_begin: int | None = None, n_end: int | None = None) -> np.ndarray:
+                  n_begin: int | None = None, n_end: int | None = None, threads: int = 1) -> np.ndarray:
     """fp64 forward. ``x``: [N,H,W,C]; ``offset_mask``: [N,Hout,Wout,G,3*K*K].
 
     Returns out [N,Hout,Wout,C] (fp64). With ``n_begin``/``n_end`` only those
-    images are computed (the rest of the result stays zero).
+    images are computed (the rest of the result stays zero). ``threads`` != 1
+    shares the output rows out among that many OpenMP threads (0: all); every
+    element is computed by the same code in the same order, so the result is
+    the same bits.
     """
     x = _f64(x)
     om = _f64(offset_mask)
@@ -98,7 +110,12 @@ def dcnv4_forward(x, offset_mask, G: int, K: int, stride: int = 1, pad: int = 0,
     if N == 0:
         return out
     lib = _load()
-    if n_begin is None and n_end is None:
+    if threads != 1:
+        rc = lib.oracle_dcnv4_forward_images_mt(_ptr(x), _ptr(om), _ptr(out), N, H, W, C, G, K,
+                                                stride, pad, dilation, float(offset_scale),
+                                                0 if n_begin is None else n_begin,
+                                                N if n_end is None else n_end, int(threads))
+    elif n_begin is None and n_end is None:
         rc = lib.oracle_dcnv4_forward(_ptr(x), _ptr(om), _ptr(out), N, H, W, C, G, K,
                                       stride, pad, dilation, float(offset_scale))
     else:

@@ -21,8 +21,7 @@
  *    offset_mask[N,Hout,Wout,G,3*K*K] with, per group, 2*K*K offsets then
  *    K*K masks, zero padding outside the image, out[N,Hout,Wout,C].
  *
- * Readings taken where the pages are silent (each is also listed in the
- * design notes):
+ * Readings taken where the pages are silent:
  *  - grid point order is row-major, k = ky*K + kx;
  *  - the grid is convolution style: p0 = o*stride - pad + kk*dilation;
  *  - offsets are component-major inside the 2*K*K block: r[k] moves along
@@ -41,6 +40,9 @@
 #include <math.h>
 #include <stdint.h>
 #include <stddef.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
 
 /* Output extent of one spatial axis, convolution style. Returns <= 0 when no
  * output position exists. */
@@ -143,6 +145,48 @@ int oracle_dcnv4_forward_images(const double *x, const double *om, double *out,
                     aggregate_one(x, om, out, N, H, W, C, G, K, stride, pad, dilation,
                                   offset_scale, Hout, Wout, n, ho, wo, g);
     return 0;
+}
+
+/* oracle_dcnv4_forward_images with the (image, output row) pairs shared out
+ * among `threads` OpenMP threads (threads <= 0: the OpenMP default). Every
+ * output element is still computed by aggregate_one, alone and in the same
+ * order, so the result is bit-identical to the single-thread call; only the
+ * wall time changes. Used to time the oracle on all host cores. */
+int oracle_dcnv4_forward_images_mt(const double *x, const double *om, double *out,
+                                   int N, int H, int W, int C, int G, int K,
+                                   int stride, int pad, int dilation, float offset_scale,
+                                   int n_begin, int n_end, int threads)
+{
+    if (n_begin < 0 || n_end > N || n_begin > n_end || C % G) return -1;
+    const int Hout = oracle_output_size(H, K, stride, pad, dilation);
+    const int Wout = oracle_output_size(W, K, stride, pad, dilation);
+    if (Hout <= 0 || Wout <= 0) return -1;
+    const long rows = (long)(n_end - n_begin) * Hout;
+#ifdef _OPENMP
+    if (threads > 0) omp_set_num_threads(threads);
+#else
+    (void)threads;
+#endif
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long r = 0; r < rows; ++r) {
+        const int n = n_begin + (int)(r / Hout), ho = (int)(r % Hout);
+        for (int wo = 0; wo < Wout; ++wo)
+            for (int g = 0; g < G; ++g)
+                aggregate_one(x, om, out, N, H, W, C, G, K, stride, pad, dilation,
+                              offset_scale, Hout, Wout, n, ho, wo, g);
+    }
+    return 0;
+}
+
+/* Number of threads an OpenMP parallel region of this library would use
+ * (1 when it is built without OpenMP). */
+int oracle_max_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
 }
 
 /* Integer part of every sample: the top-left corner (y0, x0) and a 4-bit mask

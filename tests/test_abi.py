@@ -247,3 +247,27 @@ def test_backward_ex_reports_each_error_class_before_any_cuda_call(kw, status):
 
 def test_backward_ex_empty_batch_touches_nothing():
     assert _bwx(x=0, om=0, z=0, go=0, gx=0, gom=0, gz=0, N=0, flags=7) == B.DCNV4_OK
+
+
+def test_forward_trace_checks():
+    lib = B.load_library()
+    TR = 0x40000000
+    a = dict(GOOD)
+    args = (a["N"], a["H"], a["W"], a["C"], a["G"], a["K"], 1, 1, 1, ctypes.c_float(1.0), a["dtype"], None)
+    # the forward's own checks come first
+    assert lib.dcnv4_forward_trace(X, OM, X, TR, *args) == B.STATUS["DCNV4_ERR_ALIAS"]
+    # then the trace buffer: present, 16-byte aligned, overlapping nothing
+    assert lib.dcnv4_forward_trace(X, OM, OUT, 0, *args) == B.STATUS["DCNV4_ERR_NULL"]
+    assert lib.dcnv4_forward_trace(X, OM, OUT, TR + 4, *args) == B.STATUS["DCNV4_ERR_ALIGN"]
+    assert lib.dcnv4_forward_trace(X, OM, OUT, OUT, *args) == B.STATUS["DCNV4_ERR_ALIAS"]
+    assert lib.dcnv4_forward_trace(X, OM, OUT, OM - 64, *args) == B.STATUS["DCNV4_ERR_ALIAS"]
+    # an empty batch launches nothing and succeeds, also without a GPU
+    assert lib.dcnv4_forward_trace(0, 0, 0, 0, 0, 8, 8, 16, 2, 3, 1, 1, 1, ctypes.c_float(1.0), a["dtype"],
+                                   None) == B.DCNV4_OK
+
+
+def test_probe_smem_gather_checks_before_any_cuda_call():
+    lib = B.load_library()
+    v = ctypes.c_double(0.0)
+    assert lib.dcnv4_probe_smem_gather(0, None) == B.STATUS["DCNV4_ERR_NULL"]
+    assert lib.dcnv4_probe_smem_gather(7, ctypes.byref(v)) == B.STATUS["DCNV4_ERR_SHAPE"]

@@ -20,6 +20,7 @@ import pytest
 import torch
 
 import oracle
+from deformable_convolution_sparse_b200.workloads import WORKLOADS, workload_inputs
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "hand_cases.json")
 
@@ -378,3 +379,19 @@ def test_output_size_matches_convolution_arithmetic():
                                        padding=p, dilation=d)
         assert oracle.output_size(H, K, s, p, d) == t.shape[-1]
     assert oracle.output_size(2, 5, 1, 0, 1) <= 0
+
+
+@pytest.mark.parametrize("name", ["tiny_f32", "stage3_f16", "sd_latent_f16", "highres_bf16"])
+def test_parallel_oracle_gives_the_same_bits(name):
+    """The all-core oracle (OpenMP over output rows, used to time the CPU
+    baseline) computes every element with the same code in the same order as
+    the single-thread one: the results are identical."""
+    w = WORKLOADS[name]
+    x, om = workload_inputs(w)
+    xd, omd = x.double().numpy(), om.double().numpy()
+    n1 = min(w.N, 2)
+    a = oracle.dcnv4_forward(xd, omd, **w.kwargs(), n_begin=0, n_end=n1)
+    b = oracle.dcnv4_forward(xd, omd, **w.kwargs(), n_begin=0, n_end=n1, threads=0)
+    c = oracle.dcnv4_forward(xd, omd, **w.kwargs(), n_begin=0, n_end=n1, threads=3)
+    np.testing.assert_array_equal(a, b)
+    np.testing.assert_array_equal(a, c)
