@@ -88,7 +88,9 @@ probe_smem_gather_kernel(int pattern, int iters) {
                 const uint4 b = *reinterpret_cast<const uint4*>(psm + pc + 128u);
                 const uint4 c2 = *reinterpret_cast<const uint4*>(psm + pc + 26u * 128u);
                 const uint4 d = *reinterpret_cast<const uint4*>(psm + pc + 27u * 128u);
-                acc ^= a.x ^ b.y ^ c2.z ^ d.w ^ a.w ^ b.x ^ c2.y ^ d.z;
+                // every word of every load is used, so each stays one 16-byte load
+                acc ^= a.x ^ a.y ^ a.z ^ a.w ^ b.x ^ b.y ^ b.z ^ b.w;
+                acc ^= c2.x ^ c2.y ^ c2.z ^ c2.w ^ d.x ^ d.y ^ d.z ^ d.w;
             }
         }
     }

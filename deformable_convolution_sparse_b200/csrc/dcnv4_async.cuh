@@ -71,7 +71,10 @@ __device__ __forceinline__ uint64_t global_ns() {
     return t;
 }
 // Waits for phase `parity` of `bar`, giving up after `limit_ns` nanoseconds.
+// The global timer (a slow special-register read) is read only once the first
+// try has failed: a phase that has already completed costs one try_wait.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, unsigned parity, uint64_t limit_ns) {
+    if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_ns();
     for (unsigned i = 1;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;

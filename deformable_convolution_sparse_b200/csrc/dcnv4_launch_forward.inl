@@ -25,8 +25,11 @@ int env_int(const char* name, int dflt) {
 // consumer threads (15 warps) per CTA, plus one producer warp: 16 warps, 4 per SM
 // sub-partition, whose 16 K registers then hold 4 warps at the kernel's 112-register cap
 // (a 17th warp would put 5 on one sub-partition: 17,920 registers, and the CTA would not launch)
-constexpr int kUnitsMax = 480;
-static_assert(((kUnitsMax / 32 + 1 + 3) / 4) * 112 * 32 <= 16384,
+#ifndef DCNV4_RING_UNITS_MAX
+#define DCNV4_RING_UNITS_MAX 480  // consumer threads per CTA (build option, with DCNV4_RING_MAXREG)
+#endif
+constexpr int kUnitsMax = DCNV4_RING_UNITS_MAX;
+static_assert(((kUnitsMax / 32 + 1 + 3) / 4) * DCNV4_RING_MAXREG * 32 <= 16384,
               "the ring kernel's register cap must fit the warps of one SM sub-partition");
 
 // Mean shared-memory wavefronts of one quarter-warp LDS.128 in the ring
@@ -104,21 +107,27 @@ struct RingShape {  // one candidate of the planner
     double score;
 };
 
-// The best plan for halo R (score < 0: none fits). Everything but R leaves the
-// per-unit arithmetic unchanged; it is chosen for speed and may depend on N.
-// The score multiplies estimated efficiencies: filled columns and rows,
-// shared-memory wavefronts of the gather, active warps, the window width
-// against the band (L2 -> SM traffic), record-buffer depth, and the part of a
-// CTA's time spent waiting for windows:
-//  - the ring should hold the current window plus the next item's rows
-//    (NR >= nrows + TH*stride), else every item waits for its own rows;
-//  - a CTA whose row range crosses into a new strip loads a whole window
-//    there; with NR >= 2*nrows that load overlaps the last items of the
-//    previous strip, else the CTA waits for it (about 1500 cycles plus the
-//    window's bytes at 100 B per cycle from L2), against about
-//    (0.75*Q + 0.5) cycles of SM time per sampling point.
+// The best plan for halo R (score < 0: none fits) with at least `min_units`
+// consumer threads. Everything but R leaves the per-unit arithmetic unchanged;
+// it is chosen for speed and may depend on N. The score is the inverse of an
+// estimated launch time (microseconds at 1.9 GHz), the sum of
+//  - compute: a CTA's rows x band width x groups x points at (0.75*Q + 0.5)
+//    SM cycles per sampling point (the measured rate of the 128-byte-pixel
+//    gather), divided by the gather's bank efficiency (1 / wavefronts^2), the
+//    record layout (per-pixel runs measured about 20 % slower than one run per
+//    output row), warp occupancy (below 12 consumer warps, 8 with four or more
+//    chunks per group), the filled lanes of
+//    the consumer warps and bands narrower
+//    than half their window (measured slower: (2 TW stride / WW)^(1/4));
+//  - start-up: every CTA loads its first window and records at once, from HBM
+//    at about 6.5 TB/s;
+//  - strip changes that the ring cannot prefetch (NR < 2*nrows): about 1 us
+//    plus the window's bytes at 100 B per cycle each, one per Hout rows of a
+//    CTA's range;
+//  - items whose rows cannot load during the previous item (NR < nrows +
+//    TH*stride): about 1 us each.
 template <typename T>
-RingShape best_ring_shape(const FwdParams& f, int R, int nsm) {
+RingShape best_ring_shape(const FwdParams& f, int R, int nsm, int min_units) {
     constexpr int E = sizeof(T);
     const int row_bytes = f.Cg * E;
     const int Q = row_bytes / 16;
@@ -130,6 +139,7 @@ RingShape best_ring_shape(const FwdParams& f, int R, int nsm) {
     const int forceNR = env_int("DCNV4_RING", 0);
     const int s = f.stride;
     const int UH = (f.K - 1) * f.dilation + 2 * R + 1;
+    const double clk = 1.9e3;  // SM cycles per microsecond
     RingShape best{};
     best.score = -1.0;
     static const int TWs[] = {1, 2, 4, 7, 8, 14, 16, 28, 32, 56, 64};
@@ -148,6 +158,7 @@ RingShape best_ring_shape(const FwdParams& f, int R, int nsm) {
         const double w = gather_wavefronts(Q, GS);
         const double banks = 1.0 / (w * w);
         const bool row_runs = GS == f.G;
+        const double runs = row_runs ? 1.0 : 0.8;
         for (int TW : TWs) {
             if (forceTW && TW != forceTW) continue;
             if (TW > f.Wout && TW != TWs[0]) {
@@ -160,13 +171,14 @@ RingShape best_ring_shape(const FwdParams& f, int R, int nsm) {
             if (WW > 256) continue;
             const int rowB = (WW * PB + 127) / 128 * 128;  // ring row pitch: every TMA destination 128-byte aligned
             const int bands = (f.Wout + TW - 1) / TW;
-            const double fill_w = static_cast<double>(f.Wout) / (static_cast<double>(bands) * TW);
+            const double rows_per_cta =
+                static_cast<double>(f.N) * bands * (f.G / GS) * f.Hout / std::max(1, nsm);
             for (int TH = 1; TH <= 16; ++TH) {
                 if (forceTH && TH != forceTH) continue;
                 if (TH > f.Hout) break;
                 const int units = TH * TW * GS;
                 if (units > kUnitsMax) break;
-                if (units < 32) continue;
+                if (units < min_units) continue;
                 const int nrows = (TH - 1) * s + UH;
                 const int slot = odd16((row_runs ? TW * f.G : GS) * R3 * E + 32);
                 const int rec = ((row_runs ? TH : TH * TW) * slot + 127) / 128 * 128;
@@ -182,23 +194,19 @@ RingShape best_ring_shape(const FwdParams& f, int R, int nsm) {
                                         static_cast<size_t>(nrec) * rec;
                     if (smem > kTileSmemLimit) continue;
                     const int threads = (units + 31) / 32 * 32 + 32;
-                    // a new strip's window loaded while the last one is still read
-                    // (NR >= 2 nrows), or at least the next item's rows (NR >= nrows + TH s)
-                    double prefetch = NR >= nrows + TH * s ? 1.0 : 0.5;
-                    if (NR < 2 * nrows) {
-                        const int bands_ = (f.Wout + TW - 1) / TW;
-                        const double rows_per_cta = static_cast<double>(f.N) * bands_ * (f.G / GS) * f.Hout / nsm;
-                        const double compute = rows_per_cta * TW * GS * f.npts * (0.75 * Q + 0.5);
-                        const double stall = rows_per_cta / f.Hout * (1500.0 + static_cast<double>(nrows) * rowB / 100.0);
-                        prefetch *= compute / (compute + stall);
-                    }
-                    const int tiles_h = (f.Hout + TH - 1) / TH;
-                    const double fill_h = static_cast<double>(f.Hout) / (static_cast<double>(tiles_h) * TH);
-                    const double occ = std::min(1.0, (threads - 32) / 384.0);
-                    const double l2 = std::sqrt(std::sqrt(static_cast<double>(TW * s) / WW));
-                    (void)nsm;
-                    const double depth = nrec >= 3 ? 1.0 : 0.97;
-                    const double score = fill_w * fill_w * fill_h * banks * prefetch * occ * l2 * depth;
+                    const double warps = (threads - 32) / 32.0;
+                    const double occ = std::min(1.0, warps / (Q >= 4 ? 8.0 : 12.0));  // fewer loads per point want more warps
+                    // bands narrower than half their window (WW > 2 TW stride) measured slower
+                    const double narrow = std::sqrt(std::sqrt(std::min(1.0, 2.0 * TW * s / WW)));
+                    const double lanes = static_cast<double>(units) / (threads - 32);  // filled lanes of the last warp
+                    const double cpp = (0.75 * Q + 0.5) / (banks * runs * occ * narrow * lanes);
+                    const double t_compute = rows_per_cta * TW * GS * f.npts * cpp / clk;
+                    const double t_start = static_cast<double>(nsm) * (static_cast<double>(nrows) * rowB + rec) / 6.5e6;
+                    double t_wait = 0.0;
+                    if (NR < 2 * nrows) t_wait += rows_per_cta / f.Hout * (1.0 + static_cast<double>(nrows) * rowB / (100.0 * clk));
+                    if (NR < nrows + TH * s) t_wait += rows_per_cta / TH * 1.0;
+                    const double t_depth = nrec >= 3 ? 0.0 : 0.01 * t_compute;
+                    const double score = 1.0 / (t_compute + t_start + t_wait + t_depth);
                     if (score > best.score) {
                         best = RingShape{GS, R, TW, TH, nrec, NR, units, threads, slot, rec, WW, UH, c2, smem, score};
                     }
@@ -227,18 +235,17 @@ bool plan_ring(const void* x, const void* om, const void* out, const FwdParams& 
     if (nsm <= 0) return false;
     int Rhi = default_halo(f.dilation), Rlo = 1;
     if (const int h = env_int("DCNV4_HALO", 0); h > 0) Rhi = Rlo = h;
-    // the largest halo whose best plan keeps at least 8 consumer warps busy (or
-    // covers a whole item of a small image), judged for a nominal batch of 64
-    // images and 148 SMs so that the halo does not depend on N
+    // the largest halo for which a plan with at least 8 consumer warps fits (or
+    // one covering a whole item of a small image); it depends on the geometry
+    // alone, so an image's result does not depend on N
+    const int min_units = std::min(256, f.Hout * f.Wout * f.G);
     int R = -1;
     FwdParams nominal = f;
     nominal.N = 64;
-    for (int r = Rhi; r >= Rlo && R < 0; --r) {
-        const RingShape c = best_ring_shape<T>(nominal, r, 148);
-        if (c.score >= 0.0 && (c.units >= 256 || r == Rlo || c.units >= f.Hout * f.Wout * f.G)) R = r;
-    }
+    for (int r = Rhi; r >= Rlo && R < 0; --r)
+        if (best_ring_shape<T>(nominal, r, 148, min_units).score >= 0.0) R = r;
     if (R < 0) return false;
-    const RingShape sh = best_ring_shape<T>(f, R, nsm);
+    const RingShape sh = best_ring_shape<T>(f, R, nsm, min_units);
     if (sh.score < 0.0) return false;
 
     dcnv4::RingParams bp{};

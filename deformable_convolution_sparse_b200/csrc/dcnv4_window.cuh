@@ -145,6 +145,19 @@ __device__ __forceinline__ uint4 pack_chunk(const float2* a) {
     return v;
 }
 
+// 16-byte shared-memory load at a 32-bit shared-window address plus a
+// compile-time byte offset. Ordered after the item's "full" wait by its data
+// dependence: every address is computed from records read after that wait.
+template <int OFF = 0>
+__device__ __forceinline__ uint4 lds128(unsigned a) {
+    uint4 v;
+    asm("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4+%5];"
+        : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+        : "r"(a), "n"(OFF));
+    return v;
+}
+__device__ __forceinline__ uint4 lds128r(unsigned a, unsigned off) { return lds128<0>(a + off); }
+
 // Two fp32 weights to a pair of fp16 (round to nearest even), one instruction.
 __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
     __half2 h = __floats2half2_rn(lo, hi);
@@ -345,10 +358,13 @@ __device__ __forceinline__ void issue_rows(const RingParams& p, const CUtensorMa
 // gather used; compiled out of the forward's own builds.
 // PBC: the window's pixel pitch as a compile-time constant (0: p.PB), so that
 // the right-hand corners are immediate offsets of the left-hand ones.
-// Registers: capped at 112 per thread; the planner keeps CTAs at 16 warps or
-// fewer, so that each SM sub-partition (16 K registers) holds its share.
+// Registers: capped at DCNV4_RING_MAXREG (112) per thread; the planner keeps
+// CTAs small enough that each SM sub-partition (16 K registers) holds its share.
+#ifndef DCNV4_RING_MAXREG
+#define DCNV4_RING_MAXREG 112  // registers per thread (build option)
+#endif
 template <typename T, int Q, int KS, bool HW, int PBC, bool VF, bool TRACE>
-__global__ void __maxnreg__(112)
+__global__ void __maxnreg__(DCNV4_RING_MAXREG)
 fwd_ring_kernel(const __grid_constant__ CUtensorMap xmap, const T* __restrict__ x, const T* __restrict__ om,
                 T* __restrict__ out, RingParams p) {
     extern __shared__ __align__(128) unsigned char smem[];
@@ -382,17 +398,20 @@ fwd_ring_kernel(const __grid_constant__ CUtensorMap xmap, const T* __restrict__ 
     if (warp == nc) {
         // ---------------------------------------------------------------- producer
         ItemCursor cur = item_cursor(p, blockIdx.x, gridDim.x);
-        int vh[4] = {0, 0, 0, 0};  // window start (virtual row) of the items in flight, by i % 4
-        int d = 0;                 // items known to be done
+        // window start (virtual row) of the items in flight: vh0 is item d's, vh1 item d+1's, ...
+        // (at most nrec <= 4 items are in flight; kept in registers, shifted as d advances)
+        int vh0 = 0, vh1 = 0, vh2 = 0, vh3 = 0;
+        int d = 0;  // items known to be done
         for (int i = 0;; ++i) {
             Item it;
             if (!next_item(p, cur, it)) break;
             // the rows below `need` (virtual) are overwritten; the record/barrier slot is item i - nrec's
             const int need = it.lv + it.ln - p.NR;
             bool ok = true;
-            while (ok && d < i && (d <= i - nrec || vh[d & 3] < need)) {
+            while (ok && d < i && (d <= i - nrec || vh0 < need)) {
                 ok = mbar_wait_bounded(&done[d % nrec], (d / nrec) & 1, kCopyWaitLimitNs);
                 ++d;
+                vh0 = vh1; vh1 = vh2; vh2 = vh3;
             }
             if (!__all_sync(0xffffffffu, ok)) {
                 if (lane == 0) atomicOr(p.status, kStatusCopyTimeout);
@@ -401,7 +420,12 @@ fwd_ring_kernel(const __grid_constant__ CUtensorMap xmap, const T* __restrict__ 
                     mbar_wait_bounded(&full[q % nrec], (q / nrec) & 1, kCopyWaitLimitNs);
                 return;
             }
-            vh[i & 3] = it.v;
+            // item i is the (i - d)-th in flight
+            const int slot = i - d;
+            if (slot == 0) vh0 = it.v;
+            else if (slot == 1) vh1 = it.v;
+            else if (slot == 2) vh2 = it.v;
+            else vh3 = it.v;
             fence_proxy_async();  // the consumers' reads of those buffers before the async writes
             issue_records<T>(p, om, it, recbuf + (i % nrec) * p.rec_bytes, &full[i % nrec], lane);
             issue_rows(p, &xmap, it, ring, &full[i % nrec], lane);
@@ -437,11 +461,13 @@ fwd_ring_kernel(const __grid_constant__ CUtensorMap xmap, const T* __restrict__ 
     const int rowC = f.W * f.C;
     const int within = row_runs ? (px * f.G + gl) : gl;  // unit index inside its record run
     const unsigned char* const ubase = ring + gl * (Q * 16);
-    const unsigned char* cbase[Q];  // this lane's chunks of ring pixel (0, 0), in its rotated order
-#pragma unroll
-    for (int j = 0; j < Q; ++j) cbase[j] = ubase + choff[j];
     const int cb = px * f.stride;  // this unit's first window column
-    const float2 scale2 = make_float2(f.offset_scale, f.offset_scale);
+    // this lane's chunks of ring pixel (0, cb), in its rotated order (32-bit shared-window addresses)
+    unsigned cbase_s[Q];
+#pragma unroll
+    for (int j = 0; j < Q; ++j) cbase_s[j] = smem_addr(ubase + choff[j] + cb * PB);
+    const unsigned rowBu = static_cast<unsigned>(p.rowB), PBu = static_cast<unsigned>(PB);
+    const unsigned ringB = NR * rowBu;  // bytes of the ring rows (the mirror row follows)
 
     ItemCursor cur = item_cursor(p, blockIdx.x, gridDim.x);
     for (int i = 0;; ++i) {
@@ -470,9 +496,10 @@ fwd_ring_kernel(const __grid_constant__ CUtensorMap xmap, const T* __restrict__ 
 #pragma unroll
                 for (int q = 0; q < CH / 2; ++q) acc[j][q] = make_float2(0.f, 0.f);
 
-            // ring row of this unit's window top
+            // ring row of this unit's window top, as a byte offset
             unsigned rb0 = static_cast<unsigned>(it.p0 + py * f.stride);
             rb0 = min(rb0, rb0 - NR);
+            const unsigned rowoff = rb0 * rowBu;
             const int by = ho * f.stride - f.pad;  // grid row of ky = 0 (image coordinates)
             const int bx = wo * f.stride - f.pad;
             unsigned long long slow = 0ull;  // grid points left for the global-memory pass (K*K <= 64)
@@ -486,29 +513,27 @@ fwd_ring_kernel(const __grid_constant__ CUtensorMap xmap, const T* __restrict__ 
                 const float rx = ElemTraits<T>::to_float(rec[jp]);
                 const float ry = ElemTraits<T>::to_float(rec[NP + jp]);
                 const float m = mask_value(ElemTraits<T>::to_float(rec[2 * NP + jp]), mn);
-                // (dy, dx) = fl32(scale * r), their floors and fractions: packed fp32x2
-                // operations, each lane rounded exactly as its scalar counterpart
-                const float2 d = __fmul2_rn(scale2, make_float2(ry, rx));
-                const float2 fl = make_float2(floorf(d.x), floorf(d.y));
-                const float2 l = __fadd2_rn(d, make_float2(-fl.x, -fl.y));  // (ly, lx), exact
+                const float dy = __fmul_rn(f.offset_scale, ry);
+                const float dx = __fmul_rn(f.offset_scale, rx);
+                const float fy0 = floorf(dy), fx0 = floorf(dx);
                 // corner row / column inside the unit's window (saturating conversions;
                 // NaN converts to 0 and is caught by the ordered test below)
-                const unsigned uy = static_cast<unsigned>(__float2int_rz(fl.x)) + static_cast<unsigned>(ky * f.dilation + p.R);
-                const unsigned ux = static_cast<unsigned>(__float2int_rz(fl.y)) + static_cast<unsigned>(kx * f.dilation + p.R);
-                if (max(uy, ux) <= umax && !isnan(d.x + d.y) && fabsf(m) < INFINITY) {
+                const unsigned uy = static_cast<unsigned>(__float2int_rz(fy0)) + static_cast<unsigned>(ky * f.dilation + p.R);
+                const unsigned ux = static_cast<unsigned>(__float2int_rz(fx0)) + static_cast<unsigned>(kx * f.dilation + p.R);
+                if (max(uy, ux) <= umax && !isnan(dy + dx) && fabsf(m) < INFINITY) {
                     // all four corners inside the window; outside-image corners read
                     // the window's zeros and the finite weight adds exactly 0
-                    const float a1 = m * l.x, a0 = m - a1;                    // m ly, m (1 - ly)
-                    const float2 aa = make_float2(a0, a1);
-                    const float2 wr = __fmul2_rn(aa, make_float2(l.y, l.y));   // (w01, w11) = (a0 lx, a1 lx)
-                    const float2 wl = __ffma2_rn(wr, make_float2(-1.f, -1.f), aa);  // (w00, w10): a - w, one rounding
-                    const float w00 = wl.x, w01 = wr.x, w10 = wl.y, w11 = wr.y;
-                    unsigned t = rb0 + uy;  // ring row of the top corners
-                    t = min(t, t - NR);
-                    const int off = static_cast<int>(t) * rowB + (cb + static_cast<int>(ux)) * PB;
+                    const float ly = dy - fy0, lx = dx - fx0;
+                    const float a1 = m * ly, a0 = m - a1;          // m ly, m (1 - ly)
+                    const float w01 = a0 * lx, w00 = a0 - w01;    // a0 lx, a0 (1 - lx)
+                    const float w11 = a1 * lx, w10 = a1 - w11;
+                    // byte offset of the top-left corner in the ring (rows wrap once)
+                    unsigned roff = rowoff + uy * rowBu;
+                    roff = min(roff, roff - ringB);
+                    const unsigned off = roff + ux * PBu;
                     if constexpr (TRACE) {
-                        const int y0 = by + ky * f.dilation + __float2int_rz(fl.x);
-                        const int x0 = bx + kx * f.dilation + __float2int_rz(fl.y);
+                        const int y0 = by + ky * f.dilation + __float2int_rz(fy0);
+                        const int x0 = bx + kx * f.dilation + __float2int_rz(fx0);
                         const bool vy0 = y0 >= 0 && y0 < f.H, vy1 = y0 + 1 >= 0 && y0 + 1 < f.H;
                         const bool vx0 = x0 >= 0 && x0 < f.W, vx1 = x0 + 1 >= 0 && x0 + 1 < f.W;
                         const int bits = (vy0 && vx0 ? 1 : 0) | (vy0 && vx1 ? 2 : 0) | (vy1 && vx0 ? 4 : 0) |
@@ -516,30 +541,28 @@ fwd_ring_kernel(const __grid_constant__ CUtensorMap xmap, const T* __restrict__ 
                         const size_t ti = (static_cast<size_t>((it.n * f.Hout + ho) * f.Wout + wo) * f.G + g) * NP + jp;
                         p.trace[ti] = make_int4(bits ? y0 : INT_MIN, bits ? x0 : INT_MIN, bits, 0);
                     }
-                    if constexpr (HW && std::is_same<T, __half>::value) {
-                        const uint32_t wt = pack_half2(w00, w01), wbt = pack_half2(w10, w11);
 #pragma unroll
-                        for (int j = 0; j < Q; ++j) {
-                            const unsigned char* pc = cbase[j] + off;
-                            const unsigned char* pd = pc + rowB;
-                            const uint4 v00 = *reinterpret_cast<const uint4*>(pc);
-                            const uint4 v01 = *reinterpret_cast<const uint4*>(pc + PB);
-                            const uint4 v10 = *reinterpret_cast<const uint4*>(pd);
-                            const uint4 v11 = *reinterpret_cast<const uint4*>(pd + PB);
+                    for (int j = 0; j < Q; ++j) {
+                        const unsigned a = cbase_s[j] + off;
+                        uint4 v00, v01, v10, v11;
+                        if constexpr (PBC > 0) {
+                            v00 = lds128<0>(a);
+                            v01 = lds128<PBC>(a);
+                            v10 = lds128r(a, rowBu);
+                            v11 = lds128<PBC>(a + rowBu);
+                        } else {
+                            v00 = lds128<0>(a);
+                            v01 = lds128r(a, PBu);
+                            v10 = lds128r(a, rowBu);
+                            v11 = lds128r(a, rowBu + PBu);
+                        }
+                        if constexpr (HW && std::is_same<T, __half>::value) {
+                            const uint32_t wt = pack_half2(w00, w01), wbt = pack_half2(w10, w11);
                             fma_chunk_h<false>(acc[j], wt, v00);
                             fma_chunk_h<true>(acc[j], wt, v01);
                             fma_chunk_h<false>(acc[j], wbt, v10);
                             fma_chunk_h<true>(acc[j], wbt, v11);
-                        }
-                    } else {
-#pragma unroll
-                        for (int j = 0; j < Q; ++j) {
-                            const unsigned char* pc = cbase[j] + off;
-                            const unsigned char* pd = pc + rowB;
-                            const uint4 v00 = *reinterpret_cast<const uint4*>(pc);
-                            const uint4 v01 = *reinterpret_cast<const uint4*>(pc + PB);
-                            const uint4 v10 = *reinterpret_cast<const uint4*>(pd);
-                            const uint4 v11 = *reinterpret_cast<const uint4*>(pd + PB);
+                        } else {
                             fma_chunk<T, HW>(acc[j], w00, v00);
                             fma_chunk<T, HW>(acc[j], w01, v01);
                             fma_chunk<T, HW>(acc[j], w10, v10);
