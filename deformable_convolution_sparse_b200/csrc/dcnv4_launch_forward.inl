@@ -29,7 +29,8 @@ int env_int(const char* name, int dflt) {
 #define DCNV4_RING_UNITS_MAX 480  // consumer threads per CTA (build option, with DCNV4_RING_MAXREG)
 #endif
 constexpr int kUnitsMax = DCNV4_RING_UNITS_MAX;
-static_assert(((kUnitsMax / 32 + 1 + 3) / 4) * DCNV4_RING_MAXREG * 32 <= 16384,
+static_assert(((kUnitsMax / 32 + 1 + 3) / 4) * DCNV4_RING_MAXREG * 32 <= 16384 &&
+                  ((kUnitsMax / 32 + 1 + 3) / 4) * DCNV4_RING_MAXREG_NARROW * 32 <= 16384,
               "the ring kernel's register cap must fit the warps of one SM sub-partition");
 
 // Mean shared-memory wavefronts of one quarter-warp LDS.128 in the ring
@@ -90,9 +91,10 @@ int odd16(int bytes) {
 
 // The halo the planner aims for: samples whose corners stay within R pixels of
 // their unit's grid footprint are gathered from shared memory, so R bounds the
-// offsets served from the window. It grows with the dilation (the spacing of
-// the grid the offsets move around): 6 pixels at dilation 1, 9 at 2 and more.
-int default_halo(int dilation) { return std::min(9, 4 * dilation + 2); }
+// offsets served from the window. The target R = 4*dilation + 1 serves every
+// offset of up to four grid spacings (|d| <= 4*dilation: floor(d) + 1 <= R);
+// the planner considers one pixel less and one more (see plan_ring).
+int target_halo(int dilation) { return std::min(15, 4 * dilation + 1); }
 
 struct RingPlan {
     dcnv4::RingParams p;
@@ -200,7 +202,10 @@ RingShape best_ring_shape(const FwdParams& f, int R, int nsm, int min_units) {
                     const double narrow = std::sqrt(std::sqrt(std::min(1.0, 2.0 * TW * s / WW)));
                     const double lanes = static_cast<double>(units) / (threads - 32);  // filled lanes of the last warp
                     const double cpp = (0.75 * Q + 0.5) / (banks * runs * occ * narrow * lanes);
-                    const double t_compute = rows_per_cta * TW * GS * f.npts * cpp / clk;
+                    // an item of fewer rows takes as long as a full one (one unit per thread)
+                    const int items_h = (f.Hout + TH - 1) / TH;
+                    const double fill_h = static_cast<double>(f.Hout) / (static_cast<double>(items_h) * TH);
+                    const double t_compute = rows_per_cta / fill_h * TW * GS * f.npts * cpp / clk;
                     const double t_start = static_cast<double>(nsm) * (static_cast<double>(nrows) * rowB + rec) / 6.5e6;
                     double t_wait = 0.0;
                     if (NR < 2 * nrows) t_wait += rows_per_cta / f.Hout * (1.0 + static_cast<double>(nrows) * rowB / (100.0 * clk));
@@ -233,17 +238,30 @@ bool plan_ring(const void* x, const void* om, const void* out, const FwdParams& 
     if (f.KK > 64) return false;  // the per-unit mask of points outside the window has 64 bits
     const int nsm = sm_count();
     if (nsm <= 0) return false;
-    int Rhi = default_halo(f.dilation), Rlo = 1;
+    // The halo: among target - 1 .. target + 1, the one whose best plan (at least
+    // 8 consumer warps, or a whole item of a small image) has the shortest
+    // estimated time, with 5 % added per pixel below target + 1 and 10 % more
+    // below the target, for the samples a smaller window sends to the global
+    // pass (the offsets' spread is not known here). Smaller halos only when
+    // nothing in that range fits. Judged for a nominal batch of 64 images on
+    // 148 SMs, so that it depends on the geometry alone and an image's result
+    // does not depend on N.
+    const int Rt = target_halo(f.dilation);
+    int Rhi = Rt + 1, Rlo = std::max(1, Rt - 1);
     if (const int h = env_int("DCNV4_HALO", 0); h > 0) Rhi = Rlo = h;
-    // the largest halo for which a plan with at least 8 consumer warps fits (or
-    // one covering a whole item of a small image); it depends on the geometry
-    // alone, so an image's result does not depend on N
     const int min_units = std::min(256, f.Hout * f.Wout * f.G);
-    int R = -1;
     FwdParams nominal = f;
     nominal.N = 64;
-    for (int r = Rhi; r >= Rlo && R < 0; --r)
-        if (best_ring_shape<T>(nominal, r, 148, min_units).score >= 0.0) R = r;
+    int R = -1;
+    double best_t = 0.0;
+    for (int r = Rhi; r >= Rlo; --r) {
+        const RingShape c = best_ring_shape<T>(nominal, r, 148, min_units);
+        if (c.score <= 0.0) continue;
+        const double t = (1.0 + 0.05 * (Rhi - r) + (r < Rt ? 0.1 : 0.0)) / c.score;
+        if (R < 0 || t < best_t) { R = r; best_t = t; }
+    }
+    for (int r = Rlo - 1; r >= 1 && R < 0; --r)
+        if (best_ring_shape<T>(nominal, r, 148, min_units).score > 0.0) R = r;
     if (R < 0) return false;
     const RingShape sh = best_ring_shape<T>(f, R, nsm, min_units);
     if (sh.score < 0.0) return false;
