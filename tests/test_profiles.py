@@ -2,7 +2,10 @@
 well-formed machine-readable fields (the ones bench.py reads for
 roofline.traffic), and its DRAM bytes are plausible for the workload: at least
 the input bytes a launch must read once and no more than the algorithmic bytes
-plus the fp32 gradients the backward writes."""
+plus the fp32 gradients the backward writes. The forward may read x a second
+time: a band's halo rows are fetched again by the CTA that takes the
+neighbouring band one strip later, when the steps rotate over input sets
+larger than L2 and the rows have been evicted in between."""
 import glob
 import os
 import re
@@ -47,7 +50,7 @@ def test_summary_fields(path):
     out = w.N * w.Hout * w.Wout * w.C * e
     kind = f["pass"]
     if kind == "forward":
-        lo, hi = x + om, x + om + out
+        lo, hi = x + om, x + om + out + x
     elif kind == "backward":
         lo, hi = x + om + out, x + om + out + (x + om) // e * 4
     else:  # predictor: y [pixels, C] read, records written
