@@ -96,6 +96,19 @@ int odd16(int bytes) {
 // the planner considers one pixel less and one more (see plan_ring).
 int target_halo(int dilation) { return std::min(15, 4 * dilation + 1); }
 
+// Image windows need the whole image plus a one-pixel border within one TMA
+// row load (at most 256 pixels) and, for centre feature scaling, every unit's
+// centre grid position inside that border (the kernel reads the centre pixel
+// from the window).
+bool image_window_fits(const FwdParams& f) {
+    if (f.W + 2 > 256) return false;
+    if (f.flags & dcnv4::kFlagCenterScale) {
+        const int c = (f.K / 2) * f.dilation - f.pad;
+        if (c < -1 || (f.Hout - 1) * f.stride + c > f.H || (f.Wout - 1) * f.stride + c > f.W) return false;
+    }
+    return true;
+}
+
 struct RingPlan {
     dcnv4::RingParams p;
     CUtensorMap map;
@@ -104,15 +117,18 @@ struct RingPlan {
 };
 
 struct RingShape {  // one candidate of the planner
-    int GS, R, TW, TH, nrec, NR, units, threads, slot, rec, WW, UH, c2;
+    int GS, R, TW, TH, nrec, NR, units, threads, slot, rec, WW, UH, UW, c2, img;
     size_t smem;
     double score;
 };
 
-// The best plan for halo R (score < 0: none fits) with at least `min_units`
-// consumer threads. Everything but R leaves the per-unit arithmetic unchanged;
-// it is chosen for speed and may depend on N. The score is the inverse of an
-// estimated launch time (microseconds at 1.9 GHz), the sum of
+// The best plan for halo R, or with image windows when `img` (score < 0: none
+// fits), with at least `min_units` consumer threads. Everything but R and the
+// window kind leaves the per-unit arithmetic unchanged; it is chosen for speed
+// and may depend on N. An image window is the whole image plus a one-pixel
+// border (H + 2 rows of W + 2 pixels), one band of all Wout columns, loaded
+// once per strip. The score is the inverse of an estimated launch time
+// (microseconds at 1.9 GHz), the sum of
 //  - compute: a CTA's rows x band width x groups x points at (0.75*Q + 0.5)
 //    SM cycles per sampling point (the measured rate of the 128-byte-pixel
 //    gather), divided by the gather's bank efficiency (1 / wavefronts^2), the
@@ -129,7 +145,7 @@ struct RingShape {  // one candidate of the planner
 //  - items whose rows cannot load during the previous item (NR < nrows +
 //    TH*stride): about 1 us each.
 template <typename T>
-RingShape best_ring_shape(const FwdParams& f, int R, int nsm, int min_units) {
+RingShape best_ring_shape(const FwdParams& f, int R, int nsm, int min_units, bool img = false) {
     constexpr int E = sizeof(T);
     const int row_bytes = f.Cg * E;
     const int Q = row_bytes / 16;
@@ -140,7 +156,8 @@ RingShape best_ring_shape(const FwdParams& f, int R, int nsm, int min_units) {
     const int forceNrec = env_int("DCNV4_NREC", 0);
     const int forceNR = env_int("DCNV4_RING", 0);
     const int s = f.stride;
-    const int UH = (f.K - 1) * f.dilation + 2 * R + 1;
+    const int UH = img ? f.H + 2 : (f.K - 1) * f.dilation + 2 * R + 1;
+    const int UW = img ? f.W + 2 : UH;
     const double clk = 1.9e3;  // SM cycles per microsecond
     RingShape best{};
     best.score = -1.0;
@@ -162,14 +179,18 @@ RingShape best_ring_shape(const FwdParams& f, int R, int nsm, int min_units) {
         const bool row_runs = GS == f.G;
         const double runs = row_runs ? 1.0 : 0.8;
         for (int TW : TWs) {
+            if (img) {
+                if (TW != TWs[0]) break;
+                TW = f.Wout;  // one band
+            }
             if (forceTW && TW != forceTW) continue;
-            if (TW > f.Wout && TW != TWs[0]) {
+            if (!img && TW > f.Wout && TW != TWs[0]) {
                 // one band wider than the image only if no narrower TW covers it
                 bool smaller = false;
                 for (int t2 : TWs) smaller = smaller || (t2 < TW && t2 >= f.Wout);
                 if (smaller) continue;
             }
-            const int WW = (TW - 1) * s + UH;
+            const int WW = img ? UW : (TW - 1) * s + UW;
             if (WW > 256) continue;
             const int rowB = (WW * PB + 127) / 128 * 128;  // ring row pitch: every TMA destination 128-byte aligned
             const int bands = (f.Wout + TW - 1) / TW;
@@ -181,7 +202,7 @@ RingShape best_ring_shape(const FwdParams& f, int R, int nsm, int min_units) {
                 const int units = TH * TW * GS;
                 if (units > kUnitsMax) break;
                 if (units < min_units) continue;
-                const int nrows = (TH - 1) * s + UH;
+                const int nrows = img ? UH : (TH - 1) * s + UH;
                 const int slot = odd16((row_runs ? TW * f.G : GS) * R3 * E + 32);
                 const int rec = ((row_runs ? TH : TH * TW) * slot + 127) / 128 * 128;
                 for (int nrec = 2; nrec <= 4; ++nrec) {
@@ -209,11 +230,12 @@ RingShape best_ring_shape(const FwdParams& f, int R, int nsm, int min_units) {
                     const double t_start = static_cast<double>(nsm) * (static_cast<double>(nrows) * rowB + rec) / 6.5e6;
                     double t_wait = 0.0;
                     if (NR < 2 * nrows) t_wait += rows_per_cta / f.Hout * (1.0 + static_cast<double>(nrows) * rowB / (100.0 * clk));
-                    if (NR < nrows + TH * s) t_wait += rows_per_cta / TH * 1.0;
+                    if (!img && NR < nrows + TH * s) t_wait += rows_per_cta / TH * 1.0;
                     const double t_depth = nrec >= 3 ? 0.0 : 0.01 * t_compute;
                     const double score = 1.0 / (t_compute + t_start + t_wait + t_depth);
                     if (score > best.score) {
-                        best = RingShape{GS, R, TW, TH, nrec, NR, units, threads, slot, rec, WW, UH, c2, smem, score};
+                        best = RingShape{GS, R, TW, TH, nrec, NR, units, threads, slot, rec, WW, UH, UW, c2, img ? 1 : 0,
+                                         smem, score};
                     }
                 }
             }
@@ -248,7 +270,8 @@ bool plan_ring(const void* x, const void* om, const void* out, const FwdParams& 
     // does not depend on N.
     const int Rt = target_halo(f.dilation);
     int Rhi = Rt + 1, Rlo = std::max(1, Rt - 1);
-    if (const int h = env_int("DCNV4_HALO", 0); h > 0) Rhi = Rlo = h;
+    const int force_halo = env_int("DCNV4_HALO", 0);
+    if (force_halo > 0) Rhi = Rlo = force_halo;
     const int min_units = std::min(256, f.Hout * f.Wout * f.G);
     FwdParams nominal = f;
     nominal.N = 64;
@@ -262,14 +285,28 @@ bool plan_ring(const void* x, const void* om, const void* out, const FwdParams& 
     }
     for (int r = Rlo - 1; r >= 1 && R < 0; --r)
         if (best_ring_shape<T>(nominal, r, 148, min_units).score > 0.0) R = r;
-    if (R < 0) return false;
-    const RingShape sh = best_ring_shape<T>(f, R, nsm, min_units);
+    // Image windows serve every offset from shared memory (a sample outside one
+    // has no corner inside the image and adds nothing), so they are taken
+    // whenever their estimated time is no longer than the unit windows' best,
+    // judged for the same nominal batch. DCNV4_WINDOW=unit|image forces the
+    // choice where it fits; a forced halo means unit windows.
+    const char* wenv = std::getenv("DCNV4_WINDOW");
+    const bool force_unit = force_halo > 0 || (wenv && std::strcmp(wenv, "unit") == 0);
+    const bool force_img = !force_unit && wenv && std::strcmp(wenv, "image") == 0;
+    bool img = false;
+    if (!force_unit && image_window_fits(f)) {
+        const RingShape c = best_ring_shape<T>(nominal, 0, 148, min_units, true);
+        img = c.score > 0.0 && (force_img || R < 0 || 1.0 / c.score <= best_t);
+    }
+    if (R < 0 && !img) return false;
+    const RingShape sh = best_ring_shape<T>(f, img ? 0 : R, nsm, min_units, img);
     if (sh.score < 0.0) return false;
 
     dcnv4::RingParams bp{};
     bp.f = f;
     bp.TH = sh.TH; bp.TW = sh.TW; bp.GS = sh.GS; bp.nsub = f.G / sh.GS; bp.R = sh.R;
-    bp.UH = sh.UH; bp.UW = sh.UH; bp.WW = sh.WW; bp.NR = sh.NR;
+    bp.img = sh.img;
+    bp.UH = sh.UH; bp.UW = sh.UW; bp.WW = sh.WW; bp.NR = sh.NR;
     bp.PB = sh.GS * row_bytes;
     bp.rowB = (sh.WW * bp.PB + 127) / 128 * 128;
     bp.cblk = sh.GS * f.Cg / sh.c2;
@@ -315,10 +352,10 @@ bool plan_ring(const void* x, const void* om, const void* out, const FwdParams& 
     plan->threads = sh.threads;
     if (const char* d = std::getenv("DCNV4_DEBUG"); d && *d == '1')
         std::fprintf(stderr,
-                     "dcnv4 ring plan: item %dx%d GS %d (nsub %d) R %d unit window %d window width %d PB %d "
-                     "ring %d rows rows_total %d units %d threads %d nrec %d smem %zu score %.3f\n",
-                     bp.TH, bp.TW, bp.GS, bp.nsub, bp.R, bp.UH, bp.WW, bp.PB, bp.NR, bp.rows_total, bp.units,
-                     sh.threads, bp.nrec, sh.smem, sh.score);
+                     "dcnv4 ring plan: %s windows, item %dx%d GS %d (nsub %d) R %d window %dx%d width %d PB %d "
+                     "ring %d rows rows_total %d units %d threads %d nrec %d smem %zu est %.1f us\n",
+                     bp.img ? "image" : "unit", bp.TH, bp.TW, bp.GS, bp.nsub, bp.R, bp.UH, bp.UW, bp.WW, bp.PB, bp.NR,
+                     bp.rows_total, bp.units, sh.threads, bp.nrec, sh.smem, 1.0 / sh.score);
     return true;
 }
 

@@ -55,9 +55,10 @@ struct RingParams {
     FwdParams f;
     int TH, TW;          // output rows per item (at most), output columns per band
     int GS, nsub;        // groups per strip, G / GS
-    int R;               // halo (pixels) around a unit's grid footprint
-    int UH, UW;          // a unit's window: (K-1)*dilation + 2R + 1 rows and columns
-    int WW;              // window columns: (TW-1)*stride + UW
+    int R;               // halo (pixels) around a unit's grid footprint (unit windows)
+    int img;             // 1: every window is its whole image plus a one-pixel border (image windows)
+    int UH, UW;          // a unit's window: (K-1)*dilation + 2R + 1 rows and columns; image windows: H + 2, W + 2
+    int WW;              // window columns: (TW-1)*stride + UW; image windows: W + 2
     int NR;              // ring rows (a mirror of ring row 0 follows them)
     int PB;              // bytes per window pixel: GS * Cg * sizeof(T)
     int rowB;            // ring row pitch: WW * PB rounded up to 128 bytes (TMA destinations stay aligned)
@@ -145,6 +146,29 @@ __device__ __forceinline__ uint4 pack_chunk(const float2* a) {
     return v;
 }
 
+// m times the four bilinear corner weights of a sample with fractional parts
+// (ly, lx). For a finite m the window path's arithmetic: m ly, m (1 - ly) as
+// m - m ly, and likewise along x, so that both paths give the same bits. For
+// a non-finite m each corner's (m wy) wx, as in the plain definition: an
+// infinite mask then gives +-Inf, or NaN where a weight is 0, per corner
+// (m - m ly would be Inf - Inf = NaN for every corner).
+__device__ __forceinline__ void corner_weights(float m, float ly, float lx, float& w00, float& w01, float& w10,
+                                               float& w11) {
+    if (fabsf(m) < INFINITY) {
+        const float a1 = m * ly, a0 = m - a1;
+        w01 = a0 * lx;
+        w00 = a0 - w01;
+        w11 = a1 * lx;
+        w10 = a1 - w11;
+    } else {
+        const float b0 = m * (1.f - ly), b1 = m * ly;
+        w00 = b0 * (1.f - lx);
+        w01 = b0 * lx;
+        w10 = b1 * (1.f - lx);
+        w11 = b1 * lx;
+    }
+}
+
 // 1.5 * 2^23 and its bit pattern: the floor of |d| < 2^22 by one directed add.
 constexpr float kMagic = 12582912.0f;
 constexpr unsigned kMagicBits = 0x4B400000u;
@@ -226,7 +250,8 @@ __device__ __forceinline__ bool next_item(const RingParams& p, ItemCursor& c, It
     const int strip = static_cast<int>(fdiv(static_cast<unsigned>(c.g), p.div_hout));
     const int ho0 = c.g - strip * f.Hout;
     const int nh = min(p.TH, min(f.Hout - ho0, c.g1 - c.g));
-    const int nrows = (nh - 1) * f.stride + p.UH;
+    // an image window is the same for every item of its strip: loaded once, never advanced
+    const int nrows = p.img ? p.UH : (nh - 1) * f.stride + p.UH;
     const bool cont = strip == c.strip && ho0 == c.ho_end;
     int v, p0;
     if (cont) {
@@ -259,7 +284,7 @@ __device__ __forceinline__ bool next_item(const RingParams& p, ItemCursor& c, It
     c.v = v;
     c.p0 = p0;
     c.nrows = nrows;
-    c.adv = nh * f.stride;
+    c.adv = p.img ? 0 : nh * f.stride;
     return true;
 }
 
@@ -330,8 +355,9 @@ __device__ __forceinline__ void issue_records(const RingParams& p, const T* om, 
 __device__ __forceinline__ void issue_rows(const RingParams& p, const CUtensorMap* xmap, const Item& it,
                                            unsigned char* ring, uint64_t* bar, int lane) {
     const FwdParams& f = p.f;
-    const int img_top = it.ho0 * f.stride - f.pad - p.R;  // image row of the window's first row
-    const int img_left = it.wo0 * f.stride - f.pad - p.R;
+    // image row and column of the window's first row and column
+    const int img_top = p.img ? -1 : it.ho0 * f.stride - f.pad - p.R;
+    const int img_left = p.img ? -1 : it.wo0 * f.stride - f.pad - p.R;
     const int first = img_top + (it.lv - it.v);
     const unsigned box = static_cast<unsigned>(p.WW * p.PB);  // bytes of one row load
     for (int r = lane; r < it.ln; r += 32) {
@@ -470,11 +496,13 @@ fwd_ring_kernel(const __grid_constant__ CUtensorMap xmap, const T* __restrict__ 
     }
     const int rowB = p.rowB;
     const unsigned NR = static_cast<unsigned>(p.NR);
-    const unsigned umax = static_cast<unsigned>(p.UH - 2);  // a unit's window is square: UH == UW
+    // largest window row / column of a top-left corner
+    const unsigned umy = static_cast<unsigned>(p.UH - 2), umx = static_cast<unsigned>(p.UW - 2);
+    const bool img = p.img != 0;
     const int rowC = f.W * f.C;
     const int within = row_runs ? (px * f.G + gl) : gl;  // unit index inside its record run
     const unsigned char* const ubase = ring + gl * (Q * 16);
-    const int cb = px * f.stride;  // this unit's first window column
+    const int cb = img ? 0 : px * f.stride;  // this unit's first window column
     // this lane's chunks of ring pixel (0, cb), in its rotated order (32-bit shared-window addresses)
     unsigned cbase_s[Q];
 #pragma unroll
@@ -510,11 +538,15 @@ fwd_ring_kernel(const __grid_constant__ CUtensorMap xmap, const T* __restrict__ 
                 for (int q = 0; q < CH / 2; ++q) acc[j][q] = make_float2(0.f, 0.f);
 
             // ring row of this unit's window top, as a byte offset
-            unsigned rb0 = static_cast<unsigned>(it.p0 + py * f.stride);
+            unsigned rb0 = static_cast<unsigned>(img ? it.p0 : it.p0 + py * f.stride);
             rb0 = min(rb0, rb0 - NR);
             const unsigned rowoff = rb0 * rowBu;
             const int by = ho * f.stride - f.pad;  // grid row of ky = 0 (image coordinates)
             const int bx = wo * f.stride - f.pad;
+            // window row / column of the grid point (0, 0): R in a unit window, which is
+            // centred on the unit; in an image window (first row and column: image row and
+            // column -1) the grid point's own image coordinates plus one
+            const int cy = img ? by + 1 : p.R, cx = img ? bx + 1 : p.R;
             unsigned long long slow = 0ull;  // grid points left for the global-memory pass (K*K <= 64)
             const MaskNorm mn = VF ? mask_norm(rec + 2 * NP, NP, f.flags) : MaskNorm{0.f, 1.f, false};
 
@@ -535,9 +567,10 @@ fwd_ring_kernel(const __grid_constant__ CUtensorMap xmap, const T* __restrict__ 
                 // pass (where floorf decides as everywhere else).
                 const float ty = __fadd_rd(dy, kMagic), tx = __fadd_rd(dx, kMagic);
                 // corner row / column inside the unit's window
-                const unsigned uy = __float_as_uint(ty) + static_cast<unsigned>(ky * f.dilation + p.R) - kMagicBits;
-                const unsigned ux = __float_as_uint(tx) + static_cast<unsigned>(kx * f.dilation + p.R) - kMagicBits;
-                if (max(uy, ux) <= umax && fabsf(m) < INFINITY) {
+                const unsigned uy = __float_as_uint(ty) + static_cast<unsigned>(ky * f.dilation + cy) - kMagicBits;
+                const unsigned ux = __float_as_uint(tx) + static_cast<unsigned>(kx * f.dilation + cx) - kMagicBits;
+                const bool inwin = uy <= umy && ux <= umx;
+                if (inwin && fabsf(m) < INFINITY) {
                     // all four corners inside the window; outside-image corners read
                     // the window's zeros and the finite weight adds exactly 0
                     const float fy0 = ty - kMagic, fx0 = tx - kMagic;  // floor(dy), floor(dx), exact
@@ -588,8 +621,13 @@ fwd_ring_kernel(const __grid_constant__ CUtensorMap xmap, const T* __restrict__ 
                             fma_chunk<T, HW>(acc[j], w11, v11);
                         }
                     }
-                } else {
+                } else if (inwin || !img) {
                     slow |= 1ull << k;
+                } else if constexpr (TRACE) {
+                    // outside an image window: no corner lies inside the image, the
+                    // sample adds nothing and is skipped
+                    const size_t ti = (static_cast<size_t>((it.n * f.Hout + ho) * f.Wout + wo) * f.G + g) * NP + jp;
+                    p.trace[ti] = make_int4(INT_MIN, INT_MIN, 0, 3);
                 }
             }
             // the points outside the window: global gather with per-corner validity
@@ -622,12 +660,12 @@ fwd_ring_kernel(const __grid_constant__ CUtensorMap xmap, const T* __restrict__ 
                         }
                         if (kk[h] < 0) s.bits = 0u;
                         // the same weight arithmetic as the window path
-                        const float a1 = m * s.ly, a0 = m - a1;
-                        const float w01 = a0 * s.lx, w11 = a1 * s.lx;
-                        w[h][0] = (s.bits & 1u) ? a0 - w01 : 0.f;
-                        w[h][1] = (s.bits & 2u) ? w01 : 0.f;
-                        w[h][2] = (s.bits & 4u) ? a1 - w11 : 0.f;
-                        w[h][3] = (s.bits & 8u) ? w11 : 0.f;
+                        float v00, v01, v10, v11;
+                        corner_weights(m, s.ly, s.lx, v00, v01, v10, v11);
+                        w[h][0] = (s.bits & 1u) ? v00 : 0.f;
+                        w[h][1] = (s.bits & 2u) ? v01 : 0.f;
+                        w[h][2] = (s.bits & 4u) ? v10 : 0.f;
+                        w[h][3] = (s.bits & 8u) ? v11 : 0.f;
                         const T* c00 = ximg + (s.y0 * f.W + s.x0) * f.C + g * f.Cg;
 #pragma unroll
                         for (int cn = 0; cn < 4; ++cn) {
@@ -667,13 +705,8 @@ fwd_ring_kernel(const __grid_constant__ CUtensorMap xmap, const T* __restrict__ 
                     }
                     if (s.bits == 0u) continue;
                     // the same weight arithmetic as the window path
-                    const float a1 = m * s.ly, a0 = m - a1;
-                    const float w01 = a0 * s.lx, w11 = a1 * s.lx;
                     float w[4];
-                    w[0] = (s.bits & 1u) ? a0 - w01 : 0.f;
-                    w[1] = (s.bits & 2u) ? w01 : 0.f;
-                    w[2] = (s.bits & 4u) ? a1 - w11 : 0.f;
-                    w[3] = (s.bits & 8u) ? w11 : 0.f;
+                    corner_weights(m, s.ly, s.lx, w[0], w[1], w[2], w[3]);
                     const T* c00 = ximg + (s.y0 * f.W + s.x0) * f.C + g * f.Cg;
 #pragma unroll
                     for (int cn = 0; cn < 4; ++cn) {
@@ -693,10 +726,11 @@ fwd_ring_kernel(const __grid_constant__ CUtensorMap xmap, const T* __restrict__ 
                 // out = (1 - s) * aggregate + s * x at the centre grid position, read from the
                 // window (which holds zeros outside the image)
                 const float sg = center_gate<T>(f, (static_cast<size_t>((it.n * f.Hout + ho) * f.Wout + wo)) * f.G + g);
-                const int cu = (K / 2) * f.dilation + p.R;
-                unsigned t = rb0 + static_cast<unsigned>(cu);
+                // (an image window holds the centre only when the planner has checked so)
+                const int cu = (K / 2) * f.dilation;
+                unsigned t = rb0 + static_cast<unsigned>(cy + cu);
                 t = min(t, t - NR);
-                const unsigned char* pcx = ubase + static_cast<int>(t) * rowB + (cb + cu) * PB;
+                const unsigned char* pcx = ubase + static_cast<int>(t) * rowB + (cb + cx + cu) * PB;
 #pragma unroll
                 for (int j = 0; j < Q; ++j) blend_chunk<T>(acc[j], sg, *reinterpret_cast<const uint4*>(pcx + choff[j]));
             }

@@ -23,15 +23,20 @@ TOL = {"f32": 1e-5, "f16": 4e-3, "bf16": 4e-3}
 TD = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}
 
 
-@pytest.fixture(params=["window", "window_f16exact", "gather"])
+@pytest.fixture(params=["window", "window_unit", "window_f16exact", "gather"])
 def variant(request, monkeypatch):
-    """Every kernel path: the shared-memory tile kernel (default choice; for
-    fp16 storage with fp16-rounded weights), the same kernel with fp32 weights
-    for fp16 (DCNV4_F16_EXACT=1), and the global-gather kernel (forced with
+    """Every kernel path: the shared-memory ring kernel (default choice: image
+    windows for the small images here, unit windows for the large ones; for
+    fp16 storage with fp16-rounded weights), the ring kernel held to unit
+    windows (DCNV4_WINDOW=unit), the same kernel with fp32 weights for fp16
+    (DCNV4_F16_EXACT=1), and the global-gather kernel (forced with
     DCNV4_VARIANT=gather)."""
     monkeypatch.delenv("DCNV4_VARIANT", raising=False)
     monkeypatch.delenv("DCNV4_F16_EXACT", raising=False)
-    if request.param == "gather":
+    monkeypatch.delenv("DCNV4_WINDOW", raising=False)
+    if request.param == "window_unit":
+        monkeypatch.setenv("DCNV4_WINDOW", "unit")
+    elif request.param == "gather":
         monkeypatch.setenv("DCNV4_VARIANT", "gather")
     elif request.param == "window_f16exact":
         monkeypatch.setenv("DCNV4_F16_EXACT", "1")

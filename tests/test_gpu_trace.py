@@ -5,8 +5,9 @@ bit for bit against the fp64 oracle.
 as ``dcnv4_forward`` (a separate build of the ring kernel with trace stores
 compiled in) and records, per sampling point, the top-left corner, the
 validity bits and the path of the gather: the ring kernel's shared-memory
-window (corner read back from the window address arithmetic), its
-global-memory pass, or the global-gather kernel. The corners and validity must
+window (corner read back from the window address arithmetic, path 0), its
+global-memory pass (1), the global-gather kernel (2), or none: a sample
+outside an image window, which has no corner inside the image (3). The corners and validity must
 equal the oracle's (the sample sits at the regular grid position plus the
 learned offset: "不只是卷积的平替", jsqmd.com, section 1), and the output must be
 the plain forward's bit for bit.
@@ -27,7 +28,8 @@ def _trace_and_check(x, om, dev, **kw):
     out, trace = dcn.forward_trace(xd, omd, **kw)
     plain = dcn.forward(xd, omd, **kw)
     torch.cuda.synchronize()
-    assert torch.equal(out, plain), "the traced forward must write the plain forward's bits"
+    ity = torch.int32 if out.element_size() == 4 else torch.int16
+    assert torch.equal(out.view(ity), plain.view(ity)), "the traced forward must write the plain forward's bits"
     N, H, W, C = x.shape
     c_ref, v_ref = oracle.sampling_index(om.double().numpy(), H, W, **kw)
     t = trace.cpu().numpy()
@@ -41,9 +43,10 @@ def test_named_workload_corners_are_bit_exact(name, cuda_device):
     w = WORKLOADS[name]
     x, om = workload_inputs(w)
     path = _trace_and_check(x, om, cuda_device, **w.kwargs())
-    # the shared-memory window serves these workloads (the ring kernel takes every one)
-    assert (path <= 1).all()
-    assert (path == 0).mean() > 0.9, np.bincount(path.ravel())
+    # the ring kernel takes every one: the shared-memory window serves the samples
+    # (or, for an image window, skips those with no corner inside the image)
+    assert (path != 2).all()
+    assert np.isin(path, (0, 3)).mean() > 0.9, np.bincount(path.ravel())
 
 
 def test_offsets_just_below_integers(cuda_device):
@@ -59,6 +62,43 @@ def test_offsets_just_below_integers(cuda_device):
     x = torch.randn(N, H, W, C)
     path = _trace_and_check(x, om, cuda_device, G=G, K=K, pad=1)
     assert (path == 0).all()
+
+
+@pytest.mark.parametrize("dtype", ["f32", "f16", "bf16"])
+@pytest.mark.parametrize("window", ["unit", "image"])
+def test_window_kinds_route_far_samples(window, dtype, monkeypatch, cuda_device):
+    """Offsets of several image widths: a unit window sends its far samples to
+    the global-memory pass, an image window skips them (no corner of theirs is
+    inside the image); near samples take the shared-memory window either way.
+    Corners and validity must be the oracle's on every path."""
+    monkeypatch.setenv("DCNV4_WINDOW", window)
+    x, om = make_inputs(3, 17, 15, 64, 4, 3, 17, 15, dtype, ("normal", 0, 9), seed=31)
+    path = _trace_and_check(x, om, cuda_device, G=4, K=3, pad=1)
+    assert (path == 0).any()
+    if window == "unit":
+        assert set(np.unique(path)) == {0, 1}
+    else:
+        assert set(np.unique(path)) == {0, 3}
+
+
+def test_image_window_non_finite_masks_take_the_global_pass(monkeypatch, cuda_device):
+    """An image window sends a sample with a non-finite mask and a corner
+    inside the image to the global pass, where only valid corners add (NaN or
+    Inf reaches those outputs alone)."""
+    monkeypatch.setenv("DCNV4_WINDOW", "image")
+    N, H, W, C, G, K = 2, 10, 12, 32, 2, 3
+    x, om = make_inputs(N, H, W, C, G, K, H, W, "f32", ("normal", 0, 3), seed=41)
+    flat = om.view(-1, 27)
+    vals = torch.tensor([float("nan"), float("inf"), -float("inf")])
+    flat[::5, 18 + 4] = vals[torch.arange(flat[::5].shape[0]) % 3]
+    path = _trace_and_check(x, om, cuda_device, G=G, K=K, pad=1)
+    assert (path == 1).any() and set(np.unique(path)) <= {0, 1, 3}
+    out = dcn.forward(x.to(cuda_device), om.to(cuda_device), G=G, K=K, pad=1).cpu().double().numpy()
+    ref = oracle.dcnv4_forward(x.double().numpy(), om.double().numpy(), G=G, K=K, pad=1)
+    fin = np.isfinite(ref)
+    np.testing.assert_array_equal(np.isfinite(out), fin)
+    np.testing.assert_array_equal(np.isnan(out), np.isnan(ref))
+    assert np.abs(out[fin] - ref[fin]).max() <= 1e-5 * np.abs(ref[fin]).max()
 
 
 @pytest.mark.parametrize("halo", ["1", "2", "6"])

@@ -22,11 +22,14 @@ VARIANTS = {
 }
 
 
-@pytest.fixture(params=["window", "window_f16exact", "gather"])
+@pytest.fixture(params=["window", "window_unit", "window_f16exact", "gather"])
 def variant(request, monkeypatch):
     monkeypatch.delenv("DCNV4_VARIANT", raising=False)
     monkeypatch.delenv("DCNV4_F16_EXACT", raising=False)
-    if request.param == "gather":
+    monkeypatch.delenv("DCNV4_WINDOW", raising=False)
+    if request.param == "window_unit":
+        monkeypatch.setenv("DCNV4_WINDOW", "unit")
+    elif request.param == "gather":
         monkeypatch.setenv("DCNV4_VARIANT", "gather")
     elif request.param == "window_f16exact":
         monkeypatch.setenv("DCNV4_F16_EXACT", "1")

@@ -15,7 +15,10 @@ import pytest
 from deformable_convolution_sparse_b200.workloads import WORKLOADS
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-PROFILES = sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md")))
+ALL = sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md")))
+# ncu summaries of a kernel launch, and measurement summaries of probes
+PROFILES = [p for p in ALL if not os.path.basename(p).startswith("probe_")]
+PROBES = [p for p in ALL if os.path.basename(p).startswith("probe_")]
 E = {"f32": 4, "f16": 2, "bf16": 2}
 
 
@@ -58,6 +61,14 @@ def test_summary_fields(path):
     assert 0.99 * lo <= dram <= 1.01 * hi, (lo, dram, hi)
 
 
-@pytest.mark.parametrize("path", PROFILES, ids=os.path.basename)
+@pytest.mark.parametrize("path", PROBES, ids=os.path.basename)
+def test_probe_summary_names_its_command_and_values(path):
+    text = open(path).read()
+    assert "python -c" in text and "probe_smem_gather" in text
+    rates = [float(v) for v in re.findall(r"^\| \d: [^|]+\| ([0-9.]+) \|", text, re.M)]
+    assert len(rates) == 2 and all(16.0 < r <= 128.5 for r in rates), rates
+
+
+@pytest.mark.parametrize("path", ALL, ids=os.path.basename)
 def test_summary_is_short_text(path):
     assert os.path.getsize(path) < 16 * 1024
