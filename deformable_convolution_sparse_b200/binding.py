@@ -34,7 +34,7 @@ EXPORTS = ("dcnv4_output_shape", "dcnv4_validate", "dcnv4_validate_ex", "dcnv4_f
            "dcnv4_forward_trace",
            "dcnv4_backward", "dcnv4_backward_ex", "dcnv4_predictor", "dcnv4_sampling_index",
            "dcnv4_forward_host", "dcnv4_forward_host_noalloc", "dcnv4_device_status", "dcnv4_selftest_wait_timeout",
-           "dcnv4_probe_smem_gather", "dcnv4_strerror", "dcnv4_abi_version")
+           "dcnv4_probe_smem_gather", "dcnv4_probe_red_global", "dcnv4_strerror", "dcnv4_abi_version")
 DEVSTATUS_COPY_TIMEOUT, DEVSTATUS_SELFTEST_TIMEOUT = 1, 2
 
 _lib = None
@@ -88,6 +88,8 @@ def load_library():
     lib.dcnv4_selftest_wait_timeout.restype = i
     lib.dcnv4_probe_smem_gather.argtypes = [i, ctypes.POINTER(ctypes.c_double)]
     lib.dcnv4_probe_smem_gather.restype = i
+    lib.dcnv4_probe_red_global.argtypes = [i, ctypes.POINTER(ctypes.c_double)]
+    lib.dcnv4_probe_red_global.restype = i
     lib.dcnv4_strerror.argtypes = [i]
     lib.dcnv4_strerror.restype = ctypes.c_char_p
     lib.dcnv4_abi_version.argtypes = []
@@ -126,6 +128,15 @@ def probe_smem_gather(pattern: int = 0) -> float:
     rc = load_library().dcnv4_probe_smem_gather(int(pattern), ctypes.byref(v))
     if rc != DCNV4_OK:
         raise DCNv4Error(rc, "dcnv4_probe_smem_gather")
+    return v.value
+
+
+def probe_red_global(segment_bytes: int = 64) -> float:
+    """fp32 vector-reduction payload bytes per SM clock per SM into L2 (dcnv4_probe_red_global; synchronous)."""
+    v = ctypes.c_double(0.0)
+    rc = load_library().dcnv4_probe_red_global(int(segment_bytes), ctypes.byref(v))
+    if rc != DCNV4_OK:
+        raise DCNv4Error(rc, "dcnv4_probe_red_global")
     return v.value
 
 

@@ -99,6 +99,33 @@ probe_smem_gather_kernel(int pattern, int iters) {
     if (threadIdx.x == 0) g_probe_cycles[blockIdx.x] = t1 - t0;
 }
 
+// Global reduction probe (dcnv4_probe_red_global): every warp issues 16-byte
+// fp32 vector reductions (red.global.add.v4.f32) in groups of `group` lanes,
+// each group covering one segment of group*16 contiguous bytes at a random
+// segment of a buffer that stays in L2, 32/group segments per instruction.
+// The rate bounds the backward's scatter into grad_x, whose lanes send each
+// corner's group slice as such a segment.
+__global__ void __launch_bounds__(512)
+probe_red_global_kernel(float* buf, unsigned nseg_mask, int group, int iters) {
+    const int lane = threadIdx.x & 31;
+    const int gi = lane / group, gl = lane - gi * group;
+    unsigned s = 0x9e3779b9u ^ (blockIdx.x * 7919u + (threadIdx.x >> 5) * 104729u);
+    __syncthreads();
+    const unsigned long long t0 = clock64();
+    for (int it = 0; it < iters; ++it) {
+        s = s * 1664525u + 1013904223u;
+        unsigned r = s ^ (static_cast<unsigned>(gi) * 2654435761u);  // the group's own segment
+        r ^= r >> 13;
+        r *= 0x5bd1e995u;
+        r ^= r >> 15;
+        float* q = buf + static_cast<size_t>(r & nseg_mask) * group * 4 + gl * 4;
+        atomicAdd(reinterpret_cast<float4*>(q), make_float4(1.f, 1.f, 1.f, 1.f));
+    }
+    __syncthreads();
+    const unsigned long long t1 = clock64();
+    if (threadIdx.x == 0) g_probe_cycles[blockIdx.x] = t1 - t0;
+}
+
 }  // namespace dcnv4
 
 namespace {
@@ -531,6 +558,37 @@ int dcnv4_probe_smem_gather(int pattern, double* bytes_per_clock_per_sm) {
     for (int i = 0; i < nsm; ++i) mx = std::max(mx, cyc[i]);
     const double loads = static_cast<double>(threads) * iters * 8.0;  // 16-byte loads per CTA
     *bytes_per_clock_per_sm = loads * 16.0 / static_cast<double>(mx);
+    return DCNV4_OK;
+}
+
+int dcnv4_probe_red_global(int segment_bytes, double* bytes_per_clock_per_sm) {
+    if (!bytes_per_clock_per_sm) return DCNV4_ERR_NULL;
+    if (segment_bytes != 32 && segment_bytes != 64 && segment_bytes != 128) return DCNV4_ERR_SHAPE;
+    const int nsm = sm_count();
+    if (nsm <= 0 || nsm > dcnv4::kProbeMaxCtas) return DCNV4_ERR_CUDA;
+    constexpr int threads = 512, iters = 2000;
+    constexpr size_t bytes = size_t{32} << 20;  // 32 MB: resident in L2
+    const int group = segment_bytes / 16;
+    const unsigned nseg = static_cast<unsigned>(bytes / static_cast<size_t>(segment_bytes));  // a power of two
+    float* buf = nullptr;
+    if (cudaMalloc(&buf, bytes) != cudaSuccess) return DCNV4_ERR_CUDA;
+    int rc = DCNV4_OK;
+    if (cudaMemset(buf, 0, bytes) != cudaSuccess) rc = DCNV4_ERR_CUDA;
+    for (int rep = 0; rep < 2 && rc == DCNV4_OK; ++rep) {  // the first launch warms up
+        dcnv4::probe_red_global_kernel<<<nsm, threads>>>(buf, nseg - 1, group, iters);
+        if (cudaGetLastError() != cudaSuccess) rc = DCNV4_ERR_LAUNCH;
+        else if (cudaDeviceSynchronize() != cudaSuccess) rc = DCNV4_ERR_CUDA;
+    }
+    unsigned long long cyc[dcnv4::kProbeMaxCtas];
+    if (rc == DCNV4_OK &&
+        cudaMemcpyFromSymbol(cyc, dcnv4::g_probe_cycles, sizeof(unsigned long long) * nsm) != cudaSuccess)
+        rc = DCNV4_ERR_CUDA;
+    if (cudaFree(buf) != cudaSuccess && rc == DCNV4_OK) rc = DCNV4_ERR_CUDA;
+    if (rc != DCNV4_OK) return rc;
+    unsigned long long mx = 1;
+    for (int i = 0; i < nsm; ++i) mx = std::max(mx, cyc[i]);
+    const double payload = static_cast<double>(threads) * iters * 16.0;  // bytes per CTA
+    *bytes_per_clock_per_sm = payload / static_cast<double>(mx);
     return DCNV4_OK;
 }
 

@@ -12,6 +12,7 @@
 #include <cstring>
 #include <map>
 #include <mutex>
+#include <string>
 
 #include "dcnv4.h"
 #include "dcnv4_internal.h"

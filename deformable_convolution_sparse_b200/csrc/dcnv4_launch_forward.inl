@@ -244,22 +244,10 @@ RingShape best_ring_shape(const FwdParams& f, int R, int nsm, int min_units, boo
     return best;
 }
 
-// Chooses the halo, group subset, band, item height and ring depth for the
-// ring kernel and encodes the tensor map of x; false when the shape or the
-// alignment does not suit it. The halo (the only choice that changes which
-// samples take the window path) depends on the geometry alone, so an image's
-// result never depends on the batch it comes in.
+// The ring kernel's shape for a forward (score < 0: it does not fit): window
+// kind, halo, group subset, band, item height and ring depth.
 template <typename T>
-bool plan_ring(const void* x, const void* om, const void* out, const FwdParams& f, unsigned* status, int4* trace,
-               RingPlan* plan) {
-    constexpr int E = sizeof(T);
-    const int row_bytes = f.Cg * E;
-    if (!aligned(x, 16) || !aligned(out, 16) || (f.C * E) % 16 || row_bytes % 16) return false;
-    const int Q = row_bytes / 16;
-    if (!(Q == 1 || Q == 2 || Q == 4 || Q == 5 || Q == 8)) return false;
-    if (f.KK > 64) return false;  // the per-unit mask of points outside the window has 64 bits
-    const int nsm = sm_count();
-    if (nsm <= 0) return false;
+RingShape choose_ring_shape(const FwdParams& f, int nsm) {
     // The halo: among target - 1 .. target + 1, the one whose best plan (at least
     // 8 consumer warps, or a whole item of a small image) has the shortest
     // estimated time, with 5 % added per pixel below target + 1 and 10 % more
@@ -298,8 +286,52 @@ bool plan_ring(const void* x, const void* om, const void* out, const FwdParams& 
         const RingShape c = best_ring_shape<T>(nominal, 0, 148, min_units, true);
         img = c.score > 0.0 && (force_img || R < 0 || 1.0 / c.score <= best_t);
     }
-    if (R < 0 && !img) return false;
-    const RingShape sh = best_ring_shape<T>(f, img ? 0 : R, nsm, min_units, img);
+    RingShape none{};
+    none.score = -1.0;
+    if (R < 0 && !img) return none;
+    return best_ring_shape<T>(f, img ? 0 : R, nsm, min_units, img);
+}
+
+// choose_ring_shape costs 15-25 us of host time (a few thousand candidate
+// plans); forwards of the same geometry, storage type, SM count and planner
+// overrides reuse its result.
+template <typename T>
+RingShape cached_ring_shape(const FwdParams& f, int nsm) {
+    static std::mutex mu;
+    static std::map<std::string, RingShape> cache;
+    char key[512];
+    const char* names[] = {"DCNV4_HALO", "DCNV4_WINDOW", "DCNV4_TILE", "DCNV4_GS", "DCNV4_NREC", "DCNV4_RING"};
+    int n = std::snprintf(key, sizeof key, "%d %d %d %d %d %d %d %d %d %d %d %d %d %d %d", static_cast<int>(sizeof(T)),
+                          f.N, f.H, f.W, f.C, f.G, f.K, f.stride, f.pad, f.dilation, f.flags, f.npts, f.Hout, f.Wout, nsm);
+    for (const char* e : names) {
+        const char* v = std::getenv(e);
+        n += std::snprintf(key + n, sizeof key - n, " %s=%.32s", e, v ? v : "");
+    }
+    std::lock_guard<std::mutex> lock(mu);
+    if (auto it = cache.find(key); it != cache.end()) return it->second;
+    const RingShape sh = choose_ring_shape<T>(f, nsm);
+    if (cache.size() >= 256) cache.clear();
+    cache.emplace(key, sh);
+    return sh;
+}
+
+// Chooses the halo, group subset, band, item height and ring depth for the
+// ring kernel and encodes the tensor map of x; false when the shape or the
+// alignment does not suit it. The halo (the only choice that changes which
+// samples take the window path) depends on the geometry alone, so an image's
+// result never depends on the batch it comes in.
+template <typename T>
+bool plan_ring(const void* x, const void* om, const void* out, const FwdParams& f, unsigned* status, int4* trace,
+               RingPlan* plan) {
+    constexpr int E = sizeof(T);
+    const int row_bytes = f.Cg * E;
+    if (!aligned(x, 16) || !aligned(out, 16) || (f.C * E) % 16 || row_bytes % 16) return false;
+    const int Q = row_bytes / 16;
+    if (!(Q == 1 || Q == 2 || Q == 4 || Q == 5 || Q == 8)) return false;
+    if (f.KK > 64) return false;  // the per-unit mask of points outside the window has 64 bits
+    const int nsm = sm_count();
+    if (nsm <= 0) return false;
+    const RingShape sh = cached_ring_shape<T>(f, nsm);
     if (sh.score < 0.0) return false;
 
     dcnv4::RingParams bp{};
@@ -379,8 +411,21 @@ int launch_ring_q(const T* x, const T* om, T* out, const RingPlan& plan, cudaStr
         if (dbg) std::fprintf(stderr, "dcnv4 ring launch: shared-memory attribute: %s\n", cudaGetErrorString(attr));
         return DCNV4_ERR_LAUNCH;
     }
+    // resident CTAs per SM for this block size and shared memory (looked up once per pair)
+    static std::mutex occ_mu;
+    static std::map<std::pair<int, size_t>, int> occ_cache;
     int per_sm = 0;
-    const cudaError_t occ = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, plan.threads, plan.smem);
+    cudaError_t occ = cudaSuccess;
+    {
+        std::lock_guard<std::mutex> lock(occ_mu);
+        const auto key = std::make_pair(plan.threads, plan.smem);
+        if (auto it = occ_cache.find(key); it != occ_cache.end()) {
+            per_sm = it->second;
+        } else {
+            occ = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, plan.threads, plan.smem);
+            if (occ == cudaSuccess && per_sm >= 1) occ_cache.emplace(key, per_sm);
+        }
+    }
     if (occ != cudaSuccess || per_sm < 1) {
         if (dbg) std::fprintf(stderr, "dcnv4 ring launch: occupancy %d (%s) for %d threads, %zu bytes\n", per_sm,
                               cudaGetErrorString(occ), plan.threads, plan.smem);
@@ -388,8 +433,21 @@ int launch_ring_q(const T* x, const T* om, T* out, const RingPlan& plan, cudaStr
     }
     const long long slots = static_cast<long long>(sm_count()) * per_sm;
     const unsigned grid = static_cast<unsigned>(std::min<long long>(plan.p.rows_total, slots));
-    kern<<<grid, plan.threads, plan.smem, stream>>>(plan.map, x, om, out, plan.p);
-    const cudaError_t le = cudaGetLastError();
+    // programmatic stream serialisation: the CTAs may launch (and set up their
+    // barriers) while the previous kernel on the stream drains; the kernel waits
+    // for it before its first global access (DCNV4_PDL=0: plain serialisation)
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(static_cast<unsigned>(plan.threads));
+    cfg.dynamicSmemBytes = plan.smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute pdl[1];
+    pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = pdl;
+    cfg.numAttrs = env_int("DCNV4_PDL", 1) != 0 ? 1 : 0;
+    cudaError_t le = cudaLaunchKernelEx(&cfg, kern, plan.map, x, om, out, plan.p);
+    if (le == cudaSuccess) le = cudaGetLastError();
     if (le != cudaSuccess && dbg) std::fprintf(stderr, "dcnv4 ring launch: %s\n", cudaGetErrorString(le));
     return le == cudaSuccess ? DCNV4_OK : DCNV4_ERR_LAUNCH;
 }

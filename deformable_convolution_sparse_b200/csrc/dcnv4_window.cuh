@@ -433,6 +433,13 @@ fwd_ring_kernel(const __grid_constant__ CUtensorMap xmap, const T* __restrict__ 
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&xmap)) : "memory");
     }
     __syncthreads();
+    // Launched with programmatic stream serialisation, this grid may start while
+    // the kernel before it on the stream is still running: wait for that grid to
+    // complete (and its writes to be visible) before touching global memory,
+    // then let the next launch on the stream start its own prologue as our SMs
+    // free up. Without a programmatic dependency both return at once.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     if (warp == nc) {
         // ---------------------------------------------------------------- producer

@@ -393,6 +393,19 @@ DCNV4_API int dcnv4_selftest_wait_timeout(unsigned long long limit_ns, void *str
  * DCNV4_ERR_CUDA. */
 DCNV4_API int dcnv4_probe_smem_gather(int pattern, double *bytes_per_clock_per_sm);
 
+/* Measures this GPU's rate of fp32 vector reductions into L2, the ceiling of
+ * the backward's scatter into grad_x (each sampling point adds m * W * dL/dout
+ * to 4 corners x C/G fp32 channels). The pages have no counterpart; it backs
+ * the roofline discussion of the backward. One CTA of 512 threads per SM;
+ * each warp instruction is a 16-byte `red.global.add.v4.f32` per lane, lanes
+ * grouped so that each group covers one segment of `segment_bytes` (32, 64 or
+ * 128) contiguous bytes at a random segment of a 32 MB buffer (resident in
+ * L2). Writes the payload bytes per SM clock per SM (the slowest CTA's clock64
+ * span). Allocates and frees its buffer; synchronous (legacy default stream,
+ * waits for the device). Returns DCNV4_OK, DCNV4_ERR_NULL, DCNV4_ERR_SHAPE
+ * (segment size not 32, 64 or 128), DCNV4_ERR_LAUNCH or DCNV4_ERR_CUDA. */
+DCNV4_API int dcnv4_probe_red_global(int segment_bytes, double *bytes_per_clock_per_sm);
+
 /* Static description of an error code; never NULL. */
 DCNV4_API const char *dcnv4_strerror(int status);
 

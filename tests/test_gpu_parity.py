@@ -323,3 +323,33 @@ def test_an_image_result_does_not_depend_on_its_batch(dtype, cuda_device):
         part = dcn.forward(x[lo:hi].contiguous().to(cuda_device), om[lo:hi].contiguous().to(cuda_device),
                            G=4, K=3, pad=1).cpu()
         assert torch.equal(part, full[lo:hi]), (lo, hi)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "f16", "bf16"])
+def test_chained_launches_read_the_previous_output(dtype, monkeypatch, cuda_device):
+    """Each forward of a chain reads the previous one's output as its input, with
+    no synchronisation between the launches (the ring kernel is launched with
+    programmatic stream serialisation and waits for the grid before it): the
+    chain must give the bits of the same chain run launch by launch, and of
+    the same chain with plain serialisation (DCNV4_PDL=0)."""
+    monkeypatch.delenv("DCNV4_VARIANT", raising=False)
+    N, H, W, C, G, K = 16, 28, 28, 64, 4, 3
+    x, om = make_inputs(N, H, W, C, G, K, H, W, dtype, ("normal", 0, 1.5), ("normal", 0, 0.5), seed=61)
+    oms = [om.roll(i, dims=0).to(cuda_device) for i in range(6)]
+
+    def chain(sync):
+        cur = x.to(cuda_device)
+        for o in oms:
+            cur = dcn.forward(cur, o, G=G, K=K, pad=1)
+            if sync:
+                torch.cuda.synchronize()
+        torch.cuda.synchronize()
+        return cur
+
+    fast = chain(False)
+    stepwise = chain(True)
+    monkeypatch.setenv("DCNV4_PDL", "0")
+    plain = chain(False)
+    ity = torch.int32 if fast.element_size() == 4 else torch.int16
+    assert torch.equal(fast.view(ity), stepwise.view(ity))
+    assert torch.equal(fast.view(ity), plain.view(ity))

@@ -1,6 +1,7 @@
-"""GPU: the shared-memory gather probe returns a rate inside what the hardware
-can deliver (at most one 128-byte wavefront per SM clock), for the plain
-random-row pattern and for the forward kernel's own corner pattern."""
+"""GPU: the probes return rates inside what the hardware can deliver: the
+shared-memory gather (at most one 128-byte wavefront per SM clock) for the
+plain random-row pattern and the forward kernel's own corner pattern, and the
+fp32 vector reductions into L2 that bound the backward's scatter."""
 import pytest
 
 import deformable_convolution_sparse_b200 as dcn
@@ -12,3 +13,12 @@ pytestmark = pytest.mark.gpu
 def test_probe_rate_is_plausible(pattern, cuda_device):
     rate = dcn.probe_smem_gather(pattern)
     assert 16.0 < rate <= 128.5, rate
+
+
+def test_reduction_probe_rates_are_plausible_and_grow_with_the_segment(cuda_device):
+    """fp32 vector reductions into L2: payload per SM clock stays below the
+    SM's 64-byte-per-clock L1 -> L2 path, and fuller segments (more of a
+    128-byte line per request) move at least as many bytes per clock."""
+    rates = [dcn.probe_red_global(b) for b in (32, 64, 128)]
+    assert all(1.0 < r < 64.0 for r in rates), rates
+    assert rates[0] <= rates[1] * 1.05 and rates[1] <= rates[2] * 1.05, rates
