@@ -34,7 +34,7 @@ EXPORTS = ("dcnv4_output_shape", "dcnv4_validate", "dcnv4_validate_ex", "dcnv4_f
            "dcnv4_forward_trace",
            "dcnv4_backward", "dcnv4_backward_ex", "dcnv4_predictor", "dcnv4_sampling_index",
            "dcnv4_forward_host", "dcnv4_forward_host_noalloc", "dcnv4_device_status", "dcnv4_selftest_wait_timeout",
-           "dcnv4_probe_smem_gather", "dcnv4_probe_red_global", "dcnv4_strerror", "dcnv4_abi_version")
+           "dcnv4_probe_smem_gather", "dcnv4_probe_red_global", "dcnv4_probe_red_shared", "dcnv4_strerror", "dcnv4_abi_version")
 DEVSTATUS_COPY_TIMEOUT, DEVSTATUS_SELFTEST_TIMEOUT = 1, 2
 
 _lib = None
@@ -90,6 +90,8 @@ def load_library():
     lib.dcnv4_probe_smem_gather.restype = i
     lib.dcnv4_probe_red_global.argtypes = [i, ctypes.POINTER(ctypes.c_double)]
     lib.dcnv4_probe_red_global.restype = i
+    lib.dcnv4_probe_red_shared.argtypes = [i, ctypes.POINTER(ctypes.c_double)]
+    lib.dcnv4_probe_red_shared.restype = i
     lib.dcnv4_strerror.argtypes = [i]
     lib.dcnv4_strerror.restype = ctypes.c_char_p
     lib.dcnv4_abi_version.argtypes = []
@@ -137,6 +139,15 @@ def probe_red_global(segment_bytes: int = 64) -> float:
     rc = load_library().dcnv4_probe_red_global(int(segment_bytes), ctypes.byref(v))
     if rc != DCNV4_OK:
         raise DCNv4Error(rc, "dcnv4_probe_red_global")
+    return v.value
+
+
+def probe_red_shared(fp32: bool = True) -> float:
+    """Shared-memory atomic adds per SM clock per SM, fp32 or 32-bit integer (dcnv4_probe_red_shared)."""
+    v = ctypes.c_double(0.0)
+    rc = load_library().dcnv4_probe_red_shared(1 if fp32 else 0, ctypes.byref(v))
+    if rc != DCNV4_OK:
+        raise DCNv4Error(rc, "dcnv4_probe_red_shared")
     return v.value
 
 

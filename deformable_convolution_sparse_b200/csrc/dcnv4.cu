@@ -99,6 +99,31 @@ probe_smem_gather_kernel(int pattern, int iters) {
     if (threadIdx.x == 0) g_probe_cycles[blockIdx.x] = t1 - t0;
 }
 
+// Shared-memory atomic probe (dcnv4_probe_red_shared): every thread adds 1 to
+// a word of a 32 KB shared array, each lane of a warp on its own bank (the
+// word a lane picks is lane + 32 * random row), as fp32 adds or as 32-bit
+// integer adds. The rate decides whether a backward could accumulate grad_x
+// contributions in shared memory before sending them to L2.
+template <bool F32>
+__global__ void __launch_bounds__(512) probe_red_shared_kernel(int iters, float* sink) {
+    __shared__ float words[8192];
+    for (int i = threadIdx.x; i < 8192; i += blockDim.x) words[i] = 0.f;
+    __syncthreads();
+    const unsigned lane = threadIdx.x & 31u;
+    unsigned s = 12345u + 977u * threadIdx.x + 31u * blockIdx.x;
+    const unsigned long long t0 = clock64();
+    for (int it = 0; it < iters; ++it) {
+        s = s * 1664525u + 1013904223u;
+        const unsigned idx = ((s >> 8) & 255u) * 32u + lane;
+        if constexpr (F32) atomicAdd(&words[idx], 1.0f);
+        else atomicAdd(reinterpret_cast<unsigned*>(&words[idx]), 1u);
+    }
+    __syncthreads();
+    const unsigned long long t1 = clock64();
+    if (threadIdx.x == 0) g_probe_cycles[blockIdx.x] = t1 - t0;
+    if (threadIdx.x == 0 && words[7] == -1.f) sink[0] = words[7];  // keeps the adds
+}
+
 // Global reduction probe (dcnv4_probe_red_global): every warp issues 16-byte
 // fp32 vector reductions (red.global.add.v4.f32) in groups of `group` lanes,
 // each group covering one segment of group*16 contiguous bytes at a random
@@ -589,6 +614,33 @@ int dcnv4_probe_red_global(int segment_bytes, double* bytes_per_clock_per_sm) {
     for (int i = 0; i < nsm; ++i) mx = std::max(mx, cyc[i]);
     const double payload = static_cast<double>(threads) * iters * 16.0;  // bytes per CTA
     *bytes_per_clock_per_sm = payload / static_cast<double>(mx);
+    return DCNV4_OK;
+}
+
+int dcnv4_probe_red_shared(int fp32, double* adds_per_clock_per_sm) {
+    if (!adds_per_clock_per_sm) return DCNV4_ERR_NULL;
+    if (fp32 != 0 && fp32 != 1) return DCNV4_ERR_SHAPE;
+    const int nsm = sm_count();
+    if (nsm <= 0 || nsm > dcnv4::kProbeMaxCtas) return DCNV4_ERR_CUDA;
+    constexpr int threads = 512, iters = 4096;
+    float* sink = nullptr;
+    if (cudaMalloc(&sink, 16) != cudaSuccess) return DCNV4_ERR_CUDA;
+    int rc = DCNV4_OK;
+    for (int rep = 0; rep < 2 && rc == DCNV4_OK; ++rep) {  // the first launch warms up
+        if (fp32) dcnv4::probe_red_shared_kernel<true><<<nsm, threads>>>(iters, sink);
+        else dcnv4::probe_red_shared_kernel<false><<<nsm, threads>>>(iters, sink);
+        if (cudaGetLastError() != cudaSuccess) rc = DCNV4_ERR_LAUNCH;
+        else if (cudaDeviceSynchronize() != cudaSuccess) rc = DCNV4_ERR_CUDA;
+    }
+    unsigned long long cyc[dcnv4::kProbeMaxCtas];
+    if (rc == DCNV4_OK &&
+        cudaMemcpyFromSymbol(cyc, dcnv4::g_probe_cycles, sizeof(unsigned long long) * nsm) != cudaSuccess)
+        rc = DCNV4_ERR_CUDA;
+    if (cudaFree(sink) != cudaSuccess && rc == DCNV4_OK) rc = DCNV4_ERR_CUDA;
+    if (rc != DCNV4_OK) return rc;
+    unsigned long long mx = 1;
+    for (int i = 0; i < nsm; ++i) mx = std::max(mx, cyc[i]);
+    *adds_per_clock_per_sm = static_cast<double>(threads) * iters / static_cast<double>(mx);
     return DCNV4_OK;
 }
 

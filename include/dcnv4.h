@@ -406,6 +406,17 @@ DCNV4_API int dcnv4_probe_smem_gather(int pattern, double *bytes_per_clock_per_s
  * (segment size not 32, 64 or 128), DCNV4_ERR_LAUNCH or DCNV4_ERR_CUDA. */
 DCNV4_API int dcnv4_probe_red_global(int segment_bytes, double *bytes_per_clock_per_sm);
 
+/* Measures this GPU's rate of atomic adds to shared memory, which decides
+ * whether a backward could sum grad_x contributions in shared memory before
+ * sending them to L2. The pages have no counterpart. One CTA of 512 threads per
+ * SM; each thread adds 1 to a word of a 32 KB shared array, every lane of a
+ * warp on its own bank; fp32 != 0: `atomicAdd` on fp32 words, else on 32-bit
+ * unsigned words. Writes the adds per SM clock per SM (the slowest CTA's
+ * clock64 span). Synchronous (legacy default stream, waits for the device).
+ * Returns DCNV4_OK, DCNV4_ERR_NULL, DCNV4_ERR_SHAPE (fp32 not 0 or 1),
+ * DCNV4_ERR_LAUNCH or DCNV4_ERR_CUDA. */
+DCNV4_API int dcnv4_probe_red_shared(int fp32, double *adds_per_clock_per_sm);
+
 /* Static description of an error code; never NULL. */
 DCNV4_API const char *dcnv4_strerror(int status);
 

@@ -279,3 +279,10 @@ def test_probe_red_global_checks_before_any_cuda_call():
     assert lib.dcnv4_probe_red_global(64, None) == B.STATUS["DCNV4_ERR_NULL"]
     for bad in (0, 16, 48, 256):
         assert lib.dcnv4_probe_red_global(bad, ctypes.byref(v)) == B.STATUS["DCNV4_ERR_SHAPE"]
+
+
+def test_probe_red_shared_checks_before_any_cuda_call():
+    lib = B.load_library()
+    v = ctypes.c_double(0.0)
+    assert lib.dcnv4_probe_red_shared(1, None) == B.STATUS["DCNV4_ERR_NULL"]
+    assert lib.dcnv4_probe_red_shared(2, ctypes.byref(v)) == B.STATUS["DCNV4_ERR_SHAPE"]

@@ -22,3 +22,11 @@ def test_reduction_probe_rates_are_plausible_and_grow_with_the_segment(cuda_devi
     rates = [dcn.probe_red_global(b) for b in (32, 64, 128)]
     assert all(1.0 < r < 64.0 for r in rates), rates
     assert rates[0] <= rates[1] * 1.05 and rates[1] <= rates[2] * 1.05, rates
+
+
+def test_shared_atomic_probe_rates_are_plausible(cuda_device):
+    """Atomic adds to shared memory, one bank per lane: at most 32 per SM clock
+    (one warp instruction per clock), fp32 and integer alike."""
+    for fp32 in (True, False):
+        r = dcn.probe_red_shared(fp32)
+        assert 0.1 < r <= 32.5, (fp32, r)
