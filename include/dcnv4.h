@@ -40,8 +40,10 @@
  * x, offset_mask and out share one storage type (dtype).
  *
  * Conventions:
- *   - Every call is thread-safe; the library keeps no pointer after return
- *     and allocates no device memory.
+ *   - Every call is thread-safe; the library keeps no pointer to caller
+ *     memory after return and allocates no device memory (the probes below
+ *     excepted). It caches, in host memory and per geometry, storage type
+ *     and SM count, the forward's choice of kernel plan.
  *   - Compute calls are asynchronous on `stream` (a cudaStream_t; NULL is the
  *     legacy default stream) and never synchronise. Arguments are checked on
  *     the host before anything is launched; on a non-zero return nothing was
@@ -144,7 +146,10 @@ DCNV4_API int dcnv4_validate(const void *x, const void *offset_mask, const void 
  * pointers in the layouts above. Runs dcnv4_validate first and returns its
  * code without launching when it fails. On success one kernel is launched
  * on `stream` (none when N == 0) and DCNV4_OK is returned; the result is
- * ready when the stream reaches that point. */
+ * ready when the stream reaches that point. The launch uses programmatic
+ * stream serialisation: its CTAs may start while the previous kernel on the
+ * stream finishes, and wait for that kernel to complete before they read or
+ * write global memory, so stream order holds as for any launch. */
 DCNV4_API int dcnv4_forward(const void *x, const void *offset_mask, void *out,
                   int N, int H, int W, int C, int G, int K,
                   int stride, int pad, int dilation, float offset_scale, int dtype,
