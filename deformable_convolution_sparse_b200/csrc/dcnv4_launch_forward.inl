@@ -303,8 +303,9 @@ RingShape cached_ring_shape(const FwdParams& f, int nsm) {
     const char* names[] = {"DCNV4_HALO", "DCNV4_WINDOW", "DCNV4_TILE", "DCNV4_GS", "DCNV4_NREC", "DCNV4_RING"};
     int n = std::snprintf(key, sizeof key, "%d %d %d %d %d %d %d %d %d %d %d %d %d %d %d", static_cast<int>(sizeof(T)),
                           f.N, f.H, f.W, f.C, f.G, f.K, f.stride, f.pad, f.dilation, f.flags, f.npts, f.Hout, f.Wout, nsm);
-    for (const char* e : names) {
+    for (const char* e : names) {  // at most 46 bytes each: the key stays within its 512 bytes
         const char* v = std::getenv(e);
+        if (n < 0 || n >= static_cast<int>(sizeof key)) break;
         n += std::snprintf(key + n, sizeof key - n, " %s=%.32s", e, v ? v : "");
     }
     std::lock_guard<std::mutex> lock(mu);
