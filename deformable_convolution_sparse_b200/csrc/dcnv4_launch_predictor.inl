@@ -88,7 +88,20 @@ int launch_predictor(const void* y, const void* w, const float* bias, void* rec,
                         std::fprintf(stderr, "dcnv4 predictor: tcgen05 NP %d kblocks %d stages %d out bufs %d tiles %d "
                                      "grid %u smem %zu tmem cols %u epilogue warps %d\n", p.NP, p.kblocks, p.stages,
                                      p.out_bufs, p.tiles, grid, smem, p.tmem_cols, epw);
-                    kern<<<grid, threads, smem, stream>>>(amap, bmap, bias, static_cast<T*>(rec), p);
+                    // programmatic stream serialisation, as for the forward (DCNV4_PDL=0: plain)
+                    cudaLaunchConfig_t cfg{};
+                    cfg.gridDim = dim3(grid);
+                    cfg.blockDim = dim3(static_cast<unsigned>(threads));
+                    cfg.dynamicSmemBytes = smem;
+                    cfg.stream = stream;
+                    cudaLaunchAttribute pdl[1];
+                    pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+                    pdl[0].val.programmaticStreamSerializationAllowed = 1;
+                    cfg.attrs = pdl;
+                    const char* pe = std::getenv("DCNV4_PDL");
+                    cfg.numAttrs = (pe && *pe == '0') ? 0 : 1;
+                    if (cudaLaunchKernelEx(&cfg, kern, amap, bmap, bias, static_cast<T*>(rec), p) != cudaSuccess)
+                        return DCNV4_ERR_LAUNCH;
                     return launch_status();
                 }
             }

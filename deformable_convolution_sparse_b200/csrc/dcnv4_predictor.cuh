@@ -202,6 +202,11 @@ predictor_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_const
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
+    // Launched with programmatic stream serialisation: wait for the previous
+    // kernel on the stream (complete, its writes visible) before the first
+    // global access, then let the next launch start its set-up as SMs free up.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     for (int o = tid; o < p.NO; o += blockDim.x) {
         const int d = pred_dest(o, p.G, p.P);
         src[d] = o;

@@ -113,3 +113,44 @@ def test_predictor_then_aggregation_matches_the_oracle_pipeline(cuda_device):
     assert np.abs(out.double().cpu().numpy() - ref).max() <= 4e-3 * np.abs(ref).max()
     # ... and the records themselves match the oracle's predictor
     _check(rec.view(-1, wl.G, 3 * P), y.view(-1, wl.C), w, b, wl.G, P, "f16")
+
+
+def test_predictor_and_aggregation_chained_without_synchronisation(monkeypatch, cuda_device):
+    """predictor -> forward -> predictor -> forward ... on one stream with no
+    synchronisation: both kernels are launched with programmatic stream
+    serialisation and wait for the kernel before them, so every forward reads
+    the records its predictor wrote and every predictor the activations it was
+    given. The chain must give the bits of the same chain with a device
+    synchronisation after every launch, and of plain serialisation
+    (DCNV4_PDL=0)."""
+    for v in ("DCNV4_PRED_VARIANT", "DCNV4_PRED_EPI", "DCNV4_PRED_STAGES", "DCNV4_PRED_WSTAGE", "DCNV4_VARIANT"):
+        monkeypatch.delenv(v, raising=False)
+    wl = WORKLOADS["stage1_f16"]
+    n = 8
+    P = wl.K * wl.K
+    x, _ = make_inputs(n, wl.H, wl.W, wl.C, wl.G, wl.K, wl.Hout, wl.Wout, "f16", seed=15)
+    ws = []
+    for i in range(4):
+        _, w, b = _tensors(8, wl.C, wl.G, P, "f16", seed=20 + i, scale=0.05)
+        ws.append((w.to(cuda_device), b.to(cuda_device)))
+    x0 = x.to(cuda_device)
+
+    def chain(sync):
+        cur = x0
+        for w, b in ws:
+            rec = dcn.predictor(cur, w, b, G=wl.G, K=wl.K)      # the activations themselves as the predictor input
+            if sync:
+                torch.cuda.synchronize()
+            cur = dcn.forward(cur, rec, **wl.kwargs())
+            if sync:
+                torch.cuda.synchronize()
+        torch.cuda.synchronize()
+        return cur
+
+    fast = chain(False)
+    step = chain(True)
+    monkeypatch.setenv("DCNV4_PDL", "0")
+    plain = chain(False)
+    assert torch.equal(fast.view(torch.int16), step.view(torch.int16))
+    assert torch.equal(fast.view(torch.int16), plain.view(torch.int16))
+    assert torch.isfinite(fast).all()
