@@ -35,6 +35,39 @@
 
 namespace dcnv4 {
 
+// locate() without the conversion pipe, for geometries whose grid positions
+// and image sizes stay below 2^21 in magnitude (the caller checks; others call
+// locate()). floor(d) of a scaled offset |d| < 2^22 is one directed add:
+// d + 1.5*2^23 rounded toward -inf is exactly floor(d) + 1.5*2^23, whose bit
+// pattern minus 0x4B400000 is floor(d). For larger offsets, infinities and NaN
+// that difference (taken modulo 2^32) is at least 2^22 in magnitude, so every
+// corner falls outside such an image, as in locate(). Inside, the corners,
+// validity and fractional parts are locate()'s bit for bit.
+__device__ __forceinline__ Sample locate_small(int p0y, int p0x, float ry, float rx, float scale, int H, int W) {
+    constexpr float kMag = 12582912.0f;
+    constexpr unsigned kMagBits = 0x4B400000u;
+    Sample s;
+    const float dy = __fmul_rn(scale, ry);
+    const float dx = __fmul_rn(scale, rx);
+    const float ty = __fadd_rd(dy, kMag), tx = __fadd_rd(dx, kMag);
+    s.ly = dy - (ty - kMag);
+    s.lx = dx - (tx - kMag);
+    // y0 + 1 and x0 + 1 as unsigned: inside [0, H] x [0, W] iff some corner is in the image
+    const unsigned uy = __float_as_uint(ty) - kMagBits + static_cast<unsigned>(p0y + 1);
+    const unsigned ux = __float_as_uint(tx) - kMagBits + static_cast<unsigned>(p0x + 1);
+    s.bits = 0u;
+    s.y0 = 0;
+    s.x0 = 0;
+    if (uy <= static_cast<unsigned>(H) && ux <= static_cast<unsigned>(W)) {
+        s.y0 = static_cast<int>(uy) - 1;
+        s.x0 = static_cast<int>(ux) - 1;
+        const bool vy0 = uy >= 1u, vy1 = uy + 1u <= static_cast<unsigned>(H);
+        const bool vx0 = ux >= 1u, vx1 = ux + 1u <= static_cast<unsigned>(W);
+        s.bits = (vy0 && vx0 ? 1u : 0u) | (vy0 && vx1 ? 2u : 0u) | (vy1 && vx0 ? 4u : 0u) | (vy1 && vx1 ? 8u : 0u);
+    }
+    return s;
+}
+
 // CPL channels of storage type T at p (8 or 16 bytes when CPL > 1) -> floats
 template <typename T, int CPL>
 __device__ __forceinline__ void load_channels(const T* p, float (&v)[CPL]) {
@@ -90,7 +123,12 @@ __device__ __forceinline__ void scatter_add(float* dst, float a, const float (&v
 // Jacobian maps dL/dm' to dL/dm, and centre scaling adds s dL/dout at the
 // centre pixel of grad_x and writes dL/dz = s (1 - s) (sum_c g x_c -
 // sum_j m'_j u_j), u_j = sum_c g S_j, to grad_z.
-template <typename T, int CPL, int KS, bool VF>
+// LN: the lanes per unit as a compile-time constant when every lane owns
+// exactly one chunk (p.chunks == p.lanes == LN; the fp32/fp16/bf16 16-channel
+// groups: 4 lanes of 4 channels), 0 otherwise. With LN the lane's dL/dout
+// chunk is loaded once per unit instead of once per point, and the chunk loop
+// and the lane folds unroll.
+template <typename T, int CPL, int KS, bool VF, int LN = 0>
 __global__ void __launch_bounds__(256)
 bwd_kernel(const T* __restrict__ x, const T* __restrict__ om, const T* __restrict__ go,
            float* __restrict__ grad_x, float* __restrict__ grad_om, float* __restrict__ grad_z, FwdParams p) {
@@ -108,8 +146,9 @@ bwd_kernel(const T* __restrict__ x, const T* __restrict__ om, const T* __restric
     const T* rec_base = stage_run<T>(om + static_cast<size_t>(unit0) * R, nunits * R, smem_raw);
     __syncthreads();
 
-    const int lu = threadIdx.x / p.lanes;
-    const int part = threadIdx.x - lu * p.lanes;
+    const int lanes = LN > 0 ? LN : p.lanes;
+    const int lu = threadIdx.x / lanes;
+    const int part = threadIdx.x - lu * lanes;
     const bool active = lu < nunits;
     int n = 0, ho = 0, wo = 0, g = 0;
     if (active) unit_coords(unit0 + lu, p, n, ho, wo, g);
@@ -125,6 +164,21 @@ bwd_kernel(const T* __restrict__ x, const T* __restrict__ om, const T* __restric
     const float sg = cs ? center_gate<T>(p, unit) : 0.f;   // centre gate s
     const float keep = 1.f - sg;                            // the aggregation's share of dL/dout
     float mu = 0.f;                                         // sum_j m'_j u_j (centre scaling)
+    // locate_small() applies (LN builds): grid positions and image sizes below 2^21 in magnitude
+    const bool small = LN > 0 &&
+                       static_cast<long long>(p.Hout) * p.stride + p.pad + static_cast<long long>(p.K) * p.dilation +
+                               p.H < (1LL << 21) &&
+                       static_cast<long long>(p.Wout) * p.stride + p.pad + static_cast<long long>(p.K) * p.dilation +
+                               p.W < (1LL << 21);
+    float g1[CPL];                                          // LN: this lane's chunk of dL/dout
+    if constexpr (LN > 0) {
+        if (active) {
+            load_channels<T, CPL>(gop + part * CPL, g1);
+        } else {
+#pragma unroll
+            for (int q = 0; q < CPL; ++q) g1[q] = 0.f;
+        }
+    }
 
 #pragma unroll (KS > 0 ? KS * KS : 1)
     for (int k = 0; k < KK; ++k) {
@@ -136,7 +190,8 @@ bwd_kernel(const T* __restrict__ x, const T* __restrict__ om, const T* __restric
         const float rx = ElemTraits<T>::to_float(rec[jp]);
         const float ry = ElemTraits<T>::to_float(rec[NP + jp]);
         const float m = mask_value(ElemTraits<T>::to_float(rec[2 * NP + jp]), mn);
-        Sample s = locate(p0y, p0x, ry, rx, p.offset_scale, p.H, p.W);
+        Sample s = small ? locate_small(p0y, p0x, ry, rx, p.offset_scale, p.H, p.W)
+                         : locate(p0y, p0x, ry, rx, p.offset_scale, p.H, p.W);
         if (!active) s.bits = 0u;
 
         float gm = 0.f, gfx = 0.f, gfy = 0.f;
@@ -147,12 +202,20 @@ bwd_kernel(const T* __restrict__ x, const T* __restrict__ om, const T* __restric
             const float a1 = ms * ly, a0 = ms - a1;
             const float w01 = a0 * lx, w00 = a0 - w01, w11 = a1 * lx, w10 = a1 - w11;
             const float wc[4] = {w00, w01, w10, w11};
-            const size_t c00 = static_cast<size_t>(s.y0 * p.W + s.x0) * p.C;
-            const size_t coff[4] = {c00, c00 + p.C, c00 + rowC, c00 + rowC + p.C};
-            for (int ch = part; ch < p.chunks; ch += p.lanes) {
+            // element offsets inside the image (LN builds: 32-bit, an image holds fewer
+            // than 2^31 elements, checked on the host)
+            using Off = typename std::conditional<(LN > 0), unsigned, size_t>::type;
+            const Off c00 = static_cast<Off>(s.y0 * p.W + s.x0) * static_cast<Off>(p.C);
+            const Off coff[4] = {c00, c00 + p.C, c00 + rowC, c00 + rowC + p.C};
+            for (int ch = part; ch < (LN > 0 ? part + 1 : p.chunks); ch += lanes) {
                 const int c0 = g * p.Cg + ch * CPL;
                 float gv[CPL], xv[4][CPL];
-                load_channels<T, CPL>(gop + ch * CPL, gv);
+                if constexpr (LN > 0) {
+#pragma unroll
+                    for (int q = 0; q < CPL; ++q) gv[q] = g1[q];
+                } else {
+                    load_channels<T, CPL>(gop + ch * CPL, gv);
+                }
 #pragma unroll
                 for (int cn = 0; cn < 4; ++cn) {
                     if (s.bits & (1u << cn)) {
@@ -181,10 +244,19 @@ bwd_kernel(const T* __restrict__ x, const T* __restrict__ om, const T* __restric
             }
         }
         // every lane of the warp reaches the folds (inactive lanes carry zeros)
-        for (int o = p.lanes >> 1; o > 0; o >>= 1) {
-            gm += __shfl_xor_sync(0xffffffffu, gm, o);
-            gfx += __shfl_xor_sync(0xffffffffu, gfx, o);
-            gfy += __shfl_xor_sync(0xffffffffu, gfy, o);
+        if constexpr (LN > 0) {
+#pragma unroll
+            for (int o = LN >> 1; o > 0; o >>= 1) {
+                gm += __shfl_xor_sync(0xffffffffu, gm, o);
+                gfx += __shfl_xor_sync(0xffffffffu, gfx, o);
+                gfy += __shfl_xor_sync(0xffffffffu, gfy, o);
+            }
+        } else {
+            for (int o = p.lanes >> 1; o > 0; o >>= 1) {
+                gm += __shfl_xor_sync(0xffffffffu, gm, o);
+                gfx += __shfl_xor_sync(0xffffffffu, gfx, o);
+                gfy += __shfl_xor_sync(0xffffffffu, gfy, o);
+            }
         }
         if (active && part == 0) {
             const float ms = (VF ? m * keep : m) * p.offset_scale;
@@ -211,7 +283,7 @@ bwd_kernel(const T* __restrict__ x, const T* __restrict__ om, const T* __restric
             float gxc = 0.f;
             if (inside) {
                 const size_t cpix = static_cast<size_t>(cy * p.W + cx) * p.C;
-                for (int ch = part; ch < p.chunks; ch += p.lanes) {
+                for (int ch = part; ch < p.chunks; ch += lanes) {
                     const int c0 = g * p.Cg + ch * CPL;
                     float gv[CPL], xv[CPL];
                     load_channels<T, CPL>(gop + ch * CPL, gv);
@@ -221,7 +293,7 @@ bwd_kernel(const T* __restrict__ x, const T* __restrict__ om, const T* __restric
                     scatter_add<CPL>(gimg + cpix + c0, sg, gv);
                 }
             }
-            for (int o = p.lanes >> 1; o > 0; o >>= 1) gxc += __shfl_xor_sync(0xffffffffu, gxc, o);
+            for (int o = lanes >> 1; o > 0; o >>= 1) gxc += __shfl_xor_sync(0xffffffffu, gxc, o);
             if (active && part == 0) grad_z[unit] = sg * (1.f - sg) * (gxc - mu);
         }
     }

@@ -41,10 +41,14 @@ int launch_backward(const void* x, const void* om, const void* go, float* gx, fl
         return launch_status();
     };
     const bool k3 = p.K == 3;
+    // 16-channel groups on the vector path: four lanes of one chunk each, lanes known at compile time
+    const bool four = vec && p.chunks == 4 && lanes == 4;
     if (p.flags != 0) {  // the variants: their own instantiations, so that the plain backward carries none of it
+        if (four) return k3 ? run(dcnv4::bwd_kernel<T, 4, 3, true, 4>) : run(dcnv4::bwd_kernel<T, 4, 0, true, 4>);
         if (vec) return k3 ? run(dcnv4::bwd_kernel<T, 4, 3, true>) : run(dcnv4::bwd_kernel<T, 4, 0, true>);
         return k3 ? run(dcnv4::bwd_kernel<T, 1, 3, true>) : run(dcnv4::bwd_kernel<T, 1, 0, true>);
     }
+    if (four) return k3 ? run(dcnv4::bwd_kernel<T, 4, 3, false, 4>) : run(dcnv4::bwd_kernel<T, 4, 0, false, 4>);
     if (vec) return k3 ? run(dcnv4::bwd_kernel<T, 4, 3, false>) : run(dcnv4::bwd_kernel<T, 4, 0, false>);
     return k3 ? run(dcnv4::bwd_kernel<T, 1, 3, false>) : run(dcnv4::bwd_kernel<T, 1, 0, false>);
 }
