@@ -74,6 +74,23 @@ template <> CUtensorMapDataType tma_dtype<float>() { return CU_TENSOR_MAP_DATA_T
 template <> CUtensorMapDataType tma_dtype<__half>() { return CU_TENSOR_MAP_DATA_TYPE_FLOAT16; }
 template <> CUtensorMapDataType tma_dtype<__nv_bfloat16>() { return CU_TENSOR_MAP_DATA_TYPE_BFLOAT16; }
 
+// Raises a kernel's dynamic shared-memory limit, once per kernel and device
+// (function attributes belong to each device's context); returns the result
+// of that first call.
+cudaError_t smem_limit_once(const void* kern, int bytes) {
+    static std::mutex mu;
+    static std::map<std::pair<const void*, int>, cudaError_t> done;
+    int dev = 0;
+    const cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lock(mu);
+    const auto key = std::make_pair(kern, dev);
+    if (auto it = done.find(key); it != done.end()) return it->second;
+    const cudaError_t r = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    done.emplace(key, r);
+    return r;
+}
+
 int sm_count() {
     int dev = 0, n = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)

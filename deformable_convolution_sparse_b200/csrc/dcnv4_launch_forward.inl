@@ -402,11 +402,7 @@ bool f16_exact_from_env() {
 template <typename T, int Q, int KS, bool HW, int PBC, bool VF, bool TRACE>
 int launch_ring_q(const T* x, const T* om, T* out, const RingPlan& plan, cudaStream_t stream) {
     auto kern = dcnv4::fwd_ring_kernel<T, Q, KS, HW, PBC, VF, TRACE>;
-    static std::once_flag once;
-    static cudaError_t attr = cudaSuccess;
-    std::call_once(once, [&] {
-        attr = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kTileSmemLimit));
-    });
+    const cudaError_t attr = smem_limit_once(reinterpret_cast<const void*>(kern), static_cast<int>(kTileSmemLimit));
     const bool dbg = std::getenv("DCNV4_DEBUG") != nullptr;
     if (attr != cudaSuccess) {
         if (dbg) std::fprintf(stderr, "dcnv4 ring launch: shared-memory attribute: %s\n", cudaGetErrorString(attr));

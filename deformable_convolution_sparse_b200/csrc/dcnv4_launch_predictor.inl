@@ -69,18 +69,9 @@ int launch_predictor(const void* y, const void* w, const float* bias, void* rec,
                     if (const char* e = std::getenv("DCNV4_PRED_EPI")) epw = std::atoi(e) == 8 ? 8 : 16;
                     auto kern = epw == 8 ? dcnv4::predictor_tc_kernel<T, 8> : dcnv4::predictor_tc_kernel<T, 16>;
                     const int threads = 64 + 32 * epw;
-                    static std::once_flag once;
-                    static cudaError_t attr = cudaSuccess;
-                    std::call_once(once, [&] {
-                        attr = cudaFuncSetAttribute(dcnv4::predictor_tc_kernel<T, 8>,
-                                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                    static_cast<int>(kTileSmemLimit));
-                        if (attr == cudaSuccess)
-                            attr = cudaFuncSetAttribute(dcnv4::predictor_tc_kernel<T, 16>,
-                                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                        static_cast<int>(kTileSmemLimit));
-                    });
-                    if (attr != cudaSuccess) return DCNV4_ERR_LAUNCH;
+                    if (smem_limit_once(reinterpret_cast<const void*>(kern), static_cast<int>(kTileSmemLimit)) !=
+                        cudaSuccess)
+                        return DCNV4_ERR_LAUNCH;
                     const int nsm = sm_count();
                     if (nsm <= 0) return DCNV4_ERR_CUDA;
                     const unsigned grid = static_cast<unsigned>(std::min(p.tiles, nsm));
