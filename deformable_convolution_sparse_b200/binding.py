@@ -34,7 +34,7 @@ EXPORTS = ("dcnv4_output_shape", "dcnv4_validate", "dcnv4_validate_ex", "dcnv4_f
            "dcnv4_forward_trace",
            "dcnv4_backward", "dcnv4_backward_ex", "dcnv4_predictor", "dcnv4_sampling_index",
            "dcnv4_forward_host", "dcnv4_forward_host_noalloc", "dcnv4_device_status", "dcnv4_selftest_wait_timeout",
-           "dcnv4_probe_smem_gather", "dcnv4_probe_red_global", "dcnv4_probe_red_shared", "dcnv4_strerror", "dcnv4_abi_version")
+           "dcnv4_probe_smem_gather", "dcnv4_probe_red_global", "dcnv4_probe_red_shared", "dcnv4_forward_plan", "dcnv4_strerror", "dcnv4_abi_version")
 DEVSTATUS_COPY_TIMEOUT, DEVSTATUS_SELFTEST_TIMEOUT = 1, 2
 
 _lib = None
@@ -92,6 +92,8 @@ def load_library():
     lib.dcnv4_probe_red_global.restype = i
     lib.dcnv4_probe_red_shared.argtypes = [i, ctypes.POINTER(ctypes.c_double)]
     lib.dcnv4_probe_red_shared.restype = i
+    lib.dcnv4_forward_plan.argtypes = [i] * 10 + [ctypes.c_uint, i, ctypes.POINTER(ctypes.c_int), i]
+    lib.dcnv4_forward_plan.restype = i
     lib.dcnv4_strerror.argtypes = [i]
     lib.dcnv4_strerror.restype = ctypes.c_char_p
     lib.dcnv4_abi_version.argtypes = []
@@ -149,6 +151,25 @@ def probe_red_shared(fp32: bool = True) -> float:
     if rc != DCNV4_OK:
         raise DCNv4Error(rc, "dcnv4_probe_red_shared")
     return v.value
+
+
+PLAN_FIELDS = ("kernel", "image_windows", "halo", "groups_per_strip", "band_columns", "item_rows", "ring_rows",
+               "items_in_flight", "units_per_item", "threads", "smem_bytes", "unit_window_rows",
+               "unit_window_cols", "window_pixels", "pixel_bytes")
+
+
+def forward_plan(N: int, H: int, W: int, C: int, G: int, K: int, stride: int = 1, pad: int = 0, dilation: int = 1,
+                 dtype: int = DCNV4_F32, flags: int = 0, nsm: int = 148) -> dict:
+    """The forward's plan for a geometry (dcnv4_forward_plan; no GPU needed): the kernel
+    choice and the ring kernel's shape, as a dict keyed by PLAN_FIELDS."""
+    buf = (ctypes.c_int * len(PLAN_FIELDS))()
+    rc = load_library().dcnv4_forward_plan(N, H, W, C, G, K, stride, pad, dilation, int(dtype), int(flags), int(nsm),
+                                           buf, len(PLAN_FIELDS))
+    if rc != DCNV4_OK:
+        raise DCNv4Error(rc, "dcnv4_forward_plan")
+    d = dict(zip(PLAN_FIELDS, list(buf)))
+    d["kernel"] = "ring" if d["kernel"] == 0 else "gather"
+    return d
 
 
 def output_shape(H: int, W: int, K: int, stride: int = 1, pad: int = 0, dilation: int = 1):

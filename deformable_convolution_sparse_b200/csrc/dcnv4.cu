@@ -323,6 +323,26 @@ int dcnv4_forward_ex(const void* x, const void* offset_mask, const void* center_
     return run_forward(x, offset_mask, out, p, dtype, nullptr, static_cast<cudaStream_t>(stream));
 }
 
+int dcnv4_forward_plan(int N, int H, int W, int C, int G, int K, int stride, int pad, int dilation, int dtype,
+                       unsigned flags, int nsm, int* fields, int nfields) {
+    long long nx = 0, nout = 0, nom = 0;
+    int rc = check_sizes(N, H, W, C, G, K, stride, pad, dilation, 1.0f, dtype, &nx, &nout, &nom);
+    if (rc) return rc;
+    if (flags & ~static_cast<unsigned>(DCNV4_FLAG_SOFTMAX | DCNV4_FLAG_REMOVE_CENTER | DCNV4_FLAG_CENTER_SCALE))
+        return DCNV4_ERR_FLAGS;
+    if ((flags & DCNV4_FLAG_REMOVE_CENTER) && (K % 2 == 0 || K < 3)) return DCNV4_ERR_SHAPE;
+    if (!fields) return DCNV4_ERR_NULL;
+    if (nfields < DCNV4_PLAN_FIELDS || nsm < 1 || nsm > 1024) return DCNV4_ERR_SHAPE;
+    int Hout = 0, Wout = 0;
+    dcnv4_output_shape(H, W, K, stride, pad, dilation, &Hout, &Wout);
+    const FwdParams p = make_params(N, H, W, C, G, K, stride, pad, dilation, 1.0f, Hout, Wout, flags);
+    switch (dtype) {
+        case DCNV4_F32: return dcnv4_host::plan_f32(p, nsm, fields);
+        case DCNV4_F16: return dcnv4_host::plan_f16(p, nsm, fields);
+        default: return dcnv4_host::plan_bf16(p, nsm, fields);
+    }
+}
+
 int dcnv4_forward(const void* x, const void* offset_mask, void* out,
                   int N, int H, int W, int C, int G, int K,
                   int stride, int pad, int dilation, float offset_scale, int dtype,

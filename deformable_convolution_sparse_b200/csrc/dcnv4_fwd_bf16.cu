@@ -6,3 +6,7 @@ int dcnv4_host::forward_bf16(const void* x, const void* om, void* out, const dcn
                           int4* trace, cudaStream_t stream) {
     return launch_forward<__nv_bfloat16>(x, om, out, p, status, trace, stream);
 }
+
+int dcnv4_host::plan_bf16(const dcnv4::FwdParams& p, int nsm, int* fields) {
+    return plan_fields<__nv_bfloat16>(p, nsm, fields);
+}

@@ -25,4 +25,10 @@ int forward_f16(const void* x, const void* om, void* out, const dcnv4::FwdParams
 int forward_bf16(const void* x, const void* om, void* out, const dcnv4::FwdParams& p, unsigned* status, int4* trace,
                  cudaStream_t stream);
 
+// The forward's plan for a geometry on `nsm` SMs, without launching (15
+// fields, the order of dcnv4_forward_plan in dcnv4.h).
+int plan_f32(const dcnv4::FwdParams& p, int nsm, int* fields);
+int plan_f16(const dcnv4::FwdParams& p, int nsm, int* fields);
+int plan_bf16(const dcnv4::FwdParams& p, int nsm, int* fields);
+
 }  // namespace dcnv4_host

@@ -422,6 +422,25 @@ DCNV4_API int dcnv4_probe_red_global(int segment_bytes, double *bytes_per_clock_
  * DCNV4_ERR_LAUNCH or DCNV4_ERR_CUDA. */
 DCNV4_API int dcnv4_probe_red_shared(int fp32, double *adds_per_clock_per_sm);
 
+/* The forward's plan for a geometry, without launching anything or touching
+ * the GPU (the kernel choice and the ring kernel's shape that dcnv4_forward /
+ * dcnv4_forward_ex would use with 16-byte-aligned pointers on a GPU of `nsm`
+ * SMs, 1..1024). Writes DCNV4_PLAN_FIELDS ints to `fields` (nfields >= that):
+ *   [0] kernel: 0 the ring kernel, 1 the global-gather kernel (the other fields 0)
+ *   [1] 1: image windows (the whole image plus a one-pixel border), 0: unit windows
+ *   [2] halo R of the unit windows   [3] groups per strip      [4] output columns per band
+ *   [5] output rows per item         [6] ring rows             [7] items in flight
+ *   [8] units (pixel, group) per item  [9] threads per CTA     [10] dynamic shared memory (bytes)
+ *   [11] window rows and [12] columns of a unit (image windows: H + 2, W + 2)
+ *   [13] window pixels per ring row  [14] bytes per window pixel
+ * The planner overrides of the environment (DCNV4_WINDOW, DCNV4_HALO,
+ * DCNV4_TILE, DCNV4_GS, DCNV4_NREC, DCNV4_RING) apply as in the forward.
+ * Returns DCNV4_OK or the first failing check of dcnv4_validate_ex's sizes
+ * and flags, DCNV4_ERR_NULL (fields) or DCNV4_ERR_SHAPE (nfields or nsm). */
+#define DCNV4_PLAN_FIELDS 15
+DCNV4_API int dcnv4_forward_plan(int N, int H, int W, int C, int G, int K, int stride, int pad, int dilation,
+                                 int dtype, unsigned flags, int nsm, int *fields, int nfields);
+
 /* Static description of an error code; never NULL. */
 DCNV4_API const char *dcnv4_strerror(int status);
 

@@ -47,6 +47,12 @@ def test_named_workload_corners_are_bit_exact(name, cuda_device):
     # (or, for an image window, skips those with no corner inside the image)
     assert (path != 2).all()
     assert np.isin(path, (0, 3)).mean() > 0.9, np.bincount(path.ravel())
+    # the paths agree with the plan the library reports for this geometry
+    dt = {"f32": dcn.DCNV4_F32, "f16": dcn.DCNV4_F16, "bf16": dcn.DCNV4_BF16}[w.dtype]
+    plan = dcn.forward_plan(w.N, w.H, w.W, w.C, w.G, w.K, w.stride, w.pad, w.dilation, dt)
+    assert plan["kernel"] == "ring"
+    if not plan["image_windows"]:
+        assert not (path == 3).any()
 
 
 def test_offsets_just_below_integers(cuda_device):
