@@ -499,62 +499,80 @@ int dcnv4_forward_host(const void* x_host, const void* offset_mask_host, void* o
     rc = host_pipe(&pipe);
     if (rc) return rc;
     cudaStream_t user = static_cast<cudaStream_t>(stream);
-    // chunks of whole images on NS streams, so that copies in the two directions and the kernels overlap;
-    // DCNV4_HOST_CHUNKS (the most chunks) / DCNV4_HOST_STREAMS override the defaults for tuning runs
-    int max_chunks = 16, NS = 3;
-    if (const char* c = std::getenv("DCNV4_HOST_CHUNKS")) max_chunks = std::max(1, std::atoi(c));
-    if (const char* c = std::getenv("DCNV4_HOST_STREAMS")) NS = std::min(3, std::max(1, std::atoi(c)));
-    cudaEvent_t ev_start = nullptr, ev_done[3] = {nullptr, nullptr, nullptr};
+    // The library's three streams have one role each: s[0] copies the inputs in, s[1] runs the
+    // kernels, s[2] copies the results out. A chunk's kernel waits for its own inputs (ev_in) and
+    // its copy out for its kernel (ev_k); the copies in wait for nothing but each other, so the
+    // host-to-device direction, which carries x and offset_mask against the other's one result,
+    // runs back to back while the other overlaps it. cudaStreamWaitEvent takes the event's latest
+    // record at the time of the call, so one event per role serves every chunk.
+    cudaEvent_t ev_start = nullptr, ev_in = nullptr, ev_k = nullptr, ev_done[3] = {nullptr, nullptr, nullptr};
     bool queued = false;  // copies or kernels are on the library's streams
     // Ends the call: once anything is queued the caller's stream waits for all
     // of it, on success and after an error alike, so that no copy into out_host
     // is still pending when the caller's stream moves on.
     auto fail = [&](int code) {
         if (queued) {
-            for (int i = 0; i < NS; ++i) {
+            for (int i = 0; i < 3; ++i) {
                 const bool ok = ev_done[i] && cudaEventRecord(ev_done[i], pipe->s[i]) == cudaSuccess &&
                                 cudaStreamWaitEvent(user, ev_done[i], 0) == cudaSuccess;
                 if (!ok && code == DCNV4_OK) code = DCNV4_ERR_CUDA;
             }
         }
         // events may be destroyed while pending: the waits already queued keep their meaning
-        if (ev_start) cudaEventDestroy(ev_start);
-        for (auto& ev : ev_done)
+        for (cudaEvent_t ev : {ev_start, ev_in, ev_k, ev_done[0], ev_done[1], ev_done[2]})
             if (ev) cudaEventDestroy(ev);
         return code;
     };
-    if (cudaEventCreateWithFlags(&ev_start, cudaEventDisableTiming) != cudaSuccess) return fail(DCNV4_ERR_CUDA);
-    for (auto& ev : ev_done)
-        if (cudaEventCreateWithFlags(&ev, cudaEventDisableTiming) != cudaSuccess) return fail(DCNV4_ERR_CUDA);
+    for (cudaEvent_t* ev : {&ev_start, &ev_in, &ev_k, &ev_done[0], &ev_done[1], &ev_done[2]})
+        if (cudaEventCreateWithFlags(ev, cudaEventDisableTiming) != cudaSuccess) return fail(DCNV4_ERR_CUDA);
     if (cudaEventRecord(ev_start, user) != cudaSuccess) return fail(DCNV4_ERR_CUDA);
-    for (int i = 0; i < NS; ++i)
+    for (int i = 0; i < 3; ++i)
         if (cudaStreamWaitEvent(pipe->s[i], ev_start, 0) != cudaSuccess) return fail(DCNV4_ERR_CUDA);
 
-    // about 4 MiB of copies per chunk (smaller ones are dominated by per-copy overhead), 2..max_chunks
-    const size_t step_bytes = static_cast<size_t>(N) * (x_img + om_img + out_img);
-    int chunks = static_cast<int>(std::min<size_t>(static_cast<size_t>(max_chunks),
-                                                   std::max<size_t>(2, step_bytes >> 22)));
+    // Chunks of whole images, about 8 MiB of input copies each, 2 to 8 of them: every copy costs
+    // the copy engine a few microseconds beyond its bytes (measured ~3.7 us on PCIe 5), while the
+    // last chunk's kernel and copy out are the part of the call that nothing overlaps, so neither
+    // many small chunks nor one large one. DCNV4_HOST_CHUNKS sets the count (tuning runs).
+    // When a result is no larger than an image's offset_mask records, x goes over first in one
+    // copy and only the records are chunked: one copy less per chunk, and the results' copies
+    // out still have the records' transfer time to overlap with (with larger results they would
+    // queue up behind the last chunk).
+    const size_t in_bytes = static_cast<size_t>(N) * (x_img + om_img);
+    int chunks = static_cast<int>(std::min<size_t>(8, std::max<size_t>(2, in_bytes >> 23)));
+    if (const char* c = std::getenv("DCNV4_HOST_CHUNKS")) chunks = std::max(1, std::atoi(c));
     if (chunks > N) chunks = N;
+    const bool x_first = out_img <= om_img;
     const char* xh = static_cast<const char*>(x_host);
     const char* omh = static_cast<const char*>(offset_mask_host);
     char* oh = static_cast<char*>(out_host);
     char* xd = static_cast<char*>(x_dev);
     char* omd = static_cast<char*>(offset_mask_dev);
     char* od = static_cast<char*>(out_dev);
+    cudaStream_t s_in = pipe->s[0], s_k = pipe->s[1], s_out = pipe->s[2];
+    if (x_first) {
+        queued = true;
+        if (cudaMemcpyAsync(xd, xh, N * x_img, cudaMemcpyHostToDevice, s_in) != cudaSuccess)
+            return fail(DCNV4_ERR_CUDA);
+    }
     int n0 = 0;
     for (int c = 0; c < chunks; ++c) {
         const int n1 = static_cast<int>((static_cast<long long>(N) * (c + 1)) / chunks);
         const int nc = n1 - n0;
         if (nc == 0) continue;
-        cudaStream_t s = pipe->s[c % NS];
         queued = true;
-        if (cudaMemcpyAsync(xd + n0 * x_img, xh + n0 * x_img, nc * x_img, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-            cudaMemcpyAsync(omd + n0 * om_img, omh + n0 * om_img, nc * om_img, cudaMemcpyHostToDevice, s) != cudaSuccess)
+        if ((!x_first &&
+             cudaMemcpyAsync(xd + n0 * x_img, xh + n0 * x_img, nc * x_img, cudaMemcpyHostToDevice, s_in) !=
+                 cudaSuccess) ||
+            cudaMemcpyAsync(omd + n0 * om_img, omh + n0 * om_img, nc * om_img, cudaMemcpyHostToDevice, s_in) !=
+                cudaSuccess ||
+            cudaEventRecord(ev_in, s_in) != cudaSuccess || cudaStreamWaitEvent(s_k, ev_in, 0) != cudaSuccess)
             return fail(DCNV4_ERR_CUDA);
         rc = dcnv4_forward(xd + n0 * x_img, omd + n0 * om_img, od + n0 * out_img, nc, H, W, C, G, K, stride, pad,
-                           dilation, offset_scale, dtype, s);
+                           dilation, offset_scale, dtype, s_k);
         if (rc) return fail(rc);
-        if (cudaMemcpyAsync(oh + n0 * out_img, od + n0 * out_img, nc * out_img, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        if (cudaEventRecord(ev_k, s_k) != cudaSuccess || cudaStreamWaitEvent(s_out, ev_k, 0) != cudaSuccess ||
+            cudaMemcpyAsync(oh + n0 * out_img, od + n0 * out_img, nc * out_img, cudaMemcpyDeviceToHost, s_out) !=
+                cudaSuccess)
             return fail(DCNV4_ERR_CUDA);
         n0 = n1;
     }

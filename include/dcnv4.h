@@ -306,10 +306,15 @@ DCNV4_API int dcnv4_forward_trace(const void *x, const void *offset_mask, void *
  * result. x_dev, offset_mask_dev, out_dev: caller-owned device buffers of the
  * full sizes of x, offset_mask and out, used as staging (their contents
  * afterwards: the copied inputs and the result). The batch is split into
- * chunks of whole images; each chunk's host-to-device copies, kernel and
- * device-to-host copy are queued on one of two library-owned non-blocking
- * streams (created once per device on first use and kept until exit), so the
- * copies of neighbouring chunks overlap in the two copy directions. The call
+ * chunks of whole images (about 8 MiB of input copies each, 2 to 8 of them)
+ * and the work is queued on three library-owned non-blocking streams
+ * (created once per device on first use and kept until exit), one per role:
+ * the host-to-device copies back to back on the first (all of x in one copy
+ * ahead of the chunks' offset_mask copies when an image's result is no
+ * larger than its offset_mask, else each chunk's x and offset_mask), each
+ * chunk's kernel on the second once its inputs have arrived, each chunk's
+ * device-to-host copy on the third once its kernel is done; so the two copy
+ * directions and the kernels overlap. The call
  * is ordered after the work already queued on `stream`, and `stream` waits for
  * all of it before its next work: synchronise `stream` before reading
  * out_host. Checks: those of dcnv4_forward on the device buffers, plus NULL
@@ -352,7 +357,9 @@ DCNV4_API int dcnv4_forward_host(const void *x_host, const void *offset_mask_hos
  *     contents; nothing in it needs to start at zero (inputs are copied in
  *     whole, the output is written in whole). Calls whose work overlaps on the
  *     GPU race on the array: queue them on one stream, or order them.
- *   - Ordering, streams and the other checks are those of dcnv4_forward_host
+ *   - Chunks alternate between two of the library's streams, one staging
+ *     half each (a chunk's copies in, kernel and copy out on one stream).
+ *   - Ordering and the other checks are those of dcnv4_forward_host
  *     (the host pointers are checked for NULL, alignment and overlap); the
  *     result is in out_host once `stream` reaches the end of the call's work. After an error return
  *     that came once copies were queued, `stream` still waits for them (see

@@ -23,6 +23,30 @@ def test_host_path_equals_device_path(N, pinned, cuda_device):
     assert torch.equal(out, ref)
 
 
+@pytest.mark.parametrize("chunks", [None, "7", "1"])
+def test_host_path_chunkings_equal_device_path(chunks, cuda_device, monkeypatch):
+    # 45 stage-1 sized images (results smaller than their records: x goes over in one copy ahead
+    # of the records' chunks): the library's own chunking, 7 uneven chunks and a single chunk
+    if chunks is not None:
+        monkeypatch.setenv("DCNV4_HOST_CHUNKS", chunks)
+    x, om = make_inputs(45, 56, 56, 64, 4, 3, 56, 56, "f16", ("normal", 0, 1.5), ("normal", 0, 0.5), seed=45)
+    out = dcn.forward_host(x.pin_memory(), om.pin_memory(), G=4, K=3, pad=1, device=cuda_device)
+    ref = dcn.forward(x.to(cuda_device), om.to(cuda_device), G=4, K=3, pad=1).cpu()
+    assert torch.equal(out, ref)
+
+
+@pytest.mark.parametrize("chunks", [None, "5"])
+def test_host_path_results_larger_than_records_equal_device_path(chunks, cuda_device, monkeypatch):
+    # C = 256 channels in 4 groups: a result pixel (512 B) outweighs its records (216 B), so each
+    # chunk carries its own x and offset_mask
+    if chunks is not None:
+        monkeypatch.setenv("DCNV4_HOST_CHUNKS", chunks)
+    x, om = make_inputs(13, 40, 40, 256, 4, 3, 40, 40, "f16", ("normal", 0, 1.5), ("normal", 0, 0.5), seed=13)
+    out = dcn.forward_host(x.pin_memory(), om.pin_memory(), G=4, K=3, pad=1, device=cuda_device)
+    ref = dcn.forward(x.to(cuda_device), om.to(cuda_device), G=4, K=3, pad=1).cpu()
+    assert torch.equal(out, ref)
+
+
 def test_host_path_full_workload_against_oracle(cuda_device):
     w = WORKLOADS["stage1_f16"]
     x, om = workload_inputs(w)
