@@ -210,7 +210,7 @@ FwdParams make_params(int N, int H, int W, int C, int G, int K, int stride, int 
     FwdParams p{};
     p.N = N; p.H = H; p.W = W; p.C = C; p.G = G; p.K = K; p.KK = K * K; p.Cg = C / G;
     p.stride = stride; p.pad = pad; p.dilation = dilation;
-    p.Hout = Hout; p.Wout = Wout;
+    p.Hout = Hout; p.Wout = Wout; p.row0 = 0;
     p.units = N * Hout * Wout * G;
     p.offset_scale = offset_scale;
     p.flags = static_cast<int>(flags);
@@ -475,6 +475,39 @@ int dcnv4_predictor(const void* y, const void* weight, const float* bias, void* 
     }
 }
 
+namespace {
+
+// The forward's plan (dcnv4_forward_plan's fields) for the geometry in p on this device.
+int plan_of(const FwdParams& p, int dtype, int* fields) {
+    const int nsm = sm_count();
+    if (nsm <= 0) return DCNV4_ERR_CUDA;
+    switch (dtype) {
+        case DCNV4_F32: return dcnv4_host::plan_f32(p, nsm, fields);
+        case DCNV4_F16: return dcnv4_host::plan_f16(p, nsm, fields);
+        default: return dcnv4_host::plan_bf16(p, nsm, fields);
+    }
+}
+
+// True when every band of `bands` equal row ranges runs the kernel, window kind and halo of the
+// whole image, which makes its outputs the whole-image launch's bit for bit (the planner takes
+// the halo and window kind from the image geometry; the rest of a plan leaves each sample's
+// arithmetic unchanged). A band whose plan would fall back to another kernel is not used.
+bool bands_match_image(int N, int H, int W, int C, int G, int K, int stride, int pad, int dilation, int Hout,
+                       int Wout, int dtype, int bands) {
+    int whole[DCNV4_PLAN_FIELDS], part[DCNV4_PLAN_FIELDS];
+    if (plan_of(make_params(N, H, W, C, G, K, stride, pad, dilation, 1.0f, Hout, Wout), dtype, whole)) return false;
+    for (int b = 0; b < bands; ++b) {
+        const int rows = static_cast<int>((static_cast<long long>(Hout) * (b + 1)) / bands) -
+                         static_cast<int>((static_cast<long long>(Hout) * b) / bands);
+        if (plan_of(make_params(1, H, W, C, G, K, stride, pad, dilation, 1.0f, rows, Wout), dtype, part)) return false;
+        for (int i = 0; i < 3; ++i)  // kernel, window kind, halo
+            if (part[i] != whole[i]) return false;
+    }
+    return true;
+}
+
+}  // namespace
+
 int dcnv4_forward_host(const void* x_host, const void* offset_mask_host, void* out_host,
                        void* x_dev, void* offset_mask_dev, void* out_dev,
                        int N, int H, int W, int C, int G, int K,
@@ -529,10 +562,13 @@ int dcnv4_forward_host(const void* x_host, const void* offset_mask_host, void* o
     for (int i = 0; i < 3; ++i)
         if (cudaStreamWaitEvent(pipe->s[i], ev_start, 0) != cudaSuccess) return fail(DCNV4_ERR_CUDA);
 
-    // Chunks of whole images, about 8 MiB of input copies each, 2 to 8 of them: every copy costs
-    // the copy engine a few microseconds beyond its bytes (measured ~3.7 us on PCIe 5), while the
-    // last chunk's kernel and copy out are the part of the call that nothing overlaps, so neither
-    // many small chunks nor one large one. DCNV4_HOST_CHUNKS sets the count (tuning runs).
+    // Chunks of about 8 MiB of input copies each, 2 to 8 of them: every copy costs the copy
+    // engine a few microseconds beyond its bytes (measured ~3.7 us on PCIe 5), while the last
+    // chunk's kernel and copy out are the part of the call that nothing overlaps, so neither many
+    // small chunks nor one large one. DCNV4_HOST_CHUNKS sets the count (tuning runs). A chunk is
+    // whole images; with fewer images than chunks each image is cut into bands of output rows
+    // instead, each band a launch over its rows of the whole image (FwdParams::row0), so that the
+    // last launch and copy out stay short for a batch of a few large images.
     // When a result is no larger than an image's offset_mask records, x goes over first in one
     // copy and only the records are chunked: one copy less per chunk, and the results' copies
     // out still have the records' transfer time to overlap with (with larger results they would
@@ -540,8 +576,12 @@ int dcnv4_forward_host(const void* x_host, const void* offset_mask_host, void* o
     const size_t in_bytes = static_cast<size_t>(N) * (x_img + om_img);
     int chunks = static_cast<int>(std::min<size_t>(8, std::max<size_t>(2, in_bytes >> 23)));
     if (const char* c = std::getenv("DCNV4_HOST_CHUNKS")) chunks = std::max(1, std::atoi(c));
-    if (chunks > N) chunks = N;
+    int bands = chunks > N ? std::min(Hout, (chunks + N - 1) / N) : 1;  // pieces per image
+    if (bands > 1 && !bands_match_image(N, H, W, C, G, K, stride, pad, dilation, Hout, Wout, dtype, bands))
+        bands = 1;
+    const int pieces = bands > 1 ? N * bands : std::min(chunks, N);
     const bool x_first = out_img <= om_img;
+    const size_t om_row = om_img / Hout, out_row = out_img / Hout;  // bytes per output row
     const char* xh = static_cast<const char*>(x_host);
     const char* omh = static_cast<const char*>(offset_mask_host);
     char* oh = static_cast<char*>(out_host);
@@ -554,27 +594,42 @@ int dcnv4_forward_host(const void* x_host, const void* offset_mask_host, void* o
         if (cudaMemcpyAsync(xd, xh, N * x_img, cudaMemcpyHostToDevice, s_in) != cudaSuccess)
             return fail(DCNV4_ERR_CUDA);
     }
-    int n0 = 0;
-    for (int c = 0; c < chunks; ++c) {
-        const int n1 = static_cast<int>((static_cast<long long>(N) * (c + 1)) / chunks);
+    for (int c = 0; c < pieces; ++c) {
+        // piece c: images [n0, n1), output rows [r0, r1) of each (all rows unless cut into bands)
+        int n0, n1, r0 = 0, r1 = Hout;
+        if (bands > 1) {
+            n0 = c / bands;
+            n1 = n0 + 1;
+            const int b = c - n0 * bands;
+            r0 = static_cast<int>((static_cast<long long>(Hout) * b) / bands);
+            r1 = static_cast<int>((static_cast<long long>(Hout) * (b + 1)) / bands);
+        } else {
+            n0 = static_cast<int>((static_cast<long long>(N) * c) / pieces);
+            n1 = static_cast<int>((static_cast<long long>(N) * (c + 1)) / pieces);
+        }
         const int nc = n1 - n0;
-        if (nc == 0) continue;
+        if (nc == 0 || r1 == r0) continue;
         queued = true;
-        if ((!x_first &&
+        const size_t om_off = n0 * om_img + r0 * om_row, om_len = bands > 1 ? (r1 - r0) * om_row : nc * om_img;
+        const size_t out_off = n0 * out_img + r0 * out_row, out_len = bands > 1 ? (r1 - r0) * out_row : nc * out_img;
+        if ((!x_first && r0 == 0 &&
              cudaMemcpyAsync(xd + n0 * x_img, xh + n0 * x_img, nc * x_img, cudaMemcpyHostToDevice, s_in) !=
                  cudaSuccess) ||
-            cudaMemcpyAsync(omd + n0 * om_img, omh + n0 * om_img, nc * om_img, cudaMemcpyHostToDevice, s_in) !=
-                cudaSuccess ||
+            cudaMemcpyAsync(omd + om_off, omh + om_off, om_len, cudaMemcpyHostToDevice, s_in) != cudaSuccess ||
             cudaEventRecord(ev_in, s_in) != cudaSuccess || cudaStreamWaitEvent(s_k, ev_in, 0) != cudaSuccess)
             return fail(DCNV4_ERR_CUDA);
-        rc = dcnv4_forward(xd + n0 * x_img, omd + n0 * om_img, od + n0 * out_img, nc, H, W, C, G, K, stride, pad,
-                           dilation, offset_scale, dtype, s_k);
+        if (bands > 1) {
+            FwdParams p = make_params(1, H, W, C, G, K, stride, pad, dilation, offset_scale, r1 - r0, Wout);
+            p.row0 = r0;
+            rc = run_forward(xd + n0 * x_img, omd + om_off, od + out_off, p, dtype, nullptr, s_k);
+        } else {
+            rc = dcnv4_forward(xd + n0 * x_img, omd + om_off, od + out_off, nc, H, W, C, G, K, stride, pad, dilation,
+                               offset_scale, dtype, s_k);
+        }
         if (rc) return fail(rc);
         if (cudaEventRecord(ev_k, s_k) != cudaSuccess || cudaStreamWaitEvent(s_out, ev_k, 0) != cudaSuccess ||
-            cudaMemcpyAsync(oh + n0 * out_img, od + n0 * out_img, nc * out_img, cudaMemcpyDeviceToHost, s_out) !=
-                cudaSuccess)
+            cudaMemcpyAsync(oh + out_off, od + out_off, out_len, cudaMemcpyDeviceToHost, s_out) != cudaSuccess)
             return fail(DCNV4_ERR_CUDA);
-        n0 = n1;
     }
     return fail(DCNV4_OK);
 }

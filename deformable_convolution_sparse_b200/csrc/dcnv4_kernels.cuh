@@ -33,7 +33,11 @@ constexpr int kFlagCenterScale = 4;   // blend with the centre feature through a
 struct FwdParams {
     int N, H, W, C, G, K, KK, Cg;   // KK = K*K grid points
     int stride, pad, dilation;
-    int Hout, Wout;
+    int Hout, Wout;     // output rows and columns of this launch (rows: of a band when row0 > 0)
+    int row0;           // forward kernels: image row index of the launch's first output row, so that a
+                        // launch can cover a band [row0, row0 + Hout) of each image's output rows (the
+                        // offset_mask and out pointers then start at the band); 0 for whole images and
+                        // for every other kernel
     int units;          // N * Hout * Wout * G
     int lanes;          // threads per unit
     int chunks;         // channel chunks per unit (a chunk is what one thread covers per pass)
@@ -285,7 +289,7 @@ fwd_vector_kernel(const T* __restrict__ x, const T* __restrict__ om, T* __restri
             if (k == kcs) continue;
             const int jp = k - (k > kcs ? 1 : 0);  // point index in the record
             const int ky = k / K, kx = k - (k / K) * K;
-            const int p0y = ho * p.stride - p.pad + ky * p.dilation;
+            const int p0y = (ho + p.row0) * p.stride - p.pad + ky * p.dilation;
             const int p0x = wo * p.stride - p.pad + kx * p.dilation;
             const float rx = ElemTraits<T>::to_float(rec[jp]);
             const float ry = ElemTraits<T>::to_float(rec[NP + jp]);
@@ -337,7 +341,7 @@ fwd_vector_kernel(const T* __restrict__ x, const T* __restrict__ om, T* __restri
         if (VF && (p.flags & kFlagCenterScale)) {
             // out = (1 - s) * aggregate + s * x at the centre grid position (zero outside)
             const float sg = center_gate<T>(p, static_cast<size_t>(unit));
-            const int cy = ho * p.stride - p.pad + (K / 2) * p.dilation;
+            const int cy = (ho + p.row0) * p.stride - p.pad + (K / 2) * p.dilation;
             const int cx = wo * p.stride - p.pad + (K / 2) * p.dilation;
             uint32_t cw[NW];
 #pragma unroll
@@ -416,7 +420,7 @@ fwd_scalar_kernel(const T* __restrict__ x, const T* __restrict__ om, T* __restri
             if (k == kcs) continue;
             const int jp = k - (k > kcs ? 1 : 0);  // point index in the record
             const int ky = k / K, kx = k - (k / K) * K;
-            const int p0y = ho * p.stride - p.pad + ky * p.dilation;
+            const int p0y = (ho + p.row0) * p.stride - p.pad + ky * p.dilation;
             const int p0x = wo * p.stride - p.pad + kx * p.dilation;
             const float rx = ElemTraits<T>::to_float(rec[jp]);
             const float ry = ElemTraits<T>::to_float(rec[NP + jp]);
@@ -432,7 +436,7 @@ fwd_scalar_kernel(const T* __restrict__ x, const T* __restrict__ om, T* __restri
         }
         if (VF && (p.flags & kFlagCenterScale)) {
             const float sg = center_gate<T>(p, static_cast<size_t>(unit));
-            const int cy = ho * p.stride - p.pad + (K / 2) * p.dilation;
+            const int cy = (ho + p.row0) * p.stride - p.pad + (K / 2) * p.dilation;
             const int cx = wo * p.stride - p.pad + (K / 2) * p.dilation;
             const float xc = (cy >= 0 && cy < p.H && cx >= 0 && cx < p.W)
                                  ? ElemTraits<T>::to_float(ximg[(cy * p.W + cx) * p.C + g * p.Cg + c]) : 0.f;
@@ -462,7 +466,7 @@ sampling_index_kernel(const T* __restrict__ om, int32_t* __restrict__ corner, ui
         unit_coords(unit, p, n, ho, wo, g);
         const T* rec = om + static_cast<size_t>(unit) * 3 * KK;
         const int ky = k / p.K, kx = k - (k / p.K) * p.K;
-        const int p0y = ho * p.stride - p.pad + ky * p.dilation;
+        const int p0y = (ho + p.row0) * p.stride - p.pad + ky * p.dilation;
         const int p0x = wo * p.stride - p.pad + kx * p.dilation;
         const Sample s = locate(p0y, p0x, ElemTraits<T>::to_float(rec[KK + k]), ElemTraits<T>::to_float(rec[k]),
                                 p.offset_scale, p.H, p.W);
@@ -488,9 +492,9 @@ trace_index_kernel(const T* __restrict__ om, int4* __restrict__ trace, FwdParams
         unit_coords(unit, p, n, ho, wo, g);
         const T* rec = om + static_cast<size_t>(unit) * 3 * KK;
         const int ky = k / p.K, kx = k - (k / p.K) * p.K;
-        const Sample s = locate(ho * p.stride - p.pad + ky * p.dilation, wo * p.stride - p.pad + kx * p.dilation,
-                                ElemTraits<T>::to_float(rec[KK + k]), ElemTraits<T>::to_float(rec[k]),
-                                p.offset_scale, p.H, p.W);
+        const Sample s = locate((ho + p.row0) * p.stride - p.pad + ky * p.dilation,
+                                wo * p.stride - p.pad + kx * p.dilation, ElemTraits<T>::to_float(rec[KK + k]),
+                                ElemTraits<T>::to_float(rec[k]), p.offset_scale, p.H, p.W);
         trace[i] = make_int4(s.bits ? s.y0 : INT32_MIN, s.bits ? s.x0 : INT32_MIN, static_cast<int>(s.bits), 2);
     }
 }

@@ -253,16 +253,19 @@ RingShape choose_ring_shape(const FwdParams& f, int nsm) {
     // estimated time, with 5 % added per pixel below target + 1 and 10 % more
     // below the target, for the samples a smaller window sends to the global
     // pass (the offsets' spread is not known here). Smaller halos only when
-    // nothing in that range fits. Judged for a nominal batch of 64 images on
-    // 148 SMs, so that it depends on the geometry alone and an image's result
-    // does not depend on N.
+    // nothing in that range fits. Judged for a nominal batch of 64 whole images
+    // on 148 SMs, so that it depends on the image geometry alone: an image's
+    // result depends neither on N nor on the band of output rows a launch
+    // covers (row0, Hout).
     const int Rt = target_halo(f.dilation);
     int Rhi = Rt + 1, Rlo = std::max(1, Rt - 1);
     const int force_halo = env_int("DCNV4_HALO", 0);
     if (force_halo > 0) Rhi = Rlo = force_halo;
-    const int min_units = std::min(256, f.Hout * f.Wout * f.G);
     FwdParams nominal = f;
     nominal.N = 64;
+    nominal.row0 = 0;
+    nominal.Hout = (f.H + 2 * f.pad - f.dilation * (f.K - 1) - 1) / f.stride + 1;  // the whole image's rows
+    const int min_units = std::min(256, nominal.Hout * f.Wout * f.G);
     int R = -1;
     double best_t = 0.0;
     for (int r = Rhi; r >= Rlo; --r) {
@@ -282,14 +285,18 @@ RingShape choose_ring_shape(const FwdParams& f, int nsm) {
     const bool force_unit = force_halo > 0 || (wenv && std::strcmp(wenv, "unit") == 0);
     const bool force_img = !force_unit && wenv && std::strcmp(wenv, "image") == 0;
     bool img = false;
-    if (!force_unit && image_window_fits(f)) {
+    if (!force_unit && image_window_fits(nominal)) {
         const RingShape c = best_ring_shape<T>(nominal, 0, 148, min_units, true);
         img = c.score > 0.0 && (force_img || R < 0 || 1.0 / c.score <= best_t);
     }
     RingShape none{};
     none.score = -1.0;
     if (R < 0 && !img) return none;
-    return best_ring_shape<T>(f, img ? 0 : R, nsm, min_units, img);
+    RingShape sh = best_ring_shape<T>(f, img ? 0 : R, nsm, std::min(256, f.Hout * f.Wout * f.G), img);
+    // a band of a few output rows may hold no item of 256 units in the group subsets whose
+    // windows fit: then any item size, with the window kind and halo of the whole image
+    if (sh.score <= 0.0 && f.Hout < nominal.Hout) sh = best_ring_shape<T>(f, img ? 0 : R, nsm, 1, img);
+    return sh;
 }
 
 // choose_ring_shape costs 15-25 us of host time (a few thousand candidate

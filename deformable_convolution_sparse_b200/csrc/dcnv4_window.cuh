@@ -356,7 +356,7 @@ __device__ __forceinline__ void issue_rows(const RingParams& p, const CUtensorMa
                                            unsigned char* ring, uint64_t* bar, int lane) {
     const FwdParams& f = p.f;
     // image row and column of the window's first row and column
-    const int img_top = p.img ? -1 : it.ho0 * f.stride - f.pad - p.R;
+    const int img_top = p.img ? -1 : (it.ho0 + f.row0) * f.stride - f.pad - p.R;
     const int img_left = p.img ? -1 : it.wo0 * f.stride - f.pad - p.R;
     const int first = img_top + (it.lv - it.v);
     const unsigned box = static_cast<unsigned>(p.WW * p.PB);  // bytes of one row load
@@ -548,7 +548,7 @@ fwd_ring_kernel(const __grid_constant__ CUtensorMap xmap, const T* __restrict__ 
             unsigned rb0 = static_cast<unsigned>(img ? it.p0 : it.p0 + py * f.stride);
             rb0 = min(rb0, rb0 - NR);
             const unsigned rowoff = rb0 * rowBu;
-            const int by = ho * f.stride - f.pad;  // grid row of ky = 0 (image coordinates)
+            const int by = (ho + f.row0) * f.stride - f.pad;  // grid row of ky = 0 (image coordinates)
             const int bx = wo * f.stride - f.pad;
             // window row / column of the grid point (0, 0): R in a unit window, which is
             // centred on the unit; in an image window (first row and column: image row and

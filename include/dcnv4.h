@@ -306,8 +306,10 @@ DCNV4_API int dcnv4_forward_trace(const void *x, const void *offset_mask, void *
  * result. x_dev, offset_mask_dev, out_dev: caller-owned device buffers of the
  * full sizes of x, offset_mask and out, used as staging (their contents
  * afterwards: the copied inputs and the result). The batch is split into
- * chunks of whole images (about 8 MiB of input copies each, 2 to 8 of them)
- * and the work is queued on three library-owned non-blocking streams
+ * chunks of whole images (about 8 MiB of input copies each, 2 to 8 of them;
+ * a batch of fewer images than that is cut into bands of output rows, each
+ * band one launch over its rows of the whole image, with the same result bit
+ * for bit) and the work is queued on three library-owned non-blocking streams
  * (created once per device on first use and kept until exit), one per role:
  * the host-to-device copies back to back on the first (all of x in one copy
  * ahead of the chunks' offset_mask copies when an image's result is no

@@ -47,6 +47,34 @@ def test_host_path_results_larger_than_records_equal_device_path(chunks, cuda_de
     assert torch.equal(out, ref)
 
 
+# Fewer images than chunks: each image is cut into bands of output rows, one launch per band over
+# the whole image (unit windows, image windows, the global-gather kernel, stride 2, dilation 2,
+# one-row bands, bands too short for the whole image's item size)
+BAND_CASES = [
+    # N, H, W, C, G, K, stride, pad, dilation, dtype, chunks
+    (2, 64, 64, 128, 8, 3, 1, 2, 2, "bf16", "8"),
+    (1, 56, 56, 64, 4, 3, 1, 1, 1, "f16", "5"),
+    (1, 14, 14, 256, 16, 3, 1, 1, 1, "f16", "3"),
+    (1, 20, 20, 48, 2, 3, 1, 1, 1, "f16", "4"),
+    (3, 33, 29, 64, 4, 3, 2, 1, 1, "f32", "7"),
+    (1, 9, 9, 32, 2, 3, 1, 1, 1, "f32", "64"),
+    (2, 32, 32, 256, 4, 3, 1, 1, 1, "f16", "6"),  # results larger than records: x with each first band
+]
+
+
+@pytest.mark.parametrize("case", BAND_CASES)
+def test_host_path_row_bands_equal_device_path(case, cuda_device, monkeypatch):
+    N, H, W, C, G, K, s, pad, d, dtype, chunks = case
+    monkeypatch.setenv("DCNV4_HOST_CHUNKS", chunks)
+    Ho = (H + 2 * pad - d * (K - 1) - 1) // s + 1
+    Wo = (W + 2 * pad - d * (K - 1) - 1) // s + 1
+    x, om = make_inputs(N, H, W, C, G, K, Ho, Wo, dtype, ("normal", 0, 2.0), ("normal", 0, 0.5), seed=H + N)
+    kw = dict(G=G, K=K, stride=s, pad=pad, dilation=d)
+    out = dcn.forward_host(x.pin_memory(), om.pin_memory(), device=cuda_device, **kw)
+    ref = dcn.forward(x.to(cuda_device), om.to(cuda_device), **kw).cpu()
+    assert torch.equal(out, ref)
+
+
 def test_host_path_full_workload_against_oracle(cuda_device):
     w = WORKLOADS["stage1_f16"]
     x, om = workload_inputs(w)
