@@ -920,7 +920,9 @@ def run_forward(args, w, dev, world, rank, barrier, max_over_ranks):
                     "steps": args.e2e_steps,
                     "h2d_bytes_per_step": (x.numel() + om.numel()) * x.element_size(),
                     "d2h_bytes_per_step": oh.numel() * oh.element_size(),
-                    "path": "dcnv4_forward_host: pinned host buffers, chunked H2D/kernel/D2H on three streams"},
+                    "path": "dcnv4_forward_host: pinned host buffers; copies in, kernels and copies out on "
+                            "one stream each, over chunks of images (bands of output rows when the batch "
+                            "has fewer images than chunks)"},
             "gpu_launches": timed_launches,
             "clocks": clocks,
             "cpu_baseline": base,

@@ -1,6 +1,11 @@
 """GPU tests of dcnv4_forward_host: inputs and result in host memory, the
 device buffers only as staging, the copies and kernels pipelined over image
 chunks. The result must equal the device-resident forward bit for bit."""
+import os
+import re
+import subprocess
+import sys
+
 import numpy as np
 import pytest
 import torch
@@ -73,6 +78,38 @@ def test_host_path_row_bands_equal_device_path(case, cuda_device, monkeypatch):
     out = dcn.forward_host(x.pin_memory(), om.pin_memory(), device=cuda_device, **kw)
     ref = dcn.forward(x.to(cuda_device), om.to(cuda_device), **kw).cpu()
     assert torch.equal(out, ref)
+
+
+def test_host_path_row_bands_from_pageable_memory(cuda_device, monkeypatch):
+    # pageable host buffers: the copies block the calling thread, the bands and their order stay
+    monkeypatch.setenv("DCNV4_HOST_CHUNKS", "6")
+    x, om = make_inputs(2, 40, 40, 64, 4, 3, 40, 40, "f16", ("normal", 0, 2.0), ("normal", 0, 0.5), seed=9)
+    out = dcn.forward_host(x, om, G=4, K=3, pad=1, device=cuda_device)
+    ref = dcn.forward(x.to(cuda_device), om.to(cuda_device), G=4, K=3, pad=1).cpu()
+    assert torch.equal(out, ref)
+
+
+_BANDS_RUN = r"""
+import sys, torch
+sys.path.insert(0, sys.argv[1])
+import deformable_convolution_sparse_b200 as dcn
+from deformable_convolution_sparse_b200.workloads import make_inputs
+x, om = make_inputs(2, 64, 64, 128, 8, 3, 62, 62, "bf16", ("normal", 0, 2.0), ("normal", 0, 0.5), seed=5)
+dcn.forward_host(x.pin_memory(), om.pin_memory(), G=8, K=3, pad=1, dilation=2, device=torch.device("cuda:0"))
+torch.cuda.synchronize()
+"""
+
+
+def test_host_path_launches_one_plan_per_band(cuda_device):
+    # two images in eight chunks: four bands of 15-16 output rows per image, each its own launch
+    # (DCNV4_DEBUG=1 prints the ring plan of every launch); the whole-image schedule would make two
+    env = dict(os.environ, DCNV4_DEBUG="1", DCNV4_HOST_CHUNKS="8")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    res = subprocess.run([sys.executable, "-c", _BANDS_RUN, root], capture_output=True, text=True, timeout=300,
+                         env=env)
+    assert res.returncode == 0, res.stderr[-2000:]
+    plans = re.findall(r"dcnv4 ring plan: .* rows_total (\d+)", res.stderr)
+    assert len(plans) == 8, res.stderr[-2000:]
 
 
 def test_host_path_full_workload_against_oracle(cuda_device):
