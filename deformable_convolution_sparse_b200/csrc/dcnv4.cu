@@ -7,6 +7,7 @@
 #include <cmath>
 #include <cstdint>
 #include <algorithm>
+#include <array>
 #include <cmath>
 #include <map>
 #include <mutex>
@@ -492,18 +493,37 @@ int plan_of(const FwdParams& p, int dtype, int* fields) {
 // whole image, which makes its outputs the whole-image launch's bit for bit (the planner takes
 // the halo and window kind from the image geometry; the rest of a plan leaves each sample's
 // arithmetic unchanged). A band whose plan would fall back to another kernel is not used.
+// Kept per geometry, band count, storage type and device: a few plan look-ups (string keys
+// built from the planner's environment switches) would otherwise cost tens of microseconds of
+// host time on every call.
 bool bands_match_image(int N, int H, int W, int C, int G, int K, int stride, int pad, int dilation, int Hout,
                        int Wout, int dtype, int bands) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    static std::mutex mu;
+    static std::map<std::array<int, 12>, bool> cache;
+    const std::array<int, 12> key = {N, H, W, C, G, K, stride, pad, dilation, dtype, bands, dev};
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        if (auto it = cache.find(key); it != cache.end()) return it->second;
+    }
+    bool match = true;
     int whole[DCNV4_PLAN_FIELDS], part[DCNV4_PLAN_FIELDS];
-    if (plan_of(make_params(N, H, W, C, G, K, stride, pad, dilation, 1.0f, Hout, Wout), dtype, whole)) return false;
-    for (int b = 0; b < bands; ++b) {
+    if (plan_of(make_params(N, H, W, C, G, K, stride, pad, dilation, 1.0f, Hout, Wout), dtype, whole)) match = false;
+    for (int b = 0; b < bands && match; ++b) {
         const int rows = static_cast<int>((static_cast<long long>(Hout) * (b + 1)) / bands) -
                          static_cast<int>((static_cast<long long>(Hout) * b) / bands);
-        if (plan_of(make_params(1, H, W, C, G, K, stride, pad, dilation, 1.0f, rows, Wout), dtype, part)) return false;
+        if (plan_of(make_params(1, H, W, C, G, K, stride, pad, dilation, 1.0f, rows, Wout), dtype, part)) {
+            match = false;
+            break;
+        }
         for (int i = 0; i < 3; ++i)  // kernel, window kind, halo
-            if (part[i] != whole[i]) return false;
+            if (part[i] != whole[i]) match = false;
     }
-    return true;
+    std::lock_guard<std::mutex> lock(mu);
+    if (cache.size() >= 256) cache.clear();
+    cache.emplace(key, match);
+    return match;
 }
 
 }  // namespace
@@ -576,12 +596,7 @@ int dcnv4_forward_host(const void* x_host, const void* offset_mask_host, void* o
     const size_t in_bytes = static_cast<size_t>(N) * (x_img + om_img);
     int chunks = static_cast<int>(std::min<size_t>(8, std::max<size_t>(2, in_bytes >> 23)));
     if (const char* c = std::getenv("DCNV4_HOST_CHUNKS")) chunks = std::max(1, std::atoi(c));
-    int bands = chunks > N ? std::min(Hout, (chunks + N - 1) / N) : 1;  // pieces per image
-    if (bands > 1 && !bands_match_image(N, H, W, C, G, K, stride, pad, dilation, Hout, Wout, dtype, bands))
-        bands = 1;
-    const int pieces = bands > 1 ? N * bands : std::min(chunks, N);
     const bool x_first = out_img <= om_img;
-    const size_t om_row = om_img / Hout, out_row = out_img / Hout;  // bytes per output row
     const char* xh = static_cast<const char*>(x_host);
     const char* omh = static_cast<const char*>(offset_mask_host);
     char* oh = static_cast<char*>(out_host);
@@ -589,11 +604,16 @@ int dcnv4_forward_host(const void* x_host, const void* offset_mask_host, void* o
     char* omd = static_cast<char*>(offset_mask_dev);
     char* od = static_cast<char*>(out_dev);
     cudaStream_t s_in = pipe->s[0], s_k = pipe->s[1], s_out = pipe->s[2];
-    if (x_first) {
+    if (x_first) {  // queued first, so the copy runs while the pieces are worked out
         queued = true;
         if (cudaMemcpyAsync(xd, xh, N * x_img, cudaMemcpyHostToDevice, s_in) != cudaSuccess)
             return fail(DCNV4_ERR_CUDA);
     }
+    int bands = chunks > N ? std::min(Hout, (chunks + N - 1) / N) : 1;  // pieces per image
+    if (bands > 1 && !bands_match_image(N, H, W, C, G, K, stride, pad, dilation, Hout, Wout, dtype, bands))
+        bands = 1;
+    const int pieces = bands > 1 ? N * bands : std::min(chunks, N);
+    const size_t om_row = om_img / Hout, out_row = out_img / Hout;  // bytes per output row
     for (int c = 0; c < pieces; ++c) {
         // piece c: images [n0, n1), output rows [r0, r1) of each (all rows unless cut into bands)
         int n0, n1, r0 = 0, r1 = Hout;
