@@ -64,6 +64,7 @@ BAND_CASES = [
     (3, 33, 29, 64, 4, 3, 2, 1, 1, "f32", "7"),
     (1, 9, 9, 32, 2, 3, 1, 1, 1, "f32", "64"),
     (2, 32, 32, 256, 4, 3, 1, 1, 1, "f16", "6"),  # results larger than records: x with each first band
+    (1, 9, 9, 32, 1, 3, 1, 1, 1, "f16", "3"),  # a band's records start 2-byte aligned (486-byte rows)
 ]
 
 
