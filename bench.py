@@ -19,6 +19,12 @@ bracketed by a barrier and a device synchronise; the time is the max over
 ranks. The steps rotate over several resident copies of the inputs whose total
 exceeds the L2 cache, so no step starts with its inputs in L2.
 
+End to end (`e2e`): the same metric through dcnv4_forward_host, from pinned
+host buffers to a host result, the host-to-device and device-to-host copies
+inside the timed region (the library overlaps them with the kernels over
+chunks of images, or bands of output rows for a batch of a few images);
+the line states the bytes copied each way per step.
+
 --impl reference times the fp64 CPU oracle (the reference arm of this
 repository: there is no other implementation to install) on the host cores,
 for the same workloads, metric and unit.
