@@ -495,15 +495,19 @@ int plan_of(const FwdParams& p, int dtype, int* fields) {
 // arithmetic unchanged). A band whose plan would fall back to another kernel is not used.
 // Kept per geometry, band count, storage type and device: a few plan look-ups (string keys
 // built from the planner's environment switches) would otherwise cost tens of microseconds of
-// host time on every call.
+// host time on every call. Not kept while a planner override is set (tuning runs may change it
+// between calls).
 bool bands_match_image(int N, int H, int W, int C, int G, int K, int stride, int pad, int dilation, int Hout,
                        int Wout, int dtype, int bands) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return false;
     static std::mutex mu;
     static std::map<std::array<int, 12>, bool> cache;
+    bool keep = true;
+    for (const char* e : {"DCNV4_HALO", "DCNV4_WINDOW", "DCNV4_TILE", "DCNV4_GS", "DCNV4_NREC", "DCNV4_RING"})
+        if (std::getenv(e)) keep = false;
     const std::array<int, 12> key = {N, H, W, C, G, K, stride, pad, dilation, dtype, bands, dev};
-    {
+    if (keep) {
         std::lock_guard<std::mutex> lock(mu);
         if (auto it = cache.find(key); it != cache.end()) return it->second;
     }
@@ -520,9 +524,11 @@ bool bands_match_image(int N, int H, int W, int C, int G, int K, int stride, int
         for (int i = 0; i < 3; ++i)  // kernel, window kind, halo
             if (part[i] != whole[i]) match = false;
     }
-    std::lock_guard<std::mutex> lock(mu);
-    if (cache.size() >= 256) cache.clear();
-    cache.emplace(key, match);
+    if (keep) {
+        std::lock_guard<std::mutex> lock(mu);
+        if (cache.size() >= 256) cache.clear();
+        cache.emplace(key, match);
+    }
     return match;
 }
 

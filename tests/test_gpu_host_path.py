@@ -81,6 +81,17 @@ def test_host_path_row_bands_equal_device_path(case, cuda_device, monkeypatch):
     assert torch.equal(out, ref)
 
 
+def test_host_path_planner_override_keeps_the_device_result(cuda_device, monkeypatch):
+    # an item height forced above the bands' row counts leaves the bands without a ring plan of the
+    # image's kind: the host path must then keep whole images (same bits as the device path)
+    monkeypatch.setenv("DCNV4_HOST_CHUNKS", "8")
+    monkeypatch.setenv("DCNV4_TILE", "14x14")
+    x, om = make_inputs(2, 28, 28, 64, 4, 3, 28, 28, "f16", ("normal", 0, 1.5), ("normal", 0, 0.5), seed=11)
+    out = dcn.forward_host(x.pin_memory(), om.pin_memory(), G=4, K=3, pad=1, device=cuda_device)
+    ref = dcn.forward(x.to(cuda_device), om.to(cuda_device), G=4, K=3, pad=1).cpu()
+    assert torch.equal(out, ref)
+
+
 def test_host_path_row_bands_from_pageable_memory(cuda_device, monkeypatch):
     # pageable host buffers: the copies block the calling thread, the bands and their order stay
     monkeypatch.setenv("DCNV4_HOST_CHUNKS", "6")
