@@ -415,8 +415,16 @@ def time_steps(step, launches, args, dev, stream, barrier, max_over_ranks):
         step(i)
     ev1.record(stream)
     torch.cuda.synchronize(dev)
+    # a kernel that gave up on a bounded wait sets a bit of the device status word and returns
+    # early: such a run measured unfinished work and is not reported
+    # (every rank reads its own word; all of them stop if any rank's is set)
+    import deformable_convolution_sparse_b200 as dcn
+    status = dcn.device_status(clear=False)
     barrier()
     sampler.stop()
+    if max_over_ranks(float(status)) != 0.0:
+        raise SystemExit(f"device status word 0x{status:x} after the timed steps (max over ranks non-zero): "
+                         "a kernel gave up a bounded wait")
     return max_over_ranks(ev0.elapsed_time(ev1)), sampler, launches[0]
 
 
