@@ -43,7 +43,10 @@
  *   - Every call is thread-safe; the library keeps no pointer to caller
  *     memory after return and allocates no device memory (the probes below
  *     excepted). It caches, in host memory and per geometry, storage type
- *     and SM count, the forward's choice of kernel plan.
+ *     and SM count, the forward's choice of kernel plan (and, for the
+ *     host-memory entry points, three streams per device and whether a
+ *     geometry's bands of output rows take the whole image's plan); each
+ *     cache is guarded by its own lock.
  *   - Compute calls are asynchronous on `stream` (a cudaStream_t; NULL is the
  *     legacy default stream) and never synchronise. Arguments are checked on
  *     the host before anything is launched; on a non-zero return nothing was
