@@ -4,6 +4,9 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
     torchrun --nproc-per-node N bench.py --gpus N ...     (one rank per GPU)
 
+(--gpus N > 1 outside torchrun relaunches the same command under torch.distributed.run
+as N ranks of one node.)
+
 A step is one dcnv4_forward call over one batch of a named workload (seeded
 synthetic inputs in the workload's shape and value distributions). Without
 --workload the run prints one JSON line per named workload, in the order
@@ -782,11 +785,26 @@ def run_predictor(args, w, dev, world, rank, barrier, max_over_ranks):
         print(json.dumps(line), flush=True)
 
 
+def relaunch_under_torchrun(n: int) -> int:
+    """`python bench.py --gpus N` (N > 1) outside torchrun: run this same command line as N ranks of
+    one node (rendezvous on 127.0.0.1, a free port) and return their exit status."""
+    import socket
+    import subprocess
+    with socket.socket() as sock:
+        sock.bind(("127.0.0.1", 0))
+        port = sock.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.abspath(__file__), *sys.argv[1:]]
+    return subprocess.call(cmd)
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
         run_reference(args)
         return
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        sys.exit(relaunch_under_torchrun(args.gpus))
 
     import torch
     import torch.distributed as dist
