@@ -133,7 +133,7 @@ struct RingShape {  // one candidate of the planner
 //    SM cycles per sampling point (the measured rate of the 128-byte-pixel
 //    gather), divided by the gather's bank efficiency (1 / wavefronts^2), the
 //    record layout (per-pixel runs measured about 20 % slower than one run per
-//    output row), warp occupancy (below 12 consumer warps, 8 with four or more
+//    output row, except in image-window plans of 8 or more groups), warp occupancy (below 12 consumer warps, 8 with four or more
 //    chunks per group), the filled lanes of
 //    the consumer warps and bands narrower
 //    than half their window (measured slower: (2 TW stride / WW)^(1/4));
@@ -177,7 +177,10 @@ RingShape best_ring_shape(const FwdParams& f, int R, int nsm, int min_units, boo
         const double w = gather_wavefronts(Q, GS);
         const double banks = 1.0 / (w * w);
         const bool row_runs = GS == f.G;
-        const double runs = row_runs ? 1.0 : 0.8;
+        // per-pixel record runs: 20 % slower in unit-window plans; image-window plans of 8 or more
+        // groups per strip measured as fast as the row-run plan or faster (stage-3 shape: 8 groups
+        // in 4-row items 17.2 us against 18.4 for all 16 groups in 2-row items)
+        const double runs = (row_runs || (img && GS >= 8)) ? 1.0 : 0.8;
         for (int TW : TWs) {
             if (img) {
                 if (TW != TWs[0]) break;
