@@ -120,6 +120,7 @@ struct RingShape {  // one candidate of the planner
     int GS, R, TW, TH, nrec, NR, units, threads, slot, rec, WW, UH, UW, c2, img;
     size_t smem;
     double score;
+    double row_us, strip_us;  // estimated time of one output row (band x groups) and of a strip's window load
 };
 
 // The best plan for halo R, or with image windows when `img` (score < 0: none
@@ -238,7 +239,8 @@ RingShape best_ring_shape(const FwdParams& f, int R, int nsm, int min_units, boo
                     const double score = 1.0 / (t_compute + t_start + t_wait + t_depth);
                     if (score > best.score) {
                         best = RingShape{GS, R, TW, TH, nrec, NR, units, threads, slot, rec, WW, UH, UW, c2, img ? 1 : 0,
-                                         smem, score};
+                                         smem, score, TW * GS * f.npts * cpp / clk,
+                                         1.0 + static_cast<double>(nrows) * rowB / (100.0 * clk)};
                     }
                 }
             }
@@ -357,6 +359,20 @@ bool plan_ring(const void* x, const void* om, const void* out, const FwdParams& 
     const long long rows_total = static_cast<long long>(f.N) * bp.bands * bp.nsub * f.Hout;
     if (rows_total >= (1LL << 31)) return false;
     bp.rows_total = static_cast<int>(rows_total);
+    // Entering a strip costs a CTA its window load. When the ring cannot load the next strip's
+    // window during the current strip and most CTAs enter at most two strips, the CTAs that enter
+    // two run ~4 % longer (measured per CTA on the high-resolution shape): the rows are then shared
+    // out by cost, each strip charging twice its estimated window-load time in rows
+    // (DCNV4_STRIP_COST sets the charge for tuning runs).
+    {
+        const int nrows = sh.img ? sh.UH : (sh.TH - 1) * f.stride + sh.UH;
+        const double rows_per_cta = static_cast<double>(rows_total) / nsm;
+        int P = 0;
+        if (sh.NR < 2 * nrows && rows_per_cta <= f.Hout && sh.row_us > 0.0)
+            P = static_cast<int>(std::lround(2.0 * sh.strip_us / sh.row_us));
+        P = env_int("DCNV4_STRIP_COST", P);
+        bp.strip_cost = std::min(std::max(0, P), 1 << 16);
+    }
     bp.units = sh.units;
     bp.run_slot = sh.slot;
     bp.rec_bytes = sh.rec;
@@ -396,9 +412,9 @@ bool plan_ring(const void* x, const void* om, const void* out, const FwdParams& 
     if (const char* d = std::getenv("DCNV4_DEBUG"); d && *d == '1')
         std::fprintf(stderr,
                      "dcnv4 ring plan: %s windows, item %dx%d GS %d (nsub %d) R %d window %dx%d width %d PB %d "
-                     "ring %d rows rows_total %d units %d threads %d nrec %d smem %zu est %.1f us\n",
+                     "ring %d rows rows_total %d units %d threads %d nrec %d smem %zu est %.1f us strip cost %d\n",
                      bp.img ? "image" : "unit", bp.TH, bp.TW, bp.GS, bp.nsub, bp.R, bp.UH, bp.UW, bp.WW, bp.PB, bp.NR,
-                     bp.rows_total, bp.units, sh.threads, bp.nrec, sh.smem, 1.0 / sh.score);
+                     bp.rows_total, bp.units, sh.threads, bp.nrec, sh.smem, 1.0 / sh.score, bp.strip_cost);
     return true;
 }
 

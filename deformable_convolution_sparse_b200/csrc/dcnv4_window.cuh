@@ -65,6 +65,7 @@ struct RingParams {
     int cblk;            // tensor-map channel blocks per group subset
     int bands;           // ceil(Wout / TW)
     int rows_total;      // N * bands * nsub * Hout: the strip-major rows shared out among CTAs
+    int strip_cost;      // rows' worth of time a CTA spends entering a strip (its window load), >= 0
     int units;           // TH * TW * GS
     int run_slot;        // shared bytes per record run (an odd multiple of 16)
     int rec_bytes;       // one record buffer (multiple of 128)
@@ -231,10 +232,25 @@ struct ItemCursor {
     int v, p0, nrows, adv;   // last item's window: virtual row, ring row, rows, advance to a continuation
 };
 
+// First strip-major row of the rows whose cost lies at or after `cost`, where
+// the rows of strip s cost s (Hout + P) + P + (0 .. Hout - 1): every strip
+// charges P rows' worth of time for entering it (its window load) before its
+// rows. Monotonic, 0 at 0 and rows_total at the total cost.
+__device__ __forceinline__ int row_at_cost(long long cost, int Hout, int P) {
+    const long long per = static_cast<long long>(Hout) + P;
+    const long long s = cost / per;
+    const long long r = cost - s * per - P;
+    return static_cast<int>(s * Hout + (r < 0 ? 0 : r));
+}
+
+// A CTA's contiguous range of strip-major rows: an equal share of the rows'
+// total cost, so that a CTA whose range enters more strips gets fewer rows.
 __device__ __forceinline__ ItemCursor item_cursor(const RingParams& p, int cta, int ncta) {
     ItemCursor c;
-    c.g = static_cast<int>((static_cast<long long>(p.rows_total) * cta) / ncta);
-    c.g1 = static_cast<int>((static_cast<long long>(p.rows_total) * (cta + 1)) / ncta);
+    const int Hout = p.f.Hout, P = p.strip_cost;
+    const long long total = static_cast<long long>(p.rows_total / Hout) * (Hout + P);
+    c.g = row_at_cost((total * cta) / ncta, Hout, P);
+    c.g1 = row_at_cost((total * (cta + 1)) / ncta, Hout, P);
     c.strip = -1;
     c.ho_end = -1;
     c.v = 0;
